@@ -1,0 +1,276 @@
+"""CPU oracle for the BitLinear / H-BitLinear forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import this package.  The product library never does: it shares no
+code with the oracle, and its Python binding fails loudly instead of falling back here.
+
+The arithmetic lives in ``bitnet_oracle.c`` (plain loops, double precision, int64
+accumulation); this module compiles it with gcc on first use and wraps it with numpy.  Each
+wrapper names the page and section whose step it states; the readings taken where the pages
+print no formula are listed at the top of the C file.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitnet_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# -ffp-contract=off keeps every product and sum a separately rounded IEEE operation.
+CFLAGS = ["-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off",
+          "-fno-fast-math", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``bitnet_oracle.c`` into ``liboracle.so`` next to it (gcc + OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = build()
+            L = ctypes.CDLL(path)
+            i64, vp, f32, f64, i32 = (ctypes.c_int64, ctypes.c_void_p, ctypes.c_float,
+                                      ctypes.c_double, ctypes.c_int)
+            sig = {
+                "oracle_double_to_bf16": (ctypes.c_uint16, [f64]),
+                "oracle_bf16_to_double": (f64, [ctypes.c_uint16]),
+                "oracle_num_threads": (i32, []),
+                "oracle_abs_sum_bf16": (f64, [vp, i64]),
+                "oracle_absmean_gamma": (f32, [vp, i64]),
+                "oracle_ternarize": (None, [vp, i64, f32, vp]),
+                "oracle_pack_ternary": (None, [vp, i64, i64, vp]),
+                "oracle_unpack_ternary": (i64, [vp, i64, i64, vp]),
+                "oracle_pack_base3": (None, [vp, i64, vp]),
+                "oracle_unpack_base3": (None, [vp, i64, vp]),
+                "oracle_fwht": (None, [vp, i64, i64, vp]),
+                "oracle_quant_act": (None, [vp, i64, i64, i32, vp, vp, vp, vp]),
+                "oracle_pack_int4": (None, [vp, i64, i64, vp]),
+                "oracle_unpack_int4": (None, [vp, i64, i64, vp]),
+                "oracle_gemm_i64": (None, [vp, vp, i64, i64, i64, vp]),
+                "oracle_gemm_addsub": (None, [vp, vp, i64, i64, i64, vp]),
+                "oracle_dequant": (None, [vp, vp, f32, i64, i64, vp]),
+                "oracle_bitlinear_forward": (i32, [vp, i64, i64, vp, i64, i32, i32, vp,
+                                                   vp, vp, vp, vp, vp, vp]),
+            }
+            for name, (res, args) in sig.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+def num_threads() -> int:
+    """Host threads the oracle's OpenMP loops use."""
+    return int(lib().oracle_num_threads())
+
+
+# --------------------------------------------------------------------------------------
+# bf16 helpers (bf16 values are carried as uint16 bit patterns)
+# --------------------------------------------------------------------------------------
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values straight to bf16 (ties to even); returns uint16 bit patterns."""
+    L = lib()
+    flat = np.ascontiguousarray(x, dtype=np.float64).ravel()
+    out = np.fromiter((L.oracle_double_to_bf16(float(v)) for v in flat), dtype=np.uint16,
+                      count=flat.size)
+    return out.reshape(np.shape(x))
+
+
+# --------------------------------------------------------------------------------------
+# Step 1: absmean ternarisation  (b1.58 summary, 方法论 / 方法详解; 2B4T article, 一.2)
+# --------------------------------------------------------------------------------------
+
+def absmean_gamma(w_bf16: np.ndarray) -> np.float32:
+    """gamma = fp32(max(mean|W|, 1e-5)) over the whole tensor."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    return np.float32(lib().oracle_absmean_gamma(_p(w), w.size))
+
+
+def ternarize(w_bf16: np.ndarray, gamma) -> np.ndarray:
+    """q = clip(rint(w / gamma), -1, 1), decided in IEEE fp32.  Returns int8 of W's shape."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    q = np.empty(w.shape, dtype=np.int8)
+    lib().oracle_ternarize(_p(w), w.size, ctypes.c_float(float(gamma)), _p(q))
+    return q
+
+
+def pack_ternary(q: np.ndarray) -> np.ndarray:
+    """2-bit offset codes, interleaved words: [N, K/16] uint32 (see bitnet_oracle.c)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N, K = q.shape
+    out = np.empty((N, K // 16), dtype=np.uint32)
+    lib().oracle_pack_ternary(_p(q), N, K, _p(out))
+    return out
+
+
+def unpack_ternary(wp: np.ndarray, K: int):
+    """Inverse of pack_ternary.  Returns (q int8 [N, K], count of fields holding code 3)."""
+    wp = np.ascontiguousarray(wp, dtype=np.uint32).reshape(-1, K // 16)
+    N = wp.shape[0]
+    q = np.empty((N, K), dtype=np.int8)
+    bad = lib().oracle_unpack_ternary(_p(wp), N, K, _p(q))
+    return q, int(bad)
+
+
+def pack_base3(digits: np.ndarray) -> np.ndarray:
+    """Five base-3 digits per byte, first digit most significant (2B4T article, 一.1)."""
+    d = np.ascontiguousarray(digits, dtype=np.uint8).ravel()
+    out = np.empty((d.size + 4) // 5, dtype=np.uint8)
+    lib().oracle_pack_base3(_p(d), d.size, _p(out))
+    return out
+
+
+def unpack_base3(b: np.ndarray, n: int) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    out = np.empty(n, dtype=np.uint8)
+    lib().oracle_unpack_base3(_p(b), n, _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Step 2: online Hadamard transform  (BitNet v2 write-up, H-BitLinear paragraphs)
+# --------------------------------------------------------------------------------------
+
+def fwht(x: np.ndarray) -> np.ndarray:
+    """z = H_K x / sqrt(K) per row, Sylvester order, in double.  x: [M, K] float64."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if x.ndim == 1:
+        return fwht(x[None, :])[0]
+    M, K = x.shape
+    z = np.empty_like(x)
+    lib().oracle_fwht(_p(x), M, K, _p(z))
+    return z
+
+
+# --------------------------------------------------------------------------------------
+# Step 3: per-token absmax quantisation  (2B4T article, 一.2; BitNet v2 write-up, INT8/INT4)
+# --------------------------------------------------------------------------------------
+
+def quant_act(z_f32: np.ndarray, bits: int):
+    """Per-token absmax codes decided in fp32.
+
+    Returns (codes int8 [M, K], d float32 [M], pre float64 [M, K], rowsum int64 [M]) where
+    ``pre`` is the unrounded z * Q / max|z| in double.
+    """
+    z = np.ascontiguousarray(z_f32, dtype=np.float32)
+    M, K = z.shape
+    codes = np.empty((M, K), dtype=np.int8)
+    d = np.empty(M, dtype=np.float32)
+    pre = np.empty((M, K), dtype=np.float64)
+    rowsum = np.empty(M, dtype=np.int64)
+    lib().oracle_quant_act(_p(z), M, K, int(bits), _p(codes), _p(d), _p(pre), _p(rowsum))
+    return codes, d, pre, rowsum
+
+
+def pack_int4(c: np.ndarray) -> np.ndarray:
+    """Nibble storage of INT4 codes: [M, K/2] uint8 (see bitnet_oracle.c)."""
+    c = np.ascontiguousarray(c, dtype=np.int8)
+    M, K = c.shape
+    out = np.empty((M, K // 2), dtype=np.uint8)
+    lib().oracle_pack_int4(_p(c), M, K, _p(out))
+    return out
+
+
+def unpack_int4(b: np.ndarray, K: int) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8).reshape(-1, K // 2)
+    M = b.shape[0]
+    c = np.empty((M, K), dtype=np.int8)
+    lib().oracle_unpack_int4(_p(b), M, K, _p(c))
+    return c
+
+
+# --------------------------------------------------------------------------------------
+# Step 4: ternary x integer product  (2B4T article, 一.2: +1 adds, -1 subtracts, 0 skips)
+# --------------------------------------------------------------------------------------
+
+def gemm_i64(c: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """acc[m, n] = sum_k c[m, k] q[n, k] in int64."""
+    c = np.ascontiguousarray(c, dtype=np.int8)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    M, K = c.shape
+    N = q.shape[0]
+    acc = np.empty((M, N), dtype=np.int64)
+    lib().oracle_gemm_i64(_p(c), _p(q), M, N, K, _p(acc))
+    return acc
+
+
+def gemm_addsub(c: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """The same product as add / subtract / skip, without multiplications."""
+    c = np.ascontiguousarray(c, dtype=np.int8)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    M, K = c.shape
+    N = q.shape[0]
+    acc = np.empty((M, N), dtype=np.int64)
+    lib().oracle_gemm_addsub(_p(c), _p(q), M, N, K, _p(acc))
+    return acc
+
+
+# --------------------------------------------------------------------------------------
+# Step 5: rescale to bf16
+# --------------------------------------------------------------------------------------
+
+def dequant(acc: np.ndarray, d: np.ndarray, gamma) -> np.ndarray:
+    """Y = bf16_rn(acc * d * gamma) (product in double); returns uint16 bf16 bit patterns."""
+    acc = np.ascontiguousarray(acc, dtype=np.int64)
+    d = np.ascontiguousarray(d, dtype=np.float32)
+    M, N = acc.shape
+    Y = np.empty((M, N), dtype=np.uint16)
+    lib().oracle_dequant(_p(acc), _p(d), ctypes.c_float(float(gamma)), M, N, _p(Y))
+    return Y
+
+
+# --------------------------------------------------------------------------------------
+# The whole forward
+# --------------------------------------------------------------------------------------
+
+def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bits: int):
+    """Y = (H-)BitLinear(X) from bf16 X [M, K] and latent bf16 W [N, K].
+
+    Returns a dict with every stage: gamma, q, z, codes, d, acc, y (uint16 bf16 bits).
+    """
+    X = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    W = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    M, K = X.shape
+    N = W.shape[0]
+    Y = np.empty((M, N), dtype=np.uint16)
+    gamma = np.zeros(1, dtype=np.float32)
+    q = np.empty((N, K), dtype=np.int8)
+    z = np.empty((M, K), dtype=np.float64)
+    codes = np.empty((M, K), dtype=np.int8)
+    d = np.empty(M, dtype=np.float32)
+    acc = np.empty((M, N), dtype=np.int64)
+    rc = lib().oracle_bitlinear_forward(_p(X), M, K, _p(W), N, int(bool(hadamard)), int(bits),
+                                        _p(Y), _p(gamma), _p(q), _p(z), _p(codes), _p(d),
+                                        _p(acc))
+    if rc != 0:
+        raise MemoryError("oracle_bitlinear_forward could not allocate its buffers")
+    return {"gamma": np.float32(gamma[0]), "q": q, "z": z, "codes": codes, "d": d,
+            "acc": acc, "y": Y}

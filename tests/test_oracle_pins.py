@@ -1,0 +1,378 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these re-types an oracle formula.  Each compares the oracle with something
+independent of it: a worked example printed on a page (tests/golden/), a closed form, an
+invariant, a textbook or library special case, or brute force on tiny inputs.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+from bit_activation_linear_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def bf16_bits(values):
+    return synth.f32_to_bf16_bits(np.asarray(values, dtype=np.float32))
+
+
+# ----------------------------------------------------------------------------------------
+# Hadamard transform (BitNet v2 write-up: entries +-1, mutually orthogonal rows)
+# ----------------------------------------------------------------------------------------
+
+def sylvester_blocks(n):
+    """H_n by the block recursion H_2m = [[H_m, H_m], [H_m, -H_m]], H_1 = [1]."""
+    H = np.ones((1, 1))
+    while H.shape[0] < n:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def sylvester_bits(n):
+    """H_n[i, j] = (-1)^popcount(i & j): an independent closed form of the same matrix."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    parity = np.vectorize(lambda v: bin(int(v)).count("1") & 1)(i & j)
+    return 1.0 - 2.0 * parity
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64])
+def test_hadamard_entries_and_orthogonality(n):
+    H = sylvester_blocks(n)
+    assert set(np.unique(H)) <= {-1.0, 1.0}
+    np.testing.assert_array_equal(H @ H.T, n * np.eye(n))
+    np.testing.assert_array_equal(H, sylvester_bits(n))
+    np.testing.assert_array_equal(H, scipy.linalg.hadamard(n))
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 32, 64])
+def test_fwht_equals_explicit_matrix_product(n):
+    rng = np.random.default_rng(n)
+    x = rng.standard_normal((5, n))
+    z = oracle.fwht(x)
+    ref = x @ sylvester_blocks(n).T / math.sqrt(n)
+    np.testing.assert_allclose(z, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("n", [128, 256, 1024])
+def test_fwht_equals_library_hadamard(n):
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((3, n))
+    ref = x @ scipy.linalg.hadamard(n).T.astype(np.float64) / math.sqrt(n)
+    np.testing.assert_allclose(oracle.fwht(x), ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("n", [2, 64, 2048, 8192])
+def test_fwht_involution_and_parseval(n):
+    rng = np.random.default_rng(n + 1)
+    x = rng.laplace(size=(4, n))
+    z = oracle.fwht(x)
+    np.testing.assert_allclose(np.linalg.norm(z, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(oracle.fwht(z), x, rtol=0, atol=1e-12 * np.abs(x).max())
+
+
+@pytest.mark.parametrize("n", [16, 256])
+def test_fwht_basis_vectors(n):
+    H = sylvester_bits(n)
+    E = np.eye(n)
+    np.testing.assert_allclose(oracle.fwht(E), H.T / math.sqrt(n), atol=1e-14)
+    ones = np.ones((1, n))
+    e0 = np.zeros((1, n))
+    e0[0, 0] = math.sqrt(n)
+    np.testing.assert_allclose(oracle.fwht(ones), e0, atol=1e-12)
+
+
+def test_hadamard_makes_sharp_inputs_gaussian_like():
+    """BitNet v2 write-up (Figures 2-3): after the transform the outlier-heavy inputs of
+    Wo / Wdown look close to Gaussian, and low-bit quantisation loses less."""
+    K = 2048
+    x = oracle.bf16_to_f64(synth.sharp_activations(64, K, seed=3))
+    z = oracle.fwht(x)
+
+    def excess_kurtosis(a):
+        a = a - a.mean(axis=1, keepdims=True)
+        return (np.mean(a ** 4, axis=1) / np.mean(a ** 2, axis=1) ** 2 - 3.0).mean()
+
+    assert excess_kurtosis(x) > 20.0
+    assert abs(excess_kurtosis(z)) < 0.5
+
+    def int4_rel_mse(v):
+        c, d, _, _ = oracle.quant_act(v.astype(np.float32), 4)
+        err = c.astype(np.float64) * d[:, None].astype(np.float64) - v
+        return np.mean(err ** 2) / np.mean(v ** 2)
+
+    assert int4_rel_mse(z) < 0.5 * int4_rel_mse(x)
+
+
+# ----------------------------------------------------------------------------------------
+# absmean ternarisation (b1.58 summary, 方法论 / 方法详解)
+# ----------------------------------------------------------------------------------------
+
+def test_ternarize_hand_example():
+    g = golden("ternary_hand_example.json")
+    W = bf16_bits(g["W"])
+    gamma = oracle.absmean_gamma(W)
+    assert gamma == np.float32(g["gamma"])
+    np.testing.assert_array_equal(oracle.ternarize(W, gamma), np.array(g["q"], dtype=np.int8))
+
+
+def test_gamma_is_library_mean_of_abs():
+    W = synth.latent_weights(64, 512, seed=5)
+    ref = np.float32(np.mean(np.abs(oracle.bf16_to_f64(W))))
+    assert oracle.absmean_gamma(W) == ref
+
+
+def test_ternarize_brute_force_nearest():
+    """q is the element of {-1, 0, 1} nearest to w / gamma (fp32 ratio)."""
+    W = synth.latent_weights(32, 256, seed=11)
+    gamma = oracle.absmean_gamma(W)
+    q = oracle.ternarize(W, gamma)
+    r = oracle.bf16_to_f64(W).astype(np.float32) / np.float32(gamma)
+    cands = np.array([-1.0, 0.0, 1.0])
+    dist = np.abs(r.astype(np.float64)[..., None] - cands)
+    assert not np.any(np.isclose(np.sort(dist, axis=-1)[..., 0], np.sort(dist, axis=-1)[..., 1]))
+    np.testing.assert_array_equal(q, cands[np.argmin(dist, axis=-1)].astype(np.int8))
+
+
+def test_ternarize_alphabet_and_zero_fraction():
+    """Codes lie in {-1, 0, 1}; for W ~ N(0, s), |w| / mean|w| <= 1/2 happens with
+    probability 2 Phi(sqrt(2/pi) / 2) - 1 = 0.3101 (half-normal mean s sqrt(2/pi))."""
+    W = synth.latent_weights(512, 1024, seed=0)
+    q = oracle.ternarize(W, oracle.absmean_gamma(W))
+    assert set(np.unique(q)) <= {-1, 0, 1}
+    p0 = 2.0 * 0.5 * (1.0 + math.erf(math.sqrt(2.0 / math.pi) / 2.0 / math.sqrt(2.0))) - 1.0
+    assert abs(p0 - 0.3101) < 1e-4
+    n = q.size
+    frac0 = np.mean(q == 0)
+    assert abs(frac0 - p0) < 4.0 * math.sqrt(p0 * (1 - p0) / n) + 2e-3  # +bf16 rounding of W
+    assert abs(np.mean(q == 1) - np.mean(q == -1)) < 0.01
+
+
+def test_ternarize_constant_and_zero_weights():
+    W = bf16_bits(np.full((4, 16), -0.03125))
+    g = oracle.absmean_gamma(W)
+    assert g == np.float32(0.03125)
+    np.testing.assert_array_equal(oracle.ternarize(W, g), -np.ones((4, 16), np.int8))
+    Z = bf16_bits(np.zeros((2, 16)))
+    assert oracle.absmean_gamma(Z) == np.float32(1e-5)
+    np.testing.assert_array_equal(oracle.ternarize(Z, oracle.absmean_gamma(Z)), 0)
+
+
+def test_ternarize_ties_round_half_to_even():
+    """|w / gamma| = 0.5 exactly rounds to 0, 1.5 rounds to 2 and clips to 1."""
+    gamma = np.float32(0.25)
+    W = bf16_bits([0.125, -0.125, 0.375, -0.375, 0.1250001])
+    np.testing.assert_array_equal(oracle.ternarize(W, gamma), [0, 0, 1, -1, 0])
+
+
+# ----------------------------------------------------------------------------------------
+# Storage formats
+# ----------------------------------------------------------------------------------------
+
+def test_base3_example_from_the_page():
+    g = golden("base3_packing.json")
+    b = oracle.pack_base3(np.array(g["digits"], dtype=np.uint8))
+    assert b.tolist() == [g["byte"]]
+    assert format(int(b[0]), "08b") == g["binary"]
+    np.testing.assert_array_equal(oracle.unpack_base3(b, 5), g["digits"])
+    assert round(100 * 5 * math.log2(3) / 8, 2) == g["efficiency_percent"]
+
+
+def test_base3_round_trip_and_range():
+    rng = np.random.default_rng(2)
+    d = rng.integers(0, 3, size=1003).astype(np.uint8)
+    b = oracle.pack_base3(d)
+    assert b.size == 201 and int(b.max()) <= 242
+    np.testing.assert_array_equal(oracle.unpack_base3(b, d.size), d)
+
+
+def test_ternary_word_layout_hand_example():
+    g = golden("ternary_word_layout.json")
+    q = np.array([g["q"]], dtype=np.int8)
+    wp = oracle.pack_ternary(q)
+    assert wp.shape == (1, 1) and int(wp[0, 0]) == g["word"]
+    back, bad = oracle.unpack_ternary(wp, 16)
+    assert bad == 0
+    np.testing.assert_array_equal(back, q)
+
+
+def test_ternary_pack_round_trip():
+    rng = np.random.default_rng(4)
+    q = rng.integers(-1, 2, size=(37, 256)).astype(np.int8)
+    wp = oracle.pack_ternary(q)
+    assert wp.nbytes == q.size // 4
+    back, bad = oracle.unpack_ternary(wp, 256)
+    assert bad == 0
+    np.testing.assert_array_equal(back, q)
+
+
+def test_int4_nibble_layout_hand_example():
+    g = golden("int4_nibble_layout.json")
+    c = np.array([g["codes"]], dtype=np.int8)
+    b = oracle.pack_int4(c)
+    assert b.ravel().tolist() == g["bytes"]
+    np.testing.assert_array_equal(oracle.unpack_int4(b, 8), c)
+
+
+# ----------------------------------------------------------------------------------------
+# Per-token absmax quantisation (2B4T article, 一.2; BitNet v2 write-up)
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,Q", [(8, 127), (4, 7)])
+def test_quant_brute_force_nearest_and_extremes(bits, Q):
+    rng = np.random.default_rng(bits)
+    z = (rng.laplace(size=(20, 256)) * 0.3).astype(np.float32)
+    z[3] = 0.0
+    codes, d, pre, rowsum = oracle.quant_act(z, bits)
+    # zero row: zero codes, guarded scale
+    assert not codes[3].any() and d[3] == np.float32(np.float32(1e-5) / np.float32(Q))
+    live = [m for m in range(20) if m != 3]
+    # the largest |z| of each row maps to +-Q exactly; all codes lie in range
+    for m in live:
+        k = int(np.argmax(np.abs(z[m])))
+        assert codes[m, k] == Q * np.sign(z[m, k])
+    assert codes.min() >= -Q and codes.max() <= Q
+    # brute force: each code is the integer nearest to z * s with s = fp32(Q / max|z|)
+    s = (np.float32(Q) / np.abs(z).max(axis=1).clip(min=np.float32(1e-5))).astype(np.float32)
+    v = (z * s[:, None]).astype(np.float32).astype(np.float64)
+    cand = np.stack([np.floor(v), np.ceil(v)], axis=-1)
+    best = np.take_along_axis(cand, np.argmin(np.abs(cand - v[..., None]), axis=-1)[..., None],
+                              axis=-1)[..., 0]
+    np.testing.assert_array_equal(codes[live], best[live].astype(np.int8))
+    np.testing.assert_array_equal(rowsum, codes.astype(np.int64).sum(axis=1))
+    # d is the dequantisation step: codes * d reproduces z to within half a step
+    err = np.abs(codes * d[:, None].astype(np.float64) - z)
+    assert np.all(err[live] <= 0.5 * d[live, None] * (1 + 1e-6))
+
+
+# ----------------------------------------------------------------------------------------
+# Ternary product (2B4T article, 一.2: +1 adds, -1 subtracts, 0 skips)
+# ----------------------------------------------------------------------------------------
+
+def test_gemm_three_ways_agree():
+    rng = np.random.default_rng(9)
+    c = rng.integers(-128, 128, size=(7, 96)).astype(np.int8)
+    q = rng.integers(-1, 2, size=(5, 96)).astype(np.int8)
+    a = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(a, oracle.gemm_addsub(c, q))
+    np.testing.assert_array_equal(a, c.astype(np.int64) @ q.astype(np.int64).T)
+
+
+def test_gemm_all_ones_weights_give_row_sums():
+    rng = np.random.default_rng(10)
+    c = rng.integers(-128, 128, size=(4, 64)).astype(np.int8)
+    q = np.ones((3, 64), np.int8)
+    np.testing.assert_array_equal(oracle.gemm_i64(c, q),
+                                  np.repeat(c.astype(np.int64).sum(1, keepdims=True), 3, 1))
+
+
+def test_gemm_tiny_by_hand():
+    c = np.array([[1, 2, 3], [-4, 5, -6]], np.int8)
+    q = np.array([[1, 0, -1], [-1, -1, 1], [0, 1, 0]], np.int8)
+    # row 0: 1-3=-2, -1-2+3=0, 2 ; row 1: -4+6=2, 4-5-6=-7, 5
+    np.testing.assert_array_equal(oracle.gemm_i64(c, q), [[-2, 0, 2], [2, -7, 5]])
+
+
+# ----------------------------------------------------------------------------------------
+# bf16 rounding of the output
+# ----------------------------------------------------------------------------------------
+
+def test_bf16_rounding_cases():
+    f = oracle.f64_to_bf16
+    cases = {
+        1.0: 0x3F80,
+        1.0 + 2 ** -8: 0x3F80,                 # tie -> even (1.0)
+        1.0 + 3 * 2 ** -8: 0x3F82,             # tie -> even (1 + 2^-6)
+        1.0 + 2 ** -8 + 2 ** -40: 0x3F81,      # above the tie: rounding via fp32 would give 1.0
+        -2.5: 0xC020,
+        2.0 ** -133: 0x0001,                   # smallest subnormal
+        3.0 * 2.0 ** -134: 0x0002,             # subnormal tie -> even
+        1e39: 0x7F80,                          # overflow
+    }
+    for v, bits in cases.items():
+        assert int(f(np.array([v]))[0]) == bits, v
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000)
+    # for values already exact in fp32 (no double rounding possible) torch agrees
+    x32 = x.astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(x32).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy()
+    np.testing.assert_array_equal(f(x32), ref.view(np.uint16))
+
+
+def test_dequant_against_exact_products():
+    acc = np.array([[0, 1, -127, 2_000_000]], np.int64)
+    d = np.array([0.5], np.float32)
+    Y = oracle.dequant(acc, d, np.float32(0.25))
+    np.testing.assert_array_equal(oracle.bf16_to_f64(Y), [[0.0, 0.125, -15.875, 249856.0]])
+
+
+# ----------------------------------------------------------------------------------------
+# Whole forward: closed forms
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_forward_hadamard_column_input(bits):
+    """x = a * (column j of H): z = a sqrt(K) e_j, so the codes are +-Q at j only and
+    Y[n] = q[n, j] * a * sqrt(K) * gamma (up to bf16 rounding).  A transposed operand, a
+    dropped normalisation or a wrong sign fails here."""
+    K, N = 256, 64
+    H = sylvester_bits(K)
+    a = 0.125
+    js = [0, 3, 77, 255]
+    X = bf16_bits(np.stack([a * H[:, j] * (1 if t % 2 == 0 else -1) for t, j in enumerate(js)]))
+    W = synth.latent_weights(N, K, seed=1)
+    out = oracle.bitlinear_forward(X, W, hadamard=True, bits=bits)
+    Q = 127 if bits == 8 else 7
+    gamma = float(out["gamma"])
+    for t, j in enumerate(js):
+        sgn = 1 if t % 2 == 0 else -1
+        expect_codes = np.zeros(K, np.int8)
+        expect_codes[j] = sgn * Q
+        np.testing.assert_array_equal(out["codes"][t], expect_codes)
+        y = oracle.bf16_to_f64(out["y"][t])
+        ref = sgn * out["q"][:, j] * a * math.sqrt(K) * gamma
+        np.testing.assert_allclose(y, ref, rtol=2 ** -8, atol=0)
+
+
+def test_forward_plain_constant_rows():
+    """Plain BitLinear with a constant row c: every code is 127 and
+    Y[n] = c * gamma * sum_k q[n, k]."""
+    K, N = 128, 32
+    X = bf16_bits(np.array([[0.5] * K, [-3.0] * K]))
+    W = synth.latent_weights(N, K, seed=2)
+    out = oracle.bitlinear_forward(X, W, hadamard=False, bits=8)
+    assert np.all(np.abs(out["codes"]) == 127)
+    rs = out["q"].astype(np.float64).sum(axis=1)
+    for m, cval in enumerate([0.5, -3.0]):
+        np.testing.assert_allclose(oracle.bf16_to_f64(out["y"][m]), cval * float(out["gamma"]) * rs,
+                                   rtol=2 ** -8)
+
+
+def test_forward_stages_compose():
+    """The composite forward equals its own stages called one by one."""
+    wl = synth.WORKLOADS["tiny"]
+    X = wl.activations()
+    W = wl.weights()
+    out = oracle.bitlinear_forward(X, W, hadamard=True, bits=8)
+    g = oracle.absmean_gamma(W)
+    q = oracle.ternarize(W, g)
+    z = oracle.fwht(oracle.bf16_to_f64(X))
+    c, d, _, _ = oracle.quant_act(z.astype(np.float32), 8)
+    acc = oracle.gemm_i64(c, q)
+    assert out["gamma"] == g
+    np.testing.assert_array_equal(out["q"], q)
+    np.testing.assert_array_equal(out["codes"], c)
+    np.testing.assert_array_equal(out["acc"], acc)
+    np.testing.assert_array_equal(out["y"], oracle.dequant(acc, d, g))

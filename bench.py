@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the H-BitLinear forward on B200: one JSON line on rank 0.
+
+A step is one pass of the whole forward over one batch of synthetic input: absmean
+ternarisation + packing of the latent weights (2 kernels), the fused Hadamard + absmax INT8
+quantisation of the tokens (1 kernel) and the ternary x int8 tensor-core product with the bf16
+rescale (1 kernel).  Default workload: the Wo-shaped layer of a 2B-class model
+(M = 4096 tokens, K = N = 2048, H-BitLinear, INT8 activations).
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
+cuda.synchronize on both sides, timed with CUDA events on the launching stream, max over ranks.
+Inputs are rotated over several copies whose total exceeds twice the L2 cache, so no step finds
+its inputs in L2.  Each copy's step is captured in two CUDA graphs (everything before the product,
+and the product) so that host launch overhead does not starve the GPU; CUDA events recorded
+around the product's replay give its live duration for the roofline figure.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the data
+path); rank 0 prints the line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_activation_linear_b200 import synth  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
+METRIC = "H-BitLinear tokens/s and effective int8 TOPS (% of roofline) on 1 B200"
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------------------
+# algorithmic work per kernel (bytes at the stored widths, ops of the product)
+# ----------------------------------------------------------------------------------------
+
+def kernel_work(wl):
+    M, K, N = wl.M, wl.K, wl.N
+    code_bytes = M * K if wl.act_bits == 8 else M * K // 2
+    return {
+        # read W (bf16) once
+        "absmean_partials": {"bytes": 2 * N * K},
+        # read W (bf16) once, write the 2-bit weights
+        "ternarize_pack": {"bytes": 2 * N * K + N * K // 4},
+        # read X (bf16), write codes + scale + code sum per token
+        "fwht_quant": {"bytes": 2 * M * K + code_bytes + 8 * M},
+        # product: 2 M N K integer ops; bytes = codes + 2-bit weights + bf16 Y
+        "ternary_gemm_tc": {"ops": 2 * M * N * K,
+                            "bytes": code_bytes + N * K // 4 + 2 * M * N + 8 * M},
+    }
+
+
+# ----------------------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        out_dir = os.path.join(ROOT, "gpurun_out")
+        os.makedirs(out_dir, exist_ok=True)
+        self.path = os.path.join(out_dir, f"bench_clocks_rank{self.idx}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                                 "power": float(parts[3]), "active": parts[4],
+                                 "hw": parts[5], "hw_thermal": parts[6],
+                                 "sw_thermal": parts[7], "sw_power": parts[8]})
+                except ValueError:
+                    continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # samples under load: the SM clock is the one the GPU ran the steps at
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in loaded),
+                "power_w_max": max(r["power"] for r in loaded),
+                "samples": len(loaded), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------------
+# the oracle as a CPU baseline (test infrastructure, timed as it stands)
+# ----------------------------------------------------------------------------------------
+
+def oracle_sample(wl, rows: int, seed: int = 0):
+    """Time the oracle's forward on `rows` tokens (full weight preparation included once)."""
+    import oracle
+    X = wl.activations(seed=seed, rows=rows)
+    W = wl.weights(seed=seed)
+    t0 = time.perf_counter()
+    oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits)
+    return time.perf_counter() - t0
+
+
+def oracle_baseline(wl, target_s: float = 12.0):
+    """tokens/s of the oracle, measured on a bounded sample and scaled to one full step:
+    t_step = t_prep + (M / r) * t_rows(r), tokens/s = M / t_step."""
+    import oracle
+    W = wl.weights()
+    t0 = time.perf_counter()
+    g = oracle.absmean_gamma(W)
+    oracle.pack_ternary(oracle.ternarize(W, g))
+    t_prep = time.perf_counter() - t0
+    probe_rows = 16
+    t_probe = oracle_sample(wl, probe_rows) - t_prep
+    per_row = max(t_probe, 1e-6) / probe_rows
+    rows = int(max(probe_rows, min(wl.M, (target_s - t_prep) / per_row)))
+    t_rows = oracle_sample(wl, rows) - t_prep
+    t_step = t_prep + (wl.M / rows) * max(t_rows, 1e-9)
+    return {"value": wl.M / t_step, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"{rows} of {wl.M} token rows of {wl.name} through the C oracle "
+                       f"(plain loops, fp64 FWHT, int64 GEMM, OpenMP over rows) plus one full "
+                       f"weight ternarisation ({t_prep:.2f} s); per-step time scaled to all "
+                       f"{wl.M} tokens: t_prep + (M/rows) * t_rows"),
+            "t_prep_s": t_prep, "t_rows_s": t_rows, "rows": rows}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    budget_s = 150.0
+    W = wl.weights()
+    t0 = time.perf_counter()
+    g = oracle.absmean_gamma(W)
+    oracle.pack_ternary(oracle.ternarize(W, g))
+    t_prep = time.perf_counter() - t0
+    t_probe = oracle_sample(wl, 8) - t_prep
+    per_row = max(t_probe, 1e-6) / 8
+    steps_total = args.steps + args.warmup
+    rows = int(max(1, min(wl.M, (budget_s / steps_total - t_prep) / per_row)))
+    times = []
+    for i in range(steps_total):
+        X = wl.activations(seed=i, rows=rows)
+        t0 = time.perf_counter()
+        oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    t_rows = statistics.mean(times) - t_prep
+    t_step = t_prep + (wl.M / rows) * max(t_rows, 1e-9)
+    value = wl.M / t_step
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "M": wl.M, "K": wl.K, "N": wl.N,
+                   "hadamard": wl.hadamard, "act_bits": wl.act_bits},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": (f"each step: {rows} token rows of {wl.name} through the C "
+                                    f"oracle; weight ternarisation of the full W included once "
+                                    f"per step; time scaled to all {wl.M} tokens")},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------------------
+
+def aggregate_max(value: float, device) -> float:
+    """Maximum of a per-rank float over all ranks (identity without a process group)."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def run_gpu(args, wl, rank, world, device):
+    from bit_activation_linear_b200 import binding as B
+    B.load_library()
+    stream = torch.cuda.Stream(device)
+    torch.cuda.set_stream(stream)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    M, K, N = wl.M, wl.K, wl.N
+    code_bytes = M * K if wl.act_bits == 8 else M * K // 2
+    per_copy = 2 * M * K + 2 * N * K + N * K // 4 + code_bytes + 2 * M * N
+    copies = max(2, math.ceil(2 * l2 / per_copy) + 1)
+
+    # inputs: one batch per rank (seed = rank), rotated copies of X and W
+    X0 = synth.to_torch_bf16(wl.activations(seed=rank))
+    W0 = synth.to_torch_bf16(wl.weights(seed=rank))
+    bufs = []
+    for i in range(copies):
+        X = X0.to(device, non_blocking=False).clone()
+        W = W0.to(device).clone()
+        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+        gamma = torch.empty(1, dtype=torch.float32, device=device)
+        wws = torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
+                          device=device)
+        codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
+        scales = torch.empty(M, dtype=torch.float32, device=device)
+        rowsum = torch.empty(M, dtype=torch.int32, device=device)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        bufs.append(dict(X=X, W=W, Wp=Wp, gamma=gamma, wws=wws, codes=codes, scales=scales,
+                         rowsum=rowsum, Y=Y))
+
+    def prep(b):
+        B.bitnet_quantize_pack_weights(b["W"], b["Wp"], b["gamma"], b["wws"])
+        B.bitnet_act_quant(b["X"], wl.hadamard, wl.act_bits, b["codes"], b["scales"],
+                           b["rowsum"])
+
+    def gemm(b):
+        B.bitnet_ternary_gemm(b["codes"], b["scales"], b["rowsum"], K, b["Wp"], b["gamma"],
+                              wl.act_bits, want_acc=False, want_y=True, Y=b["Y"])
+
+    launches_before = B.bitnet_launch_count()
+    for b in bufs:  # eager run once (sets kernel attributes, checks status)
+        prep(b)
+        gemm(b)
+    B.bitnet_sync_status(stream)
+    launches_per_step = (B.bitnet_launch_count() - launches_before) // copies
+
+    g_prep, g_gemm = [], []
+    for b in bufs:
+        gp, gg = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp, stream=stream):
+            prep(b)
+        with torch.cuda.graph(gg, stream=stream):
+            gemm(b)
+        g_prep.append(gp)
+        g_gemm.append(gg)
+    torch.cuda.synchronize(device)
+
+    def step(i, ev=None):
+        j = i % copies
+        g_prep[j].replay()
+        if ev is not None:
+            ev[0].record(stream)
+        g_gemm[j].replay()
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    B.bitnet_sync_status(stream)
+
+    n_ev = min(args.steps, 512)
+    every = max(1, args.steps // n_ev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_ev)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize(device)
+    # a short device sleep lets the host queue the first replays before the clock starts
+    torch.cuda._sleep(int(2e7))
+    t_start.record(stream)
+    k_ev = 0
+    for i in range(args.steps):
+        use = (i % every == 0) and k_ev < n_ev
+        step(i, evs[k_ev] if use else None)
+        if use:
+            k_ev += 1
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    clocks = sampler.stop()
+    B.bitnet_sync_status(stream)
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    gemm_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(k_ev))
+    elapsed_ms = aggregate_max(elapsed_ms, device)
+    gemm_ms = aggregate_max(gemm_ms, device)
+    ms_per_step = elapsed_ms / args.steps
+
+    # end to end through the public API: pinned host X and W in, Y out, every step
+    e2e = run_e2e(args, wl, B, stream, device, X0, W0)
+
+    if rank == 0:
+        peaks, peak_kind = load_peaks()
+        work = kernel_work(wl)
+        int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        achieved = work["ternary_gemm_tc"]["ops"] / (gemm_ms * 1e-3) / 1e12
+        tokens_per_s = world * M / (ms_per_step * 1e-3)
+        line = {
+            "metric": METRIC,
+            "value": tokens_per_s,
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "int8",
+            "data": "synthetic",
+            "effective_tops": world * wl.ops / (ms_per_step * 1e-3) / 1e12,
+            "config": {"workload": wl.name, "M": M, "K": K, "N": N, "hadamard": wl.hadamard,
+                       "act_bits": wl.act_bits, "tokens_per_rank": M,
+                       "parallelism": f"replicas{world}",
+                       "l2": f"inputs rotated over {copies} copies "
+                             f"({copies * per_copy / 2**20:.0f} MiB > 2 x L2)"},
+            "roofline": {"kernel": "ternary_gemm_tc", "bound": "tensor",
+                         "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                         "frac": achieved / int8_peak, "traffic": None,
+                         "ms_per_launch": gemm_ms,
+                         "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x "
+                                        f"{INT8_PER_BF16} (nominal int8:bf16 dense ratio)"},
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = oracle_baseline(wl, args.cpu_seconds)
+        elif not args.no_cpu_baseline:
+            line["cpu_baseline"] = None
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, wl, B, stream, device, X0, W0):
+    M, K, N = wl.M, wl.K, wl.N
+    Xh = X0.pin_memory()
+    Wh = W0.pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(Xh, device=device)
+    Wd = torch.empty_like(Wh, device=device)
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+    gamma = torch.empty(1, dtype=torch.float32, device=device)
+    wws = torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
+                      device=device)
+    ws = torch.empty(max(B.bitnet_workspace_bytes(M, K, N, wl.act_bits), 256), dtype=torch.uint8,
+                     device=device)
+    fwd = B.bitnet_hbitlinear_forward if wl.hadamard else B.bitnet_bitlinear_forward
+
+    def step():
+        Xd.copy_(Xh, non_blocking=True)
+        Wd.copy_(Wh, non_blocking=True)
+        B.bitnet_quantize_pack_weights(Wd, Wp, gamma, wws)
+        fwd(Xd, Wp, gamma, wl.act_bits, Y=Yd, ws=ws)
+        Yh.copy_(Yd, non_blocking=True)
+
+    n = max(3, min(args.steps, 100))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    ms = aggregate_max(s.elapsed_time(e) / n, device)
+    world = dist.get_world_size() if dist.is_initialized() else 1
+    return {"value": world * M / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": Xh.numel() * 2 + Wh.numel() * 2,
+            "d2h_bytes_per_step": Yh.numel() * 2, "ms_per_step": ms, "steps": n}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default="wo_2048", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=device)
+    try:
+        run_gpu(args, wl, rank, world, device)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -11,9 +11,7 @@ __all__ = ["synth"]
 
 
 def __getattr__(name):
-    if name.startswith("bitnet_") or name in ("binding", "BitnetError", "load_library"):
-        from . import binding
-        if name == "binding":
-            return binding
-        return getattr(binding, name)
+    if name.startswith("bitnet_") or name in ("BitnetError", "load_library"):
+        import importlib
+        return getattr(importlib.import_module(".binding", __name__), name)
     raise AttributeError(name)

@@ -1,0 +1,239 @@
+"""Python binding of libbitnet_b200.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls (include/bitnet.h), takes torch
+CUDA tensors, checks dtype / device / contiguity, allocates outputs and workspace with torch
+(the library itself never allocates) and passes raw pointers plus the current torch stream.  All
+arithmetic runs in the library's kernels; there is no fallback of any kind: if the shared
+library is missing or cannot load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitnet_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+
+
+class BitnetError(RuntimeError):
+    """A non-zero status from the library, with its text and the library's detail message."""
+
+    def __init__(self, status: int, where: str):
+        lib = load_library()
+        self.status = status
+        text = lib.bitnet_status_string(status).decode()
+        detail = lib.bitnet_last_error().decode()
+        super().__init__(f"{where}: {text} ({status}): {detail}")
+
+
+_SIGS = {
+    "bitnet_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "bitnet_last_error": (ctypes.c_char_p, []),
+    "bitnet_launch_count": (ctypes.c_uint64, []),
+    "bitnet_packed_weight_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "bitnet_weight_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "bitnet_quantize_pack_weights": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                    ctypes.c_int64, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_act_codes_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
+    "bitnet_act_quant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_fwht_f32": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_ternary_gemm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                                 ctypes.c_int]),
+    "bitnet_bitlinear_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_hbitlinear_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
+}
+
+EXPORTED = tuple(_SIGS)
+
+
+def load_library(path: str | None = None):
+    """Load (once) and return the ctypes handle of libbitnet_b200.so.  Raises if it is absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or LIB_PATH
+            if not os.path.exists(p):
+                raise RuntimeError(
+                    f"{p} is missing: build it with `python -m bit_activation_linear_b200.build`"
+                    " (nvcc, sm_100a). There is no fallback implementation.")
+            lib = ctypes.CDLL(p)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype=None, dim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions")
+
+
+def _rc(status: int, where: str):
+    if status != OK:
+        raise BitnetError(status, where)
+
+
+def bitnet_launch_count() -> int:
+    return int(load_library().bitnet_launch_count())
+
+
+def bitnet_packed_weight_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_packed_weight_bytes(N, K))
+
+
+def bitnet_weight_workspace_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_weight_workspace_bytes(N, K))
+
+
+def bitnet_act_codes_bytes(M: int, K: int, act_bits: int) -> int:
+    return int(load_library().bitnet_act_codes_bytes(M, K, act_bits))
+
+
+def bitnet_workspace_bytes(M: int, K: int, N: int, act_bits: int) -> int:
+    return int(load_library().bitnet_workspace_bytes(M, K, N, act_bits))
+
+
+def bitnet_quantize_pack_weights(W: torch.Tensor, Wp: torch.Tensor | None = None,
+                                 gamma: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                                 stream=None):
+    """absmean-ternarise and pack bf16 W [N, K].  Returns (Wp uint8 [N, K/4], gamma float [1])."""
+    L = load_library()
+    _check(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    if Wp is None:
+        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    need = int(L.bitnet_weight_workspace_bytes(N, K))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    _rc(L.bitnet_quantize_pack_weights(W.data_ptr(), N, K, Wp.data_ptr(), gamma.data_ptr(),
+                                       ws.data_ptr(), ws.numel() * ws.element_size(),
+                                       _stream(stream)), "bitnet_quantize_pack_weights")
+    return Wp, gamma
+
+
+def bitnet_act_quant(X: torch.Tensor, hadamard: bool, act_bits: int, codes=None, scales=None,
+                     rowsum=None, stream=None):
+    """Per-token (Hadamard +) absmax quantisation.  Returns (codes, scales, rowsum)."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if codes is None:
+        codes = torch.empty((M, K if act_bits == 8 else K // 2),
+                            dtype=torch.int8 if act_bits == 8 else torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=X.device)
+    if rowsum is None:
+        rowsum = torch.empty(M, dtype=torch.int32, device=X.device)
+    _rc(L.bitnet_act_quant(X.data_ptr(), M, K, int(bool(hadamard)), int(act_bits),
+                           codes.data_ptr(), scales.data_ptr(), rowsum.data_ptr(),
+                           _stream(stream)), "bitnet_act_quant")
+    return codes, scales, rowsum
+
+
+def bitnet_fwht_f32(X: torch.Tensor, Z: torch.Tensor | None = None, stream=None):
+    """Z = H_K X / sqrt(K) per row in fp32 (debug / parity entry)."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if Z is None:
+        Z = torch.empty((M, K), dtype=torch.float32, device=X.device)
+    _rc(L.bitnet_fwht_f32(X.data_ptr(), M, K, Z.data_ptr(), _stream(stream)), "bitnet_fwht_f32")
+    return Z
+
+
+def bitnet_ternary_gemm(codes: torch.Tensor, scales: torch.Tensor, rowsum: torch.Tensor, K: int,
+                        Wp: torch.Tensor, gamma: torch.Tensor, act_bits: int, want_acc=False,
+                        want_y=True, acc=None, Y=None, stream=None):
+    """Ternary x integer product (+ rescale).  Returns (acc int32 [M, N] or None, Y bf16 or None)."""
+    L = load_library()
+    for t, n in ((codes, "codes"), (scales, "scales"), (rowsum, "rowsum"), (Wp, "Wp"),
+                 (gamma, "gamma")):
+        _check(t, n)
+    M = codes.shape[0]
+    N = Wp.shape[0]
+    if want_acc and acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=codes.device)
+    if want_y and Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=codes.device)
+    _rc(L.bitnet_ternary_gemm(codes.data_ptr(), scales.data_ptr(), rowsum.data_ptr(), M, K,
+                              Wp.data_ptr(), gamma.data_ptr(), N, int(act_bits),
+                              acc.data_ptr() if acc is not None else None,
+                              Y.data_ptr() if Y is not None else None, _stream(stream)),
+        "bitnet_ternary_gemm")
+    return acc, Y
+
+
+def _forward(fn_name: str, X, Wp, gamma, act_bits, Y, ws, stream):
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    _check(Wp, "Wp")
+    _check(gamma, "gamma", torch.float32)
+    M, K = X.shape
+    N = Wp.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    need = int(L.bitnet_workspace_bytes(M, K, N, act_bits))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _rc(getattr(L, fn_name)(X.data_ptr(), M, K, Wp.data_ptr(), gamma.data_ptr(), N,
+                            int(act_bits), Y.data_ptr(), ws.data_ptr(),
+                            ws.numel() * ws.element_size(), _stream(stream)), fn_name)
+    return Y
+
+
+def bitnet_bitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=None):
+    """Y = BitLinear(X) for bf16 X [M, K] and packed ternary Wp [N, K/4]."""
+    return _forward("bitnet_bitlinear_forward", X, Wp, gamma, act_bits, Y, ws, stream)
+
+
+def bitnet_hbitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=None):
+    """Y = H-BitLinear(X): online Hadamard transform, then BitLinear."""
+    return _forward("bitnet_hbitlinear_forward", X, Wp, gamma, act_bits, Y, ws, stream)
+
+
+def bitnet_sync_status(stream=None) -> int:
+    """Synchronise the stream and raise BitnetError if a kernel reported a fault or time-out."""
+    st = load_library().bitnet_sync_status(_stream(stream))
+    _rc(st, "bitnet_sync_status")
+    return st

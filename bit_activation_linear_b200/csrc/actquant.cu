@@ -1,0 +1,388 @@
+// actquant.cu -- steps 2 and 3 of the forward: the online Hadamard transform of every token
+// row (H-BitLinear) fused with per-token absmax quantisation to INT8 or INT4.
+//
+// BitNet v2 write-up, paragraphs on H-BitLinear: before the activations of Wo and Wdown are
+// quantised, each token row is multiplied by a Hadamard matrix (entries +-1, mutually
+// orthogonal rows), which turns the sharp, outlier-heavy distribution into a near-Gaussian
+// one.  BitNet b1.58 2B4T article, section 一.2: activations are quantised per token with
+// absmax to 8 bits; the BitNet v2 write-up adds a native 4-bit variant.  Readings: H_K in
+// Sylvester order scaled by 1/sqrt(K); Q = 127 or 7; eps 1e-5; round half to even.
+//
+// Kernel design (HBM-bound: 2 bytes in, 1 or 0.5 byte out per element):
+//   One "team" of TEAM = 2^t threads owns one token row of K = 2^k elements, V = 2^v values per
+//   thread (v = k - t <= 7, so at most 128 fp32 registers of data).
+//   Phase A  every thread loads bf16 pairs at j = c * 2*TEAM + 2*r + e (coalesced 4-byte loads)
+//            and runs the butterflies of every index bit it holds in registers: bit 0 and the
+//            top v-1 bits.  The Sylvester transform is a product of commuting per-bit
+//            butterflies, so the bits may be processed in any order.
+//   Phase B  the row goes through shared memory once (XOR-swizzled so both the 8-byte writes
+//            and the 16-byte reads are conflict-free); each thread then holds whole contiguous
+//            runs of L = 2^l elements and runs the butterflies of the remaining bits 1..t in
+//            registers (for K = 2^15 and 2^14 the last one or two bits pair neighbouring
+//            lanes through shuffles).
+//   Quantise every thread holds contiguous runs, so codes are packed in registers (float
+//            round-to-int by adding 1.5 * 2^23, byte gather with prmt) and written with 16-byte
+//            stores; the team reduces max|z| and the code sum.
+// Butterflies use the packed fp32x2 add/fma of sm_100.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bitnet {
+
+template <int LOGK>
+struct FwhtPlan {
+    static constexpr int K = 1 << LOGK;
+    static constexpr int T_BITS = (LOGK - 7) > ((LOGK - 1) / 2) ? (LOGK - 7) : ((LOGK - 1) / 2);
+    static constexpr int TEAM = 1 << T_BITS;
+    static constexpr int V_BITS = LOGK - T_BITS;
+    static constexpr int V = 1 << V_BITS;  // values per thread
+    static constexpr int L_BITS = V_BITS < T_BITS + 1 ? V_BITS : T_BITS + 1;
+    static constexpr int L = 1 << L_BITS;  // run length held by one thread in phase B
+    static constexpr int COLS = V / L;     // runs per thread
+    static constexpr int SHFL_BITS = T_BITS + 1 - L_BITS;  // bits done by lane shuffles
+    static constexpr int TPC_A = 256 / TEAM > 0 ? 256 / TEAM : 1;
+    static constexpr int TPC_B = 16384 / K > 0 ? 16384 / K : 1;  // <= 64 KB of smem per CTA
+    static constexpr int TEAMS = TPC_A < TPC_B ? TPC_A : TPC_B;
+    static constexpr int THREADS = TEAMS * TEAM;
+    static constexpr int CHUNKS = L / 4;                      // 16-byte chunks per run
+    static constexpr int SWZ = (CHUNKS < 8 ? CHUNKS : 8) - 1;  // chunk XOR mask
+    static constexpr size_t SMEM = (size_t)TEAMS * K * sizeof(float) + 64 * sizeof(float);
+    static_assert(SHFL_BITS >= 0 && SHFL_BITS <= 5, "plan");
+    static_assert(L >= 16, "runs must hold 16 codes");
+};
+
+__device__ __forceinline__ float2 bfly_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 bfly_sub(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a - b, one rounding
+}
+
+// Team-wide barrier: teams of <= 32 threads live inside one warp.
+template <int TEAM>
+__device__ __forceinline__ void team_sync(int team) {
+    if constexpr (TEAM <= 32) {
+        __syncwarp();
+    } else {
+        asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "n"(TEAM) : "memory");
+    }
+}
+
+template <int LOGK, int BITS, bool ZOUT>
+__global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
+    fwht_quant_kernel(const uint32_t *__restrict__ X, int M, float rsqrt_k,
+                      uint8_t *__restrict__ codes, float *__restrict__ scales,
+                      int32_t *__restrict__ rowsum, float *__restrict__ zout) {
+    using P = FwhtPlan<LOGK>;
+    constexpr int K = P::K, TEAM = P::TEAM, V = P::V, L = P::L;
+    extern __shared__ float4 smem4[];
+    float *smem = reinterpret_cast<float *>(smem4);
+    const int team = threadIdx.x / TEAM;
+    const int r = threadIdx.x % TEAM;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * P::TEAMS + team;
+    const bool valid = row < M;
+    float *tbuf = smem + team * K;
+    float *red = smem + P::TEAMS * K;  // 64 floats of reduction scratch
+
+    // ---- phase A: load bf16 pairs, butterflies over register bits ----
+    float2 a[V / 2];
+    {
+        const uint32_t *xr = X + row * (K / 2);
+#pragma unroll
+        for (int c = 0; c < V / 2; ++c) {
+            uint32_t w = valid ? __ldg(xr + c * TEAM + r) : 0u;
+            a[c] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < V / 2; ++c) {  // index bit 0 (inside the pair)
+        float x = a[c].x, y = a[c].y;
+        a[c] = make_float2(x + y, x - y);
+    }
+#pragma unroll
+    for (int m = 1; m < V / 2; m <<= 1) {  // index bits t+1 .. k-1
+#pragma unroll
+        for (int c = 0; c < V / 2; ++c) {
+            if (c & m) continue;
+            float2 x = a[c], y = a[c | m];
+            a[c] = bfly_add(x, y);
+            a[c | m] = bfly_sub(x, y);
+        }
+    }
+
+    // ---- to shared memory: element j -> run R = j / L, offset o = j % L, chunk-swizzled ----
+#pragma unroll
+    for (int c = 0; c < V / 2; ++c) {
+        const int j = c * 2 * TEAM + 2 * r;
+        const int R = j >> P::L_BITS, o = j & (L - 1);
+        const int phys = R * L + ((((o >> 2) ^ (R & P::SWZ))) << 2) + (o & 3);
+        *reinterpret_cast<float2 *>(tbuf + phys) = a[c];
+    }
+    team_sync<TEAM>(team);
+
+    // ---- phase B: whole runs per thread, butterflies over bits 1 .. l-1 ----
+    float2 b[P::COLS][L / 2];
+#pragma unroll
+    for (int col = 0; col < P::COLS; ++col) {
+        const int R = col * TEAM + r;
+#pragma unroll
+        for (int q = 0; q < P::CHUNKS; ++q) {
+            float4 v = *reinterpret_cast<const float4 *>(tbuf + R * L + ((q ^ (R & P::SWZ)) << 2));
+            b[col][2 * q] = make_float2(v.x, v.y);
+            b[col][2 * q + 1] = make_float2(v.z, v.w);
+        }
+#pragma unroll
+        for (int m = 1; m < L / 2; m <<= 1) {
+#pragma unroll
+            for (int p = 0; p < L / 2; ++p) {
+                if (p & m) continue;
+                float2 x = b[col][p], y = b[col][p | m];
+                b[col][p] = bfly_add(x, y);
+                b[col][p | m] = bfly_sub(x, y);
+            }
+        }
+        // remaining bits l .. t: the partner run belongs to lane ^ (1 << sb)
+#pragma unroll
+        for (int sb = 0; sb < P::SHFL_BITS; ++sb) {
+            const float sg = ((r >> sb) & 1) ? -1.f : 1.f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int p = 0; p < L / 2; ++p) {
+                float2 mine = b[col][p];
+                float2 other;
+                other.x = __shfl_xor_sync(0xFFFFFFFFu, mine.x, 1 << sb);
+                other.y = __shfl_xor_sync(0xFFFFFFFFu, mine.y, 1 << sb);
+                b[col][p] = __ffma2_rn(mine, sg2, other);  // low: mine+other, high: other-mine
+            }
+        }
+    }
+
+    // ---- normalise and reduce max|z| over the team ----
+    const float2 rk2 = make_float2(rsqrt_k, rsqrt_k);
+    float mx = 0.f;
+#pragma unroll
+    for (int col = 0; col < P::COLS; ++col)
+#pragma unroll
+        for (int p = 0; p < L / 2; ++p) {
+            b[col][p] = __fmul2_rn(b[col][p], rk2);
+            mx = fmaxf(mx, fmaxf(fabsf(b[col][p].x), fabsf(b[col][p].y)));
+        }
+
+    if constexpr (ZOUT) {
+        if (valid) {
+            float *zr = zout + row * K;
+#pragma unroll
+            for (int col = 0; col < P::COLS; ++col) {
+                const int R = col * TEAM + r;
+#pragma unroll
+                for (int q = 0; q < L / 4; ++q)
+                    *reinterpret_cast<float4 *>(zr + R * L + 4 * q) =
+                        make_float4(b[col][2 * q].x, b[col][2 * q].y, b[col][2 * q + 1].x,
+                                    b[col][2 * q + 1].y);
+            }
+        }
+        return;
+    } else {
+        constexpr int W = TEAM < 32 ? TEAM : 32;
+#pragma unroll
+        for (int o = W / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        if constexpr (TEAM > 32) {
+            // all warps of this team finished their phase-B reads of tbuf before this barrier
+            if (lane == 0) red[team * 8 + (r >> 5)] = mx;
+            team_sync<TEAM>(team);
+            mx = red[team * 8];
+#pragma unroll
+            for (int i = 1; i < TEAM / 32; ++i) mx = fmaxf(mx, red[team * 8 + i]);
+        }
+        constexpr float Q = BITS == 4 ? 7.f : 127.f;
+        const float g = fmaxf(mx, 1e-5f);
+        const float s = __fdiv_rn(Q, g);
+        const float dq = __fdiv_rn(g, Q);
+        const float2 s2 = make_float2(s, s);
+        const float2 magic2 = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+
+        int sum = 0;
+#pragma unroll
+        for (int col = 0; col < P::COLS; ++col) {
+            const int R = col * TEAM + r;
+#pragma unroll
+            for (int g16 = 0; g16 < L / 16; ++g16) {
+                // 16 consecutive values -> round(z * s); the integer is the low byte of the
+                // float t + 1.5 * 2^23 (exact round-half-even for |t| < 2^22)
+                uint32_t f[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float2 t = __fmul2_rn(b[col][g16 * 8 + i], s2);
+                    float2 u = __fadd2_rn(t, magic2);
+                    f[2 * i] = __float_as_uint(u.x);
+                    f[2 * i + 1] = __float_as_uint(u.y);
+                }
+                const int64_t k0 = (int64_t)R * L + 16 * g16;
+                if constexpr (BITS == 8) {
+                    uint4 w;
+                    w.x = gather_low_bytes(f[0], f[1], f[2], f[3]);
+                    w.y = gather_low_bytes(f[4], f[5], f[6], f[7]);
+                    w.z = gather_low_bytes(f[8], f[9], f[10], f[11]);
+                    w.w = gather_low_bytes(f[12], f[13], f[14], f[15]);
+                    sum = __dp4a((int)w.x, 0x01010101, sum);
+                    sum = __dp4a((int)w.y, 0x01010101, sum);
+                    sum = __dp4a((int)w.z, 0x01010101, sum);
+                    sum = __dp4a((int)w.w, 0x01010101, sum);
+                    if (valid) *reinterpret_cast<uint4 *>(codes + row * K + k0) = w;
+                } else {
+                    uint32_t A0 = gather_low_bytes(f[0], f[1], f[2], f[3]);
+                    uint32_t B0 = gather_low_bytes(f[4], f[5], f[6], f[7]);
+                    uint32_t A1 = gather_low_bytes(f[8], f[9], f[10], f[11]);
+                    uint32_t B1 = gather_low_bytes(f[12], f[13], f[14], f[15]);
+                    sum = __dp4a((int)A0, 0x01010101, sum);
+                    sum = __dp4a((int)B0, 0x01010101, sum);
+                    sum = __dp4a((int)A1, 0x01010101, sum);
+                    sum = __dp4a((int)B1, 0x01010101, sum);
+                    uint2 w;
+                    w.x = (A0 & 0x0F0F0F0Fu) | ((B0 << 4) & 0xF0F0F0F0u);
+                    w.y = (A1 & 0x0F0F0F0Fu) | ((B1 << 4) & 0xF0F0F0F0u);
+                    if (valid) *reinterpret_cast<uint2 *>(codes + row * (K / 2) + k0 / 2) = w;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = W / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if constexpr (TEAM > 32) {
+            int *redi = reinterpret_cast<int *>(red) + 32;
+            if (lane == 0) redi[team * 8 + (r >> 5)] = sum;
+            team_sync<TEAM>(team);
+            sum = 0;
+#pragma unroll
+            for (int i = 0; i < TEAM / 32; ++i) sum += redi[team * 8 + i];
+        }
+        if (valid && r == 0) {
+            scales[row] = dq;
+            rowsum[row] = sum;
+        }
+    }
+}
+
+// ---- plain BitLinear: absmax quantisation without a transform (any K % 128 == 0) ----
+// One warp per token row, two passes over the row (the second one hits L1/L2).
+template <int BITS>
+__global__ void __launch_bounds__(256)
+    act_quant_plain_kernel(const uint4 *__restrict__ X, int64_t M, int64_t K,
+                           uint8_t *__restrict__ codes, float *__restrict__ scales,
+                           int32_t *__restrict__ rowsum) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (row >= M) return;  // whole warp leaves together
+    const uint4 *xr = X + row * (K / 8);
+    const int64_t nchunk = K / 8;
+    float mx = 0.f;
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        uint4 v = __ldg(xr + c);
+        const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            mx = fmaxf(mx, __uint_as_float((h[i] & 0x7FFFu) << 16));
+            mx = fmaxf(mx, __uint_as_float(h[i] & 0x7FFF0000u));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    constexpr float Q = BITS == 4 ? 7.f : 127.f;
+    const float g = fmaxf(mx, 1e-5f);
+    const float s = __fdiv_rn(Q, g);
+    const float dq = __fdiv_rn(g, Q);
+    const float2 s2 = make_float2(s, s);
+    const float2 magic2 = make_float2(12582912.f, 12582912.f);
+    int sum = 0;
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        uint4 v = __ldg(xr + c);
+        const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+        uint32_t f[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 x = make_float2(__uint_as_float(h[i] << 16), __uint_as_float(h[i] & 0xFFFF0000u));
+            float2 u = __fadd2_rn(__fmul2_rn(x, s2), magic2);
+            f[2 * i] = __float_as_uint(u.x);
+            f[2 * i + 1] = __float_as_uint(u.y);
+        }
+        uint32_t A = gather_low_bytes(f[0], f[1], f[2], f[3]);
+        uint32_t B = gather_low_bytes(f[4], f[5], f[6], f[7]);
+        sum = __dp4a((int)A, 0x01010101, sum);
+        sum = __dp4a((int)B, 0x01010101, sum);
+        if constexpr (BITS == 8) {
+            *reinterpret_cast<uint2 *>(codes + row * K + 8 * c) = make_uint2(A, B);
+        } else {
+            *reinterpret_cast<uint32_t *>(codes + row * (K / 2) + 4 * c) =
+                (A & 0x0F0F0F0Fu) | ((B << 4) & 0xF0F0F0F0u);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane == 0) {
+        scales[row] = dq;
+        rowsum[row] = sum;
+    }
+}
+
+template <int LOGK, int BITS, bool ZOUT>
+static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *scales,
+                                 int32_t *rowsum, float *zout, cudaStream_t stream) {
+    using P = FwhtPlan<LOGK>;
+    auto kern = fwht_quant_kernel<LOGK, BITS, ZOUT>;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)P::SMEM);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    const int64_t blocks = (M + P::TEAMS - 1) / P::TEAMS;
+    const float rk = (float)(1.0 / sqrt((double)P::K));
+    kern<<<(unsigned)blocks, P::THREADS, P::SMEM, stream>>>(
+        reinterpret_cast<const uint32_t *>(X), (int)M, rk, reinterpret_cast<uint8_t *>(codes),
+        scales, rowsum, zout);
+    return cudaGetLastError();
+}
+
+template <int LOGK>
+static cudaError_t launch_fwht_k(const void *X, int64_t M, int act_bits, void *codes,
+                                 float *scales, int32_t *rowsum, float *zout,
+                                 cudaStream_t stream) {
+    if (zout) return launch_fwht_t<LOGK, 8, true>(X, M, codes, scales, rowsum, zout, stream);
+    if (act_bits == 4)
+        return launch_fwht_t<LOGK, 4, false>(X, M, codes, scales, rowsum, zout, stream);
+    return launch_fwht_t<LOGK, 8, false>(X, M, codes, scales, rowsum, zout, stream);
+}
+
+cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
+                              float *scales, int32_t *rowsum, float *zout, cudaStream_t stream) {
+    switch (logk) {
+        case 7: return launch_fwht_k<7>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 8: return launch_fwht_k<8>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 9: return launch_fwht_k<9>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 10: return launch_fwht_k<10>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 11: return launch_fwht_k<11>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 12: return launch_fwht_k<12>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 13: return launch_fwht_k<13>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 14: return launch_fwht_k<14>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 15: return launch_fwht_k<15>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
+                                   void *codes, float *scales, int32_t *rowsum,
+                                   cudaStream_t stream) {
+    const int64_t blocks = (M + 7) / 8;
+    if (act_bits == 4)
+        act_quant_plain_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(
+            reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<uint8_t *>(codes),
+            scales, rowsum);
+    else
+        act_quant_plain_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(
+            reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<uint8_t *>(codes),
+            scales, rowsum);
+    return cudaGetLastError();
+}
+
+}  // namespace bitnet

@@ -1,0 +1,49 @@
+// kernels.h -- internal launchers of libbitnet_b200.so (not part of the C ABI).
+// Every launcher enqueues on `stream` and returns the cudaError_t of its launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bitnet {
+
+// ---- step 1: weights (weights.cu) ----
+int absmean_num_partials(int64_t n);
+cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, int P,
+                                    cudaStream_t stream);
+cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partials, int P,
+                                  uint32_t *Wp, float *gamma, cudaStream_t stream);
+
+// ---- steps 2-3: activations (actquant.cu) ----
+// Hadamard + quantise (or z output when zout != nullptr).  K = 2^logk, 7 <= logk <= 15.
+cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
+                              float *scales, int32_t *rowsum, float *zout, cudaStream_t stream);
+// Quantise without a transform; K % 128 == 0.
+cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
+                                   void *codes, float *scales, int32_t *rowsum,
+                                   cudaStream_t stream);
+
+// ---- step 4: product (gemv.cu, gemm_tc.cu) ----
+struct GemmArgs {
+    const void *codes;      // int8 [M][K] or packed int4 [M][K/2]
+    const float *scales;    // [M]
+    const int32_t *rowsum;  // [M]
+    const uint32_t *Wp;     // [N][K/16]
+    const float *gamma;     // [1]
+    int64_t M, N, K;
+    int act_bits;
+    int32_t *acc;           // optional int32 [M][N]
+    void *Y;                // optional bf16 [M][N]
+    int *status;            // device status word
+};
+
+// Weight-streaming kernel for few tokens (decode).
+constexpr int kGemvMaxTokens = 8;
+cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream);
+
+// tcgen05 tensor-core kernel (prefill).  encode is cuTensorMapEncodeTiled.
+cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
+                                   cudaStream_t stream);
+
+}  // namespace bitnet

@@ -1,0 +1,121 @@
+// weights.cu -- step 1 of the forward: absmean ternarisation of the latent weights and their
+// 2-bit packing.
+//
+// absmean ("The Era of 1-bit LLMs" summary page, sections 方法论 and 方法详解; BitNet b1.58 2B4T
+// article, section 一.2): one scale per tensor, gamma = mean |W|; every weight becomes
+// RoundClip(w / gamma, -1, 1).  The pages print no formula; the readings used here are
+// gamma = fp32(max(mean, 1e-5)) with the mean in double, an IEEE fp32 division and
+// round-half-to-even.
+//
+// Two launches, both HBM-bound streams over W (2 bytes per weight):
+//   absmean_partials_kernel  fixed grid of P blocks (P depends only on the weight count), each
+//                            sums |w| in fp64 over a fixed grid-stride subset and writes one
+//                            partial; the reduction tree is fixed, so gamma is deterministic.
+//   ternarize_pack_kernel    every block first sums the P partials in a fixed order (2.4 KB,
+//                            L2-resident), so no third launch or atomic is needed; then each
+//                            thread turns 16 weights into one packed 32-bit word.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bitnet {
+
+constexpr int kWeightThreads = 256;
+constexpr int kMaxPartials = 1184;  // 8 blocks per SM on 148 SMs
+
+int absmean_num_partials(int64_t n) {
+    int64_t vec = n / 8;  // 16-byte vectors of 8 bf16
+    int64_t p = (vec + kWeightThreads * 4 - 1) / (kWeightThreads * 4);
+    if (p < 1) p = 1;
+    if (p > kMaxPartials) p = kMaxPartials;
+    return (int)p;
+}
+
+__device__ __forceinline__ double abs_bf16_pair_sum(uint32_t w) {
+    // |bf16| is the bit pattern with the sign cleared; widening to fp32 is exact.
+    float lo = __uint_as_float((w & 0x7FFFu) << 16);
+    float hi = __uint_as_float(w & 0x7FFF0000u);
+    return (double)lo + (double)hi;
+}
+
+__global__ void __launch_bounds__(kWeightThreads)
+    absmean_partials_kernel(const uint4 *__restrict__ w, int64_t nvec,
+                            double *__restrict__ partials) {
+    double acc0 = 0.0, acc1 = 0.0;
+    const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nvec; i += stride) {
+        uint4 v = ldg_nc_v4(w + i);
+        acc0 += abs_bf16_pair_sum(v.x);
+        acc1 += abs_bf16_pair_sum(v.y);
+        acc0 += abs_bf16_pair_sum(v.z);
+        acc1 += abs_bf16_pair_sum(v.w);
+    }
+    double s = acc0 + acc1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    __shared__ double warp_sums[kWeightThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int i = 0; i < kWeightThreads / 32; ++i) t += warp_sums[i];
+        partials[blockIdx.x] = t;
+    }
+}
+
+__global__ void __launch_bounds__(kWeightThreads)
+    ternarize_pack_kernel(const uint4 *__restrict__ w, int64_t nwords, double n_weights,
+                          const double *__restrict__ partials, int P, uint32_t *__restrict__ wp,
+                          float *__restrict__ gamma_out) {
+    __shared__ float s_gamma;
+    if (threadIdx.x < 32) {
+        double s = 0.0;
+        for (int i = threadIdx.x; i < P; i += 32) s += partials[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        if (threadIdx.x == 0) {
+            double mean = s / n_weights;
+            float g = (float)fmax(mean, 1e-5);
+            s_gamma = g;
+            if (blockIdx.x == 0) *gamma_out = g;
+        }
+    }
+    __syncthreads();
+    const float g = s_gamma;
+    const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nwords; i += stride) {
+        // 16 consecutive weights k = 16i + e; weight e = 4p + j goes to bits 8j + 2p as u = q + 1.
+        uint4 a = ldg_nc_v4(w + 2 * i);
+        uint4 b = ldg_nc_v4(w + 2 * i + 1);
+        const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            uint32_t bits = (e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16);
+            float r = __fdiv_rn(__uint_as_float(bits), g);
+            // clip(rint(r), -1, 1) with ties to even: |r| <= 0.5 gives 0, otherwise sign(r).
+            uint32_t u = r > 0.5f ? 2u : (r < -0.5f ? 0u : 1u);
+            word |= u << (8 * (e & 3) + 2 * (e >> 2));
+        }
+        wp[i] = word;
+    }
+}
+
+cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, int P,
+                                    cudaStream_t stream) {
+    absmean_partials_kernel<<<P, kWeightThreads, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(W), n / 8, partials);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partials, int P,
+                                  uint32_t *Wp, float *gamma, cudaStream_t stream) {
+    int64_t nwords = n / 16;
+    int64_t blocks = (nwords + kWeightThreads - 1) / kWeightThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    ternarize_pack_kernel<<<(unsigned)blocks, kWeightThreads, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(W), nwords, (double)n, partials, P, Wp, gamma);
+    return cudaGetLastError();
+}
+
+}  // namespace bitnet

@@ -1,0 +1,173 @@
+/*
+ * bitnet.h -- C ABI of libbitnet_b200.so: the BitLinear / H-BitLinear forward (BitNet b1.58,
+ * BitNet v2) on one NVIDIA B200 (sm_100a).
+ *
+ * The forward has four steps:
+ *   1. the latent weights W are ternarised with absmean (one scale gamma = mean|W| per tensor)
+ *      and packed two bits per weight        ["The Era of 1-bit LLMs" summary page,
+ *                                              sections 方法论 and 方法详解; BitNet b1.58 2B4T
+ *                                              article, section 一.2 (BitLinear, W1.58A8)];
+ *   2. in H-BitLinear every token row gets an online Hadamard transform  [BitNet v2 write-up,
+ *      paragraphs on H-BitLinear; BitNet v2 abstract];
+ *   3. every token row is quantised with absmax to INT8 (or INT4)  [2B4T article, 一.2;
+ *      BitNet v2 write-up, 8-bit / 4-bit activation paragraph];
+ *   4. a ternary x integer product accumulates in int32 and is rescaled to bf16
+ *      [2B4T article, 一.2: multiplying by 1 adds, by -1 subtracts, by 0 skips].
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named *_dev are device pointers the caller owns; the library never allocates,
+ *     frees or keeps them.  Every device pointer must be 16-byte aligned.
+ *   - Matrices are row-major.  X and Y are bf16 (passed as void*), W is bf16.
+ *   - Calls are asynchronous on `stream` (0 = the legacy default stream).  A return value of
+ *     BITNET_OK means the work was enqueued.  Any other return means nothing was launched,
+ *     except BITNET_ERR_CUDA (a launch failed part-way).  Faults of kernels that already ran,
+ *     and device-side wait time-outs, are reported by bitnet_sync_status().
+ *   - Shape rules: M >= 1 tokens; K >= 128 input features with K % 128 == 0; N >= 8 output
+ *     features with N % 8 == 0.  H-BitLinear also needs K to be a power of two, 128..32768
+ *     (else BITNET_ERR_UNSUPPORTED).  act_bits is 8 or 4.
+ *   - bitnet_last_error() returns a text description of the last failure on this host thread.
+ */
+#ifndef BITNET_B200_H
+#define BITNET_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA headers. */
+typedef struct CUstream_st *bitnet_stream_t;
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID = -1,     /* null or misaligned pointer, bad size, bad act_bits */
+    BITNET_ERR_UNSUPPORTED = -2, /* valid arguments the library does not handle (e.g. K not a
+                                    power of two for H-BitLinear, not an sm_100 device) */
+    BITNET_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
+    BITNET_ERR_TIMEOUT = -4,     /* a kernel gave up a bounded device-side wait (reported by
+                                    bitnet_sync_status) */
+    BITNET_ERR_WORKSPACE = -5    /* workspace smaller than the size query returned */
+} bitnet_status;
+
+/* Text for a status code (static storage). */
+const char *bitnet_status_string(int status);
+
+/* Detail of the last failure returned on the calling host thread (thread-local storage). */
+const char *bitnet_last_error(void);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Step 1: weight ternarisation and packing                                                  */
+/* ---------------------------------------------------------------------------------------- */
+
+/* Bytes of packed weights for an [N, K] matrix: N * K / 4. */
+size_t bitnet_packed_weight_bytes(int64_t N, int64_t K);
+
+/* Bytes of device workspace bitnet_quantize_pack_weights needs (partial sums of |w|). */
+size_t bitnet_weight_workspace_bytes(int64_t N, int64_t K);
+
+/*
+ * absmean ternarisation ["The Era of 1-bit LLMs" summary, 方法论 / 方法详解]:
+ *   gamma = fp32(max(mean |W|, 1e-5)), the mean taken in double over all N*K weights in a
+ *   fixed order (the result does not depend on the launch);
+ *   q = clip(round_half_even(w / gamma), -1, 1), the division IEEE fp32.
+ * W_dev     bf16 [N, K] latent weights (read only).
+ * Wp_dev    out: packed weights, N*K/4 bytes.  Row n is K/16 little-endian 32-bit words; word
+ *           g holds k = 16g .. 16g+15 as offset codes u = q + 1 in {0, 1, 2}, weight
+ *           k = 16g + 4p + j (p, j in 0..3) at bits 8j + 2p.
+ * gamma_dev out: one float.
+ * ws_dev    scratch of ws_bytes >= bitnet_weight_workspace_bytes(N, K); contents undefined
+ *           afterwards.
+ */
+int bitnet_quantize_pack_weights(const void *W_dev, int64_t N, int64_t K, void *Wp_dev,
+                                 float *gamma_dev, void *ws_dev, size_t ws_bytes,
+                                 bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Steps 2 and 3: online Hadamard transform and per-token activation quantisation            */
+/* ---------------------------------------------------------------------------------------- */
+
+/* Bytes of activation codes for M tokens: M*K (INT8) or M*K/2 (INT4). */
+size_t bitnet_act_codes_bytes(int64_t M, int64_t K, int act_bits);
+
+/*
+ * Per token row m (BitNet v2 write-up, H-BitLinear; 2B4T article, 一.2):
+ *   z = (1/sqrt(K)) H_K x  when hadamard != 0 (H_K in Sylvester order, H_2n = [[H,H],[H,-H]],
+ *       computed in fp32 by a fast Walsh-Hadamard transform), else z = x;
+ *   mx = max(max_k |z_k|, 1e-5); s = Q / mx (IEEE fp32); codes = round_half_even(z * s),
+ *   Q = 127 (act_bits 8) or 7 (act_bits 4);  scales[m] = mx / Q;  rowsum[m] = sum_k codes.
+ * X_dev       bf16 [M, K].
+ * codes_dev   out: int8 [M, K] (act_bits 8) or [M, K/2] bytes (act_bits 4: every 8 codes
+ *             k0..k0+7 fill 4 bytes, byte j = code k0+j in the low nibble and k0+4+j in the
+ *             high nibble, two's complement).
+ * scales_dev  out: float [M], the dequantisation step of each token.
+ * rowsum_dev  out: int32 [M], the sum of each token's codes (used by the product kernels to
+ *             remove the +1 offset of the stored weight codes).
+ */
+int bitnet_act_quant(const void *X_dev, int64_t M, int64_t K, int hadamard, int act_bits,
+                     void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
+                     bitnet_stream_t stream);
+
+/* Debug / parity entry: Z = (1/sqrt(K)) H_K X per row in fp32, X bf16 [M, K], Z float [M, K].
+ * Same transform code as bitnet_act_quant. */
+int bitnet_fwht_f32(const void *X_dev, int64_t M, int64_t K, float *Z_dev,
+                    bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Step 4: ternary x integer product and rescale                                             */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * acc[m, n] = sum_k codes[m, k] * q[n, k]            (exact, int32)
+ * Y[m, n]   = bf16_rn(float(acc[m, n]) * (scales[m] * gamma))   (fp32 product)
+ * codes/scales/rowsum as written by bitnet_act_quant; Wp/gamma as written by
+ * bitnet_quantize_pack_weights.  acc_dev (int32 [M, N]) and Y_dev (bf16 [M, N]) are each
+ * optional (NULL to skip); at least one must be given.  Large M runs on the tcgen05 tensor
+ * cores, small M (decode) on a weight-streaming kernel; both give the same integers.
+ */
+int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
+                        const int32_t *rowsum_dev, int64_t M, int64_t K, const void *Wp_dev,
+                        const float *gamma_dev, int64_t N, int act_bits, int32_t *acc_dev,
+                        void *Y_dev, bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* The whole layer                                                                          */
+/* ---------------------------------------------------------------------------------------- */
+
+/* Bytes of workspace the two forward calls need: codes + scales + rowsums, 256-byte aligned. */
+size_t bitnet_workspace_bytes(int64_t M, int64_t K, int64_t N, int act_bits);
+
+/*
+ * Y = BitLinear(X): per-token absmax quantisation of X (no transform), then the ternary
+ * product with Wp and the rescale to bf16.  X_dev bf16 [M, K], Y_dev bf16 [M, N],
+ * ws_dev scratch of ws_bytes >= bitnet_workspace_bytes(M, K, N, act_bits).
+ */
+int bitnet_bitlinear_forward(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                             const float *gamma_dev, int64_t N, int act_bits, void *Y_dev,
+                             void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
+
+/* Y = H-BitLinear(X): as bitnet_bitlinear_forward with the online Hadamard transform before
+ * the quantisation (BitNet v2 write-up: used for the attention output projection Wo and the
+ * FFN down projection Wdown).  K must be a power of two. */
+int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                              const float *gamma_dev, int64_t N, int act_bits, void *Y_dev,
+                              void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Status                                                                                   */
+/* ---------------------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then returns BITNET_ERR_CUDA if the stream reported a fault,
+ * BITNET_ERR_TIMEOUT if a kernel of this library on the current device gave up a bounded
+ * wait since the last call (the flag is cleared), else BITNET_OK. */
+int bitnet_sync_status(bitnet_stream_t stream);
+
+/* Number of kernel launches this library has issued in this process (all devices). */
+uint64_t bitnet_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_B200_H */

@@ -1,0 +1,110 @@
+"""The C-ABI library loads and exports what include/bitnet.h declares (no GPU needed).
+
+Only calls that never reach the device run here: size queries, status strings and the argument
+checks that reject a call before any CUDA work.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_activation_linear_b200 import build, binding
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("bitnet_quantize_pack_weights", "bitnet_bitlinear_forward",
+                     "bitnet_hbitlinear_forward", "bitnet_act_quant", "bitnet_fwht_f32",
+                     "bitnet_ternary_gemm", "bitnet_sync_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from bit_activation_linear_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (bitnet_[a-z0-9_]+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # the binding wraps every exported entry point under the same name
+    for name in declared_functions():
+        assert name in binding.EXPORTED
+
+
+def test_library_targets_sm100a_only():
+    from bit_activation_linear_b200 import binding
+    out = subprocess.run(["cuobjdump", "--list-elf", binding.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    assert "sm_100a" in out
+    assert not re.search(r"sm_(?!100a)\d+", out)
+
+
+def test_size_queries(lib):
+    assert lib.bitnet_packed_weight_bytes(2048, 2048) == 2048 * 2048 // 4
+    assert lib.bitnet_act_codes_bytes(16, 256, 8) == 16 * 256
+    assert lib.bitnet_act_codes_bytes(16, 256, 4) == 16 * 128
+    ws = lib.bitnet_workspace_bytes(4096, 2048, 2048, 8)
+    assert ws >= 4096 * 2048 + 2 * 4096 * 4 and ws % 256 == 0
+    assert lib.bitnet_weight_workspace_bytes(2048, 2048) % 256 == 0
+    assert lib.bitnet_weight_workspace_bytes(2048, 2048) >= 8
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert lib.bitnet_status_string(code).decode()
+    assert lib.bitnet_status_string(0).decode() == "ok"
+
+
+@pytest.mark.parametrize("M,K,N,bits", [
+    (0, 256, 256, 8),      # no tokens
+    (16, 100, 256, 8),     # K not a multiple of 128
+    (16, 256, 12, 8),      # N not a multiple of 8
+    (16, 256, 256, 5),     # act_bits
+])
+def test_forward_rejects_bad_shapes_before_touching_the_device(lib, M, K, N, bits):
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the call must fail in the host check
+    rc = lib.bitnet_hbitlinear_forward(fake, M, K, fake, fake, N, bits, fake, fake, 1 << 30, None)
+    assert rc == -1
+    assert lib.bitnet_last_error().decode()
+
+
+def test_forward_rejects_null_and_misaligned_pointers(lib):
+    good = ctypes.c_void_p(1 << 20)
+    rc = lib.bitnet_bitlinear_forward(None, 16, 256, good, good, 256, 8, good, good, 1 << 30, None)
+    assert rc == -1
+    bad = ctypes.c_void_p((1 << 20) + 4)
+    rc = lib.bitnet_bitlinear_forward(bad, 16, 256, good, good, 256, 8, good, good, 1 << 30, None)
+    assert rc == -1
+    assert "aligned" in lib.bitnet_last_error().decode()
+
+
+def test_forward_rejects_small_workspace(lib):
+    good = ctypes.c_void_p(1 << 20)
+    rc = lib.bitnet_hbitlinear_forward(good, 16, 256, good, good, 256, 8, good, good, 64, None)
+    assert rc == -5
+
+
+def test_binding_raises_without_library(tmp_path):
+    from bit_activation_linear_b200 import binding
+    code = ("import bit_activation_linear_b200.binding as b\n"
+            f"try:\n    b.load_library({str(tmp_path / 'missing.so')!r})\n"
+            "except RuntimeError as e:\n    print('raised', 'no fallback' in str(e).lower())\n")
+    out = subprocess.run(["python", "-c", code], capture_output=True, text=True, cwd=ROOT)
+    assert "raised True" in out.stdout, out.stdout + out.stderr

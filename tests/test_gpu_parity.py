@@ -1,0 +1,226 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle, through the C ABI.
+
+Tolerances (written here, from the contract of the forward):
+  * packed weights and gamma: bit-exact;
+  * Hadamard output (fp32): per row, max|z - z_ref| <= 1e-5 * max|z_ref|;
+  * activation codes: a code may differ by +-1 only where the oracle's unrounded value lies
+    within 1e-4 of a .5 boundary, and on at most 1e-4 of the codes;
+  * int32 accumulators: bit-exact against the oracle fed the same codes;
+  * bf16 output: elementwise relative error <= 1e-2 against the oracle fed the same codes, and
+    ||Y - Y_ref||_F / ||Y_ref||_F <= 1e-2 against the fully independent oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_activation_linear_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+CODE_BOUNDARY = 1e-4
+CODE_FRACTION = 1e-4
+FWHT_REL = 1e-5
+Y_REL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def B():
+    from bit_activation_linear_b200 import build, binding
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    binding.load_library()
+    return binding
+
+
+def dev_bf16(bits):
+    return synth.to_torch_bf16(bits).cuda()
+
+
+def to_np_bits(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_codes(codes_gpu, codes_ref, pre):
+    diff = codes_gpu.astype(np.int32) - codes_ref.astype(np.int32)
+    bad = diff != 0
+    if bad.any():
+        assert np.abs(diff).max() <= 1
+        dist = np.abs(np.abs(pre[bad] - np.floor(pre[bad])) - 0.5)
+        assert np.all(dist < CODE_BOUNDARY), dist.max()
+        assert bad.mean() <= CODE_FRACTION
+    return int(bad.sum())
+
+
+# ----------------------------------------------------------------------------------------
+# step 1: weights
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(256, 256), (8, 128), (264, 384), (2048, 2048), (2048, 8192)])
+def test_weights_bit_exact(B, N, K):
+    W = synth.latent_weights(N, K, seed=N + K)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    B.bitnet_sync_status()
+    g_ref = oracle.absmean_gamma(W)
+    assert np.float32(gamma.item()) == g_ref
+    ref = oracle.pack_ternary(oracle.ternarize(W, g_ref))
+    np.testing.assert_array_equal(Wp.cpu().numpy().view(np.uint32).reshape(N, K // 16), ref)
+
+
+def test_weights_degenerate(B):
+    Z = np.zeros((16, 128), np.uint16)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(Z))
+    assert np.float32(gamma.item()) == np.float32(1e-5)
+    q, bad = oracle.unpack_ternary(Wp.cpu().numpy().view(np.uint32), 128)
+    assert bad == 0 and not q.any()
+
+
+# ----------------------------------------------------------------------------------------
+# steps 2-3: Hadamard transform and quantisation
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K", [128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768])
+def test_fwht_matches_oracle(B, K):
+    M = 37 if K <= 8192 else 9
+    X = synth.sharp_activations(M, K, seed=K)
+    Z = B.bitnet_fwht_f32(dev_bf16(X)).cpu().numpy().astype(np.float64)
+    ref = oracle.fwht(oracle.bf16_to_f64(X))
+    err = np.abs(Z - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert err.max() <= FWHT_REL, err.max()
+
+
+@pytest.mark.parametrize("K", [128, 256, 2048, 8192, 16384])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_hadamard_quant_codes(B, K, bits):
+    M = 45 if K <= 8192 else 11
+    X = synth.sharp_activations(M, K, seed=3 * K + bits)
+    Xd = dev_bf16(X)
+    z = B.bitnet_fwht_f32(Xd).cpu().numpy()
+    codes, scales, rowsum = B.bitnet_act_quant(Xd, True, bits)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
+    c = codes.cpu().numpy()
+    c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+    check_codes(c, c_ref, pre)
+    np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), c.astype(np.int64).sum(axis=1))
+
+
+@pytest.mark.parametrize("K", [128, 640, 4096])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_plain_quant_codes_exact(B, K, bits):
+    M = 21
+    X = synth.gaussian_activations(M, K, seed=K + bits)
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), False, bits)
+    z = oracle.bf16_to_f64(X).astype(np.float32)
+    c_ref, d_ref, _, rs_ref = oracle.quant_act(z, bits)
+    c = codes.cpu().numpy()
+    c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+    np.testing.assert_array_equal(c, c_ref)
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
+
+
+def test_quant_zero_rows(B):
+    X = np.zeros((5, 256), np.uint16)
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), True, 8)
+    assert not codes.cpu().numpy().any()
+    assert np.all(scales.cpu().numpy() == np.float32(np.float32(1e-5) / np.float32(127)))
+    assert not rowsum.cpu().numpy().any()
+
+
+# ----------------------------------------------------------------------------------------
+# step 4: product, staged on the GPU's own codes
+# ----------------------------------------------------------------------------------------
+
+def staged_product(B, M, K, N, bits, seed):
+    X = synth.sharp_activations(M, K, seed=seed)
+    W = synth.latent_weights(N, K, seed=seed + 1)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), True, bits)
+    acc, Y = B.bitnet_ternary_gemm(codes, scales, rowsum, K, Wp, gamma, bits, want_acc=True,
+                                   want_y=True)
+    B.bitnet_sync_status()
+    c = codes.cpu().numpy()
+    c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+    q, bad = oracle.unpack_ternary(Wp.cpu().numpy().view(np.uint32), K)
+    assert bad == 0
+    return c, q, scales.cpu().numpy(), np.float32(gamma.item()), acc.cpu().numpy(), Y
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (1, 256, 256), (3, 384, 136), (8, 2048, 264),          # decode kernel
+    (9, 256, 256), (130, 384, 136), (300, 2048, 264),       # tensor-core kernel, ragged tiles
+    (256, 1024, 1024), (513, 128, 8),
+])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_product_int32_exact_and_bf16(B, M, K, N, bits):
+    c, q, d, gamma, acc, Y = staged_product(B, M, K, N, bits, seed=M * 7 + N)
+    acc_ref = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(acc.astype(np.int64), acc_ref)
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc_ref, d, gamma))
+    y = oracle.bf16_to_f64(to_np_bits(Y))
+    rel = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), 1e-30)
+    assert np.all((rel <= Y_REL) | (y_ref == 0)), rel.max()
+    assert np.all(y[y_ref == 0] == 0)
+
+
+# ----------------------------------------------------------------------------------------
+# the whole layer against the independent oracle, on every workload shape
+# ----------------------------------------------------------------------------------------
+
+def forward_case(B, wl, sample_rows, seed=0):
+    X = wl.activations(seed=seed)
+    W = wl.weights(seed=seed)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    fwd = B.bitnet_hbitlinear_forward if wl.hadamard else B.bitnet_bitlinear_forward
+    Y = fwd(dev_bf16(X), Wp, gamma, wl.act_bits)
+    B.bitnet_sync_status()
+    rows = np.arange(wl.M) if sample_rows is None else np.sort(
+        np.random.default_rng(seed).choice(wl.M, size=sample_rows, replace=False))
+    ref = oracle.bitlinear_forward(X[rows], W, wl.hadamard, wl.act_bits)
+    assert np.float32(gamma.item()) == ref["gamma"]
+    y = oracle.bf16_to_f64(to_np_bits(Y)[rows])
+    y_ref = oracle.bf16_to_f64(ref["y"])
+    fro = np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref)
+    assert fro <= Y_REL, fro
+    return fro
+
+
+@pytest.mark.parametrize("name,rows", [
+    ("tiny", None),
+    ("wo_2048", 64),
+    ("wdown_8192", 24),
+    ("decode_m1_k8192", None), ("decode_m8_k8192", None), ("decode_m32_k8192", None),
+    ("decode_m64_k8192", None), ("decode_m1_k2048", None), ("decode_m64_k2048", None),
+])
+def test_forward_end_to_end(B, name, rows):
+    forward_case(B, synth.WORKLOADS[name], rows)
+
+
+@pytest.mark.parametrize("name,rows", [("down_7b", 6), ("up_7b", 8)])
+def test_forward_end_to_end_7b(B, name, rows):
+    forward_case(B, synth.WORKLOADS[name], rows)
+
+
+def test_forward_equals_staged_calls(B):
+    wl = synth.WORKLOADS["wo_2048"]
+    X = dev_bf16(wl.activations(rows=640))
+    W = dev_bf16(wl.weights())
+    Wp, gamma = B.bitnet_quantize_pack_weights(W)
+    Y = B.bitnet_hbitlinear_forward(X, Wp, gamma, 8)
+    codes, scales, rowsum = B.bitnet_act_quant(X, True, 8)
+    _, Y2 = B.bitnet_ternary_gemm(codes, scales, rowsum, wl.K, Wp, gamma, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_errors_are_reported(B):
+    X = torch.zeros((4, 384), dtype=torch.bfloat16, device="cuda")
+    Wp = torch.zeros((8, 96), dtype=torch.uint8, device="cuda")
+    gamma = torch.ones(1, device="cuda")
+    with pytest.raises(B.BitnetError) as e:
+        B.bitnet_hbitlinear_forward(X, Wp, gamma, 8)  # 384 is not a power of two
+    assert e.value.status == B.ERR_UNSUPPORTED
+    Y = B.bitnet_bitlinear_forward(X, Wp, gamma, 8)  # fine without the transform
+    B.bitnet_sync_status()
+    assert not Y.float().abs().sum().item()

@@ -258,7 +258,8 @@ def run_gpu(args, wl, rank, world, device):
         gamma = torch.empty(1, dtype=torch.float32, device=device)
         wws = torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
                           device=device)
-        codes = torch.empty(code_bytes, dtype=torch.uint8, device=device)
+        codes = torch.empty((M, K if wl.act_bits == 8 else K // 2), dtype=torch.uint8,
+                            device=device)
         scales = torch.empty(M, dtype=torch.float32, device=device)
         rowsum = torch.empty(M, dtype=torch.int32, device=device)
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)

@@ -107,6 +107,12 @@ def _check(t: torch.Tensor, name: str, dtype=None, dim=None):
         raise ValueError(f"{name} must have {dim} dimensions")
 
 
+def _nbytes_at_least(t: torch.Tensor, need: int, name: str):
+    have = t.numel() * t.element_size()
+    if have < need:
+        raise ValueError(f"{name} holds {have} bytes, {need} needed")
+
+
 def _rc(status: int, where: str):
     if status != OK:
         raise BitnetError(status, where)
@@ -141,6 +147,7 @@ def bitnet_quantize_pack_weights(W: torch.Tensor, Wp: torch.Tensor | None = None
     N, K = W.shape
     if Wp is None:
         Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
     if gamma is None:
         gamma = torch.empty(1, dtype=torch.float32, device=W.device)
     need = int(L.bitnet_weight_workspace_bytes(N, K))
@@ -165,6 +172,9 @@ def bitnet_act_quant(X: torch.Tensor, hadamard: bool, act_bits: int, codes=None,
         scales = torch.empty(M, dtype=torch.float32, device=X.device)
     if rowsum is None:
         rowsum = torch.empty(M, dtype=torch.int32, device=X.device)
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, act_bits)), "codes")
+    _nbytes_at_least(scales, 4 * M, "scales")
+    _nbytes_at_least(rowsum, 4 * M, "rowsum")
     _rc(L.bitnet_act_quant(X.data_ptr(), M, K, int(bool(hadamard)), int(act_bits),
                            codes.data_ptr(), scales.data_ptr(), rowsum.data_ptr(),
                            _stream(stream)), "bitnet_act_quant")
@@ -190,8 +200,11 @@ def bitnet_ternary_gemm(codes: torch.Tensor, scales: torch.Tensor, rowsum: torch
     for t, n in ((codes, "codes"), (scales, "scales"), (rowsum, "rowsum"), (Wp, "Wp"),
                  (gamma, "gamma")):
         _check(t, n)
-    M = codes.shape[0]
+    M = scales.numel()
     N = Wp.shape[0]
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, act_bits)), "codes")
+    _nbytes_at_least(rowsum, 4 * M, "rowsum")
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
     if want_acc and acc is None:
         acc = torch.empty((M, N), dtype=torch.int32, device=codes.device)
     if want_y and Y is None:
@@ -211,8 +224,10 @@ def _forward(fn_name: str, X, Wp, gamma, act_bits, Y, ws, stream):
     _check(gamma, "gamma", torch.float32)
     M, K = X.shape
     N = Wp.shape[0]
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _nbytes_at_least(Y, 2 * M * N, "Y")
     need = int(L.bitnet_workspace_bytes(M, K, N, act_bits))
     if ws is None:
         ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)

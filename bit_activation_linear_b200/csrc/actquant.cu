@@ -23,7 +23,9 @@
 //   Quantise every thread holds contiguous runs, so codes are packed in registers (float
 //            round-to-int by adding 1.5 * 2^23, byte gather with prmt) and written with 16-byte
 //            stores; the team reduces max|z| and the code sum.
-// Butterflies use the packed fp32x2 add/fma of sm_100.
+// Butterflies use the packed fp32x2 add/fma of sm_100.  The product that decides a code is a
+// scalar __fmul_rn, which the compiler never fuses with the rounding add that follows (the
+// packed forms give no such guarantee: a fused multiply-add rounds once and moves near-ties).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -51,7 +53,7 @@ struct FwhtPlan {
     static_assert(L >= 16, "runs must hold 16 codes");
 };
 
-__device__ __forceinline__ float2 bfly_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 bfly_add(float2 a, float2 b) { return add2_rn(a, b); }
 __device__ __forceinline__ float2 bfly_sub(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a - b, one rounding
 }
@@ -78,21 +80,30 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
     const int team = threadIdx.x / TEAM;
     const int r = threadIdx.x % TEAM;
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * P::TEAMS + team;
-    const bool valid = row < M;
     float *tbuf = smem + team * K;
     float *red = smem + P::TEAMS * K;  // 64 floats of reduction scratch
+    const int64_t stride = (int64_t)gridDim.x * P::TEAMS;
 
-    // ---- phase A: load bf16 pairs, butterflies over register bits ----
-    float2 a[V / 2];
-    {
-        const uint32_t *xr = X + row * (K / 2);
+    // Persistent: the team walks rows base + team, base += stride.  The trip count is the same
+    // for every team of the CTA (teams of <= 32 threads share a warp and its __syncwarp).  The
+    // next row's bf16 pairs are loaded while the current row is transformed.
+    uint32_t raw[V / 2];
+    auto load_row = [&](int64_t rw) {
+        const uint32_t *xr = X + rw * (K / 2);
 #pragma unroll
-        for (int c = 0; c < V / 2; ++c) {
-            uint32_t w = valid ? __ldg(xr + c * TEAM + r) : 0u;
-            a[c] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-        }
-    }
+        for (int c = 0; c < V / 2; ++c) raw[c] = rw < M ? __ldg(xr + c * TEAM + r) : 0u;
+    };
+    load_row((int64_t)blockIdx.x * P::TEAMS + team);
+    for (int64_t base = (int64_t)blockIdx.x * P::TEAMS; base < M; base += stride) {
+    const int64_t row = base + team;
+    const bool valid = row < M;
+
+    // ---- phase A: bf16 pairs -> fp32, butterflies over register bits ----
+    float2 a[V / 2];
+#pragma unroll
+    for (int c = 0; c < V / 2; ++c)
+        a[c] = make_float2(__uint_as_float(raw[c] << 16), __uint_as_float(raw[c] & 0xFFFF0000u));
+    load_row(row + stride);
 #pragma unroll
     for (int c = 0; c < V / 2; ++c) {  // index bit 0 (inside the pair)
         float x = a[c].x, y = a[c].y;
@@ -108,6 +119,7 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
             a[c | m] = bfly_sub(x, y);
         }
     }
+    team_sync<TEAM>(team);  // the previous row's phase-B reads of tbuf are done
 
     // ---- to shared memory: element j -> run R = j / L, offset o = j % L, chunk-swizzled ----
 #pragma unroll
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
     for (int col = 0; col < P::COLS; ++col)
 #pragma unroll
         for (int p = 0; p < L / 2; ++p) {
-            b[col][p] = __fmul2_rn(b[col][p], rk2);
+            b[col][p] = mul2_rn(b[col][p], rk2);
             mx = fmaxf(mx, fmaxf(fabsf(b[col][p].x), fabsf(b[col][p].y)));
         }
 
@@ -180,7 +192,6 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
                                     b[col][2 * q + 1].y);
             }
         }
-        return;
     } else {
         constexpr int W = TEAM < 32 ? TEAM : 32;
 #pragma unroll
@@ -197,7 +208,6 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
         const float g = fmaxf(mx, 1e-5f);
         const float s = __fdiv_rn(Q, g);
         const float dq = __fdiv_rn(g, Q);
-        const float2 s2 = make_float2(s, s);
         const float2 magic2 = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
 
         int sum = 0;
@@ -211,7 +221,10 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
                 uint32_t f[16];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float2 t = __fmul2_rn(b[col][g16 * 8 + i], s2);
+                    // __fmul_rn is never contracted with the following add: the code is
+                    // round(fl(z * s)), the same two roundings the reference takes
+                    float2 t = make_float2(__fmul_rn(b[col][g16 * 8 + i].x, s),
+                                           __fmul_rn(b[col][g16 * 8 + i].y, s));
                     float2 u = __fadd2_rn(t, magic2);
                     f[2 * i] = __float_as_uint(u.x);
                     f[2 * i + 1] = __float_as_uint(u.y);
@@ -259,6 +272,7 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
             rowsum[row] = sum;
         }
     }
+    }  // row loop
 }
 
 // ---- plain BitLinear: absmax quantisation without a transform (any K % 128 == 0) ----
@@ -289,7 +303,6 @@ __global__ void __launch_bounds__(256)
     const float g = fmaxf(mx, 1e-5f);
     const float s = __fdiv_rn(Q, g);
     const float dq = __fdiv_rn(g, Q);
-    const float2 s2 = make_float2(s, s);
     const float2 magic2 = make_float2(12582912.f, 12582912.f);
     int sum = 0;
     for (int64_t c = lane; c < nchunk; c += 32) {
@@ -299,7 +312,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float2 x = make_float2(__uint_as_float(h[i] << 16), __uint_as_float(h[i] & 0xFFFF0000u));
-            float2 u = __fadd2_rn(__fmul2_rn(x, s2), magic2);
+            float2 u = __fadd2_rn(make_float2(__fmul_rn(x.x, s), __fmul_rn(x.y, s)), magic2);
             f[2 * i] = __float_as_uint(u.x);
             f[2 * i + 1] = __float_as_uint(u.y);
         }
@@ -336,7 +349,16 @@ static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *s
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    const int64_t blocks = (M + P::TEAMS - 1) / P::TEAMS;
+    static int per_sm[64] = {};
+    static int num_sms[64] = {};
+    if (dev >= 0 && dev < 64 && per_sm[dev] == 0) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev], kern, P::THREADS, P::SMEM);
+        cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (per_sm[dev] < 1) per_sm[dev] = 1;
+    }
+    const int64_t want = (M + P::TEAMS - 1) / P::TEAMS;
+    const int64_t cap = (int64_t)(dev >= 0 && dev < 64 ? per_sm[dev] * num_sms[dev] : 148);
+    const int64_t blocks = want < cap ? want : cap;
     const float rk = (float)(1.0 / sqrt((double)P::K));
     kern<<<(unsigned)blocks, P::THREADS, P::SMEM, stream>>>(
         reinterpret_cast<const uint32_t *>(X), (int)M, rk, reinterpret_cast<uint8_t *>(codes),

@@ -234,6 +234,31 @@ __host__ __device__ constexpr uint32_t idesc_i8_u8s8(int M, int N) {
 }
 
 // ------------------------------------------------------------------------------------------
+// Packed fp32x2 arithmetic with an explicit rounding mode: PTX add/mul carrying .rn are never
+// contracted into a fused multiply-add, so a product followed by a sum rounds twice, exactly as
+// two IEEE fp32 operations (the float2 intrinsics alone do not guarantee that).
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// ------------------------------------------------------------------------------------------
 // Small helpers
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {

@@ -8,22 +8,25 @@
 // on chip, never in HBM.
 //
 // Tile: 128 output features (MMA M, operand A) x 128 tokens (MMA N, operand B), K in stages of
-// 128.  Roles of the 13 warps of a persistent CTA (one per SM):
-//   warps 0-3   B producer.  INT8 codes: one thread issues TMA loads of [128 tokens x 128 B]
-//               with the 128-byte swizzle straight into the UMMA K-major layout.  INT4 codes:
-//               all 128 threads load one token's 64 bytes each, sign-extend the nibbles to
-//               int8 in registers and store them in the same swizzled layout.
-//   warps 4-7   A producer.  Thread i owns output feature n0 + i (= TMEM lane i): it loads the
-//               32 bytes of packed weights of a stage, expands each 2-bit offset code
-//               u = q + 1 to a byte with one shift-and-mask per four weights, and writes the 32
-//               words into TMEM with tcgen05.st.  The weights never touch shared memory.
-//   warp 12     MMA issuer: tcgen05.mma.kind::i8 with A from TMEM (unsigned bytes u) and B
-//               from shared memory (signed codes c), D += u * c in TMEM; tcgen05.commit frees
-//               the stages and publishes finished accumulators.
-//   warps 8-11  epilogue: tcgen05.ld of the int32 accumulator, subtract the token's code sum
-//               (sum_k q*c = sum_k u*c - sum_k c), scale by d_m * gamma, round to bf16, stage in
-//               shared memory and TMA-store.  Two accumulators in TMEM let the epilogue of one
-//               tile overlap the main loop of the next.
+// 128.  A persistent CTA per SM walks its tiles; warp roles:
+//   warp 0       TMA producer: packed weight tiles [128 rows x 32 B] into a shared-memory ring,
+//                and (INT8) code tiles [128 tokens x 128 B] with the 128-byte swizzle straight
+//                into the UMMA K-major layout.
+//   warp 1       MMA issuer (and TMEM owner): tcgen05.mma.kind::i8 with A from TMEM (unsigned
+//                bytes u = q + 1) and B from shared memory (signed codes c), D += u * c;
+//                tcgen05.commit frees stages and publishes finished accumulators.
+//   warps 4-11   two A-producer warpgroups taking alternate stages, so one group's TMEM store
+//                latency hides behind the other's work.  Thread i of a group owns TMEM lane i
+//                (output feature n0 + i): it reads its 32 packed bytes from shared memory,
+//                expands each 2-bit code to a byte with one shift-and-mask per four weights and
+//                writes 32 words into TMEM (tcgen05.st).
+//   warps 12-15  epilogue: tcgen05.ld of the int32 accumulator, subtract the token's code sum
+//                (sum_k q*c = sum_k u*c - sum_k c), scale by d_m * gamma, round to bf16 (lane
+//                pairs swap values so each lane stores one bf16x2 word: conflict-free), stage in
+//                shared memory and TMA-store.  Two TMEM accumulators let one tile's epilogue
+//                overlap the next tile's main loop.
+//   warps 16-19  (INT4 only) B producer: coalesced 16-byte loads of nibble codes, sign-extended
+//                to int8 in registers and stored in the swizzled K-major layout.
 // Every wait is bounded: after ~1 s a role records BITNET_ERR_TIMEOUT and stops; in-flight TMA
 // loads and MMAs are drained before TMEM is released.  No cluster multicast is used.
 #include "common.cuh"
@@ -39,20 +42,29 @@ constexpr int BT = 128;  // tokens per tile (MMA N)
 constexpr int BK = 128;  // K per stage: one 128-byte swizzled row of int8 codes
 constexpr int UMMA_K = 32;
 constexpr int B_STAGES = 6;
-constexpr int A_STAGES = 4;
+constexpr int W_STAGES = 8;   // packed-weight shared-memory ring
+constexpr int A_STAGES = 4;   // TMEM A stages (even ones for group 0, odd ones for group 1)
 constexpr int ACC_BUFS = 2;
 constexpr int TMEM_COLS = 512;
 constexpr int A_COL0 = ACC_BUFS * BT;  // A stages live after the accumulators
-constexpr int NUM_WARPS = 13;
-constexpr int NUM_THREADS = NUM_WARPS * 32;
 constexpr int B_STAGE_BYTES = BT * BK;
+constexpr int W_STAGE_BYTES = BW * BK / 4;
 constexpr int EPI_BUF_BYTES = 32 * 32 * 4;
 constexpr uint32_t IDESC = idesc_i8_u8s8(BW, BT);
 static_assert(A_COL0 + A_STAGES * (BK / 4) <= TMEM_COLS, "TMEM budget");
+static_assert(A_STAGES % 2 == 0, "two producer groups take alternate stages");
+
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_A0 = 4, WARP_EPI = 12, WARP_B4 = 16;
+template <int BITS>
+struct Threads {
+    static constexpr int value = (BITS == 8 ? 16 : 20) * 32;
+};
 
 struct __align__(8) Barriers {
     uint64_t full_b[B_STAGES];
     uint64_t empty_b[B_STAGES];
+    uint64_t full_w[W_STAGES];
+    uint64_t empty_w[W_STAGES];
     uint64_t full_a[A_STAGES];
     uint64_t empty_a[A_STAGES];
     uint64_t acc_full[ACC_BUFS];
@@ -62,11 +74,11 @@ struct __align__(8) Barriers {
 };
 
 constexpr size_t OFF_B = 0;
-constexpr size_t OFF_EPI = OFF_B + (size_t)B_STAGES * B_STAGE_BYTES;
-constexpr size_t OFF_SCALE = OFF_EPI + 4 * 2 * EPI_BUF_BYTES;  // [4 warps][BT] floats
+constexpr size_t OFF_W = OFF_B + (size_t)B_STAGES * B_STAGE_BYTES;
+constexpr size_t OFF_EPI = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
+constexpr size_t OFF_SCALE = OFF_EPI + 4 * 2 * EPI_BUF_BYTES;    // [4 warps][BT] floats
 constexpr size_t OFF_RSUM = OFF_SCALE + 4 * BT * sizeof(float);  // [4 warps][BT] ints
 constexpr size_t OFF_BAR = OFF_RSUM + 4 * BT * sizeof(int32_t);
-constexpr int PREFETCH = 4;  // producer register ring depth (stages in flight per thread)
 constexpr size_t SMEM_BYTES = OFF_BAR + sizeof(Barriers) + 1024;  // + alignment slack
 
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, __syncwarp orders the
@@ -87,17 +99,18 @@ __device__ __forceinline__ void iter_coords(int it, int KB, int &tile, int &kb) 
 }
 
 template <int BITS, bool OUT_I32>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(Threads<BITS>::value, 1)
     ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
+                           const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ CUtensorMap tmap_out,
-                           const uint8_t *__restrict__ codes4, const uint4 *__restrict__ wp,
-                           const float *__restrict__ scales, const int32_t *__restrict__ rowsum,
-                           const float *__restrict__ gamma_ptr, int M, int N, int K,
-                           int *status) {
+                           const uint8_t *__restrict__ codes4, const float *__restrict__ scales,
+                           const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
+                           int M, int N, int K, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sb = smem + OFF_B;
+    uint8_t *sw = smem + OFF_W;
     uint8_t *sepi = smem + OFF_EPI;
     float *s_scale = reinterpret_cast<float *>(smem + OFF_SCALE);
     int32_t *s_rsum = reinterpret_cast<int32_t *>(smem + OFF_RSUM);
@@ -109,11 +122,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int n_ttiles = (M + BT - 1) / BT;
     const int num_tiles = n_wtiles * n_ttiles;
     const int KB = K / BK;
+    const int my_tiles =
+        (int)blockIdx.x < num_tiles ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_tiles * KB;  // (tile, k-block) iterations of this CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < B_STAGES; ++s) {
             mbar_init(&bar->full_b[s], BITS == 8 ? 1 : 4);
             mbar_init(&bar->empty_b[s], 1);
+        }
+        for (int s = 0; s < W_STAGES; ++s) {
+            mbar_init(&bar->full_w[s], 1);
+            mbar_init(&bar->empty_w[s], 4);
         }
         for (int s = 0; s < A_STAGES; ++s) {
             mbar_init(&bar->full_a[s], 4);
@@ -126,11 +146,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_init(&bar->done, 1);
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == WARP_TMA && lane == 0) {
         if (BITS == 8) prefetch_tensormap(&tmap_codes);
+        prefetch_tensormap(&tmap_w);
         prefetch_tensormap(&tmap_out);
     }
-    if (warp == 12) {
+    if (warp == WARP_MMA) {
         tmem_alloc(&bar->tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
@@ -139,147 +160,121 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
-    if (warp < 4) {
-        // ------------------------------------------------------------------ B producer
-        if constexpr (BITS == 8) {
-            if (warp == 0 && lane == 0) {
-                int s = 0;
-                uint32_t ph = 0;
-                uint32_t issued = 0, issued_ph = 0;  // per-stage bits, for the final drain
-                bool ok = true;
-                for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                    const int mt = tile / n_wtiles;
-                    for (int kb = 0; kb < KB; ++kb) {
-                        if (!mbar_wait(&bar->empty_b[s], ph ^ 1, status)) { ok = false; break; }
-                        mbar_arrive_expect_tx(&bar->full_b[s], B_STAGE_BYTES);
-                        tma_load_2d(sb + (size_t)s * B_STAGE_BYTES, &tmap_codes, kb * BK, mt * BT,
-                                    &bar->full_b[s]);
-                        issued |= 1u << s;
-                        issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-                        if (++s == B_STAGES) { s = 0; ph ^= 1; }
-                    }
-                }
-                // no copy may still be writing shared memory when the CTA exits
-                for (int t = 0; t < B_STAGES; ++t)
-                    if (issued & (1u << t)) mbar_wait(&bar->full_b[t], (issued_ph >> t) & 1, status);
-            }
-        } else {
-            // INT4: thread i loads token i of the tile (64 bytes per stage), unpacks to int8
-            const int rr = warp * 32 + lane;
-            const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-            const int total = my_tiles * KB;
-            auto fetch = [&](int it, uint4 (&dst)[4]) {
-                if (it < total) {
-                    int tile, kb;
-                    iter_coords(it, KB, tile, kb);
-                    const int64_t m = (int64_t)(tile / n_wtiles) * BT + rr;
-                    if (m < M) {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(codes4 + m * (K / 2)) + 4 * kb;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = ldg_nc_v4(src + i);
-                        return;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-            };
-            uint4 ring[PREFETCH][4];
-#pragma unroll
-            for (int u = 0; u < PREFETCH - 1; ++u) fetch(u, ring[u]);
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int it0 = 0; it0 < total && ok; it0 += PREFETCH) {
-#pragma unroll
-                for (int u = 0; u < PREFETCH; ++u) {
-                    const int it = it0 + u;
-                    if (it >= total || !ok) break;
-                    fetch(it + PREFETCH - 1, ring[(u + PREFETCH - 1) % PREFETCH]);
-                    if (!warp_wait(&bar->empty_b[s], ph ^ 1, status, lane)) { ok = false; break; }
-                    uint8_t *dst = sb + (size_t)s * B_STAGE_BYTES + rr * 128;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {  // 16 codes k = 16c .. 16c+15
-                        const uint4 v = ring[u][c >> 1];
-                        const uint32_t w0 = (c & 1) ? v.z : v.x;
-                        const uint32_t w1 = (c & 1) ? v.w : v.y;
-                        uint4 o;
-                        o.x = sext_nibbles(w0 & 0x0F0F0F0Fu);
-                        o.y = sext_nibbles((w0 >> 4) & 0x0F0F0F0Fu);
-                        o.z = sext_nibbles(w1 & 0x0F0F0F0Fu);
-                        o.w = sext_nibbles((w1 >> 4) & 0x0F0F0F0Fu);
-                        *reinterpret_cast<uint4 *>(dst + ((c ^ (rr & 7)) << 4)) = o;
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bar->full_b[s]);
-                    if (++s == B_STAGES) { s = 0; ph ^= 1; }
-                }
-            }
-        }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------------ A producer
-        const int wq = warp - 4;  // TMEM lanes 32*wq .. 32*wq+31
-        const int rr = wq * 32 + lane;
-        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-        const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-        const int total = my_tiles * KB;
-        auto fetch = [&](int it, uint4 (&dst)[2]) {
-            if (it < total) {
+    if (warp == WARP_TMA) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t issued_b = 0, ph_b = 0, issued_w = 0, ph_w = 0;  // for the final drain
+            for (int it = 0; it < total; ++it) {
                 int tile, kb;
                 iter_coords(it, KB, tile, kb);
-                const int64_t n = (int64_t)(tile % n_wtiles) * BW + rr;
-                if (n < N) {
-                    const uint4 *src = wp + n * (K / 64) + 2 * kb;
-                    dst[0] = ldg_nc_v4(src);
-                    dst[1] = ldg_nc_v4(src + 1);
-                    return;
+                const int s_w = it % W_STAGES;
+                const uint32_t p_w = (uint32_t)(it / W_STAGES) & 1;
+                if (!mbar_wait(&bar->empty_w[s_w], p_w ^ 1, status)) break;
+                mbar_arrive_expect_tx(&bar->full_w[s_w], W_STAGE_BYTES);
+                tma_load_2d(sw + (size_t)s_w * W_STAGE_BYTES, &tmap_w, kb * (BK / 4),
+                            (tile % n_wtiles) * BW, &bar->full_w[s_w]);
+                issued_w |= 1u << s_w;
+                ph_w = (ph_w & ~(1u << s_w)) | (p_w << s_w);
+                if constexpr (BITS == 8) {
+                    const int s_b = it % B_STAGES;
+                    const uint32_t p_b = (uint32_t)(it / B_STAGES) & 1;
+                    if (!mbar_wait(&bar->empty_b[s_b], p_b ^ 1, status)) break;
+                    mbar_arrive_expect_tx(&bar->full_b[s_b], B_STAGE_BYTES);
+                    tma_load_2d(sb + (size_t)s_b * B_STAGE_BYTES, &tmap_codes, kb * BK,
+                                (tile / n_wtiles) * BT, &bar->full_b[s_b]);
+                    issued_b |= 1u << s_b;
+                    ph_b = (ph_b & ~(1u << s_b)) | (p_b << s_b);
                 }
             }
-            dst[0] = make_uint4(0, 0, 0, 0);
-            dst[1] = make_uint4(0, 0, 0, 0);
-        };
-        uint4 ring[PREFETCH][2];
-#pragma unroll
-        for (int u = 0; u < PREFETCH - 1; ++u) fetch(u, ring[u]);
-        int sa = 0;
-        uint32_t pha = 0;
-        bool ok = true;
-        for (int it0 = 0; it0 < total && ok; it0 += PREFETCH) {
-#pragma unroll
-            for (int u = 0; u < PREFETCH; ++u) {
-                const int it = it0 + u;
-                if (it >= total || !ok) break;
-                fetch(it + PREFETCH - 1, ring[(u + PREFETCH - 1) % PREFETCH]);
-                if (!warp_wait(&bar->empty_a[sa], pha ^ 1, status, lane)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t w[8] = {ring[u][0].x, ring[u][0].y, ring[u][0].z, ring[u][0].w,
-                                       ring[u][1].x, ring[u][1].y, ring[u][1].z, ring[u][1].w};
-                uint32_t out[32];
-#pragma unroll
-                for (int g = 0; g < 8; ++g)
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) out[4 * g + p] = (w[g] >> (2 * p)) & 0x03030303u;
-                tmem_st_32x32b_x32(t_lane + A_COL0 + sa * (BK / 4), out);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bar->full_a[sa]);
-                if (++sa == A_STAGES) { sa = 0; pha ^= 1; }
-            }
+            // no copy may still be writing shared memory when the CTA exits
+            for (int t = 0; t < W_STAGES; ++t)
+                if (issued_w & (1u << t)) mbar_wait(&bar->full_w[t], (ph_w >> t) & 1, status);
+            for (int t = 0; t < B_STAGES; ++t)
+                if (issued_b & (1u << t)) mbar_wait(&bar->full_b[t], (ph_b >> t) & 1, status);
         }
-    } else if (warp < 12) {
+        __syncwarp();
+    } else if (warp == WARP_MMA) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t sb_addr = smem_addr(sb);
+            bool ok = true;
+            int it = 0;
+            for (int t = 0; t < my_tiles && ok; ++t) {
+                const int ab = t & 1;
+                const uint32_t p_acc = (uint32_t)(t >> 1) & 1;
+                if (!mbar_wait(&bar->acc_empty[ab], p_acc ^ 1, status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + ab * BT;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s_a = it % A_STAGES, s_b = it % B_STAGES;
+                    if (!mbar_wait(&bar->full_a[s_a], (uint32_t)(it / A_STAGES) & 1, status) ||
+                        !mbar_wait(&bar->full_b[s_b], (uint32_t)(it / B_STAGES) & 1, status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t bdesc =
+                        smem_desc_kmajor_sw128(sb_addr + (uint32_t)s_b * B_STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        mma_i8_ts(d_tmem, tmem + A_COL0 + s_a * (BK / 4) + kk * (UMMA_K / 4),
+                                  bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
+                                  (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bar->empty_b[s_b]);
+                    mma_commit(&bar->empty_a[s_a]);
+                }
+                if (!ok) break;
+                mma_commit(&bar->acc_full[ab]);
+            }
+            // every MMA issued above has finished before TMEM is released
+            mma_commit(&bar->done);
+            mbar_wait(&bar->done, 0, status);
+        }
+        __syncwarp();
+    } else if (warp >= WARP_A0 && warp < WARP_A0 + 8) {
+        // ------------------------------------------------------------------ A producers
+        const int grp = (warp - WARP_A0) >> 2;  // takes iterations it = grp, grp + 2, ...
+        const int wq = warp & 3;                // TMEM lanes 32*wq .. 32*wq+31
+        const int rr = wq * 32 + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        for (int it = grp; it < total; it += 2) {
+            const int s_w = it % W_STAGES, s_a = it % A_STAGES;
+            if (!warp_wait(&bar->full_w[s_w], (uint32_t)(it / W_STAGES) & 1, status, lane)) break;
+            const uint4 *src = reinterpret_cast<const uint4 *>(sw + (size_t)s_w * W_STAGE_BYTES +
+                                                               rr * (BK / 4));
+            const uint4 c0 = src[0], c1 = src[1];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->empty_w[s_w]);
+            if (!warp_wait(&bar->empty_a[s_a], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status, lane))
+                break;
+            tc_fence_after();
+            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint32_t out[32];
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+#pragma unroll
+                for (int p = 0; p < 4; ++p) out[4 * g + p] = (w[g] >> (2 * p)) & 0x03030303u;
+            tmem_st_32x32b_x32(t_lane + A_COL0 + s_a * (BK / 4), out);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->full_a[s_a]);
+        }
+    } else if (warp >= WARP_EPI && warp < WARP_EPI + 4) {
         // ------------------------------------------------------------------ epilogue
-        const int wq = warp - 8;
+        const int wq = warp & 3;
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         float *w_scale = s_scale + wq * BT;  // this warp's copy: no cross-warp barrier needed
         int32_t *w_rsum = s_rsum + wq * BT;
         const float gamma = *gamma_ptr;
-        int ab = 0;
-        uint32_t phacc = 0;
+        const bool odd = lane & 1;
         int buf = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        for (int t = 0; t < my_tiles; ++t) {
+            const int tile = blockIdx.x + t * gridDim.x;
             const int nw = tile % n_wtiles;
             const int mt = tile / n_wtiles;
+            const int ab = t & 1;
             __syncwarp();  // the previous tile's scales are no longer read
 #pragma unroll
             for (int i = 0; i < BT / 32; ++i) {
@@ -288,7 +283,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 w_scale[ml] = m < M ? scales[m] * gamma : 0.f;
                 w_rsum[ml] = m < M ? rowsum[m] : 0;
             }
-            if (!warp_wait(&bar->acc_full[ab], phacc, status, lane)) break;
+            if (!warp_wait(&bar->acc_full[ab], (uint32_t)(t >> 1) & 1, status, lane)) break;
             tc_fence_after();
 #pragma unroll 1
             for (int ch = 0; ch < BT / 32; ++ch) {
@@ -298,15 +293,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint8_t *stage = sepi + (size_t)(wq * 2 + buf) * EPI_BUF_BYTES;
                 if (lane == 0) bulk_wait_group_read<1>();  // this buffer's previous store is done
                 __syncwarp();
+                if constexpr (OUT_I32) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int ml = ch * 32 + i;
-                    const int a = (int)v[i] - w_rsum[ml];
-                    if constexpr (OUT_I32) {
-                        reinterpret_cast<int32_t *>(stage)[i * 32 + lane] = a;
-                    } else {
-                        reinterpret_cast<__nv_bfloat16 *>(stage)[i * 32 + lane] =
-                            __float2bfloat16_rn((float)a * w_scale[ml]);
+                    for (int i = 0; i < 32; ++i)
+                        reinterpret_cast<int32_t *>(stage)[i * 32 + lane] =
+                            (int)v[i] - w_rsum[ch * 32 + i];
+                } else {
+                    // this lane holds column n = lane of rows i; lane pairs swap one value so
+                    // the even lane stores row i (n, n+1) and the odd lane row i+1 (n-1, n)
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int m0 = ch * 32 + i;
+                        const float y0 = (float)((int)v[i] - w_rsum[m0]) * w_scale[m0];
+                        const float y1 = (float)((int)v[i + 1] - w_rsum[m0 + 1]) * w_scale[m0 + 1];
+                        const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? y0 : y1, 1);
+                        const __nv_bfloat162 pr =
+                            odd ? __floats2bfloat162_rn(other, y1) : __floats2bfloat162_rn(y0, other);
+                        *reinterpret_cast<__nv_bfloat162 *>(stage + (i + (odd ? 1 : 0)) * 64 +
+                                                            (lane & ~1) * 2) = pr;
                     }
                 }
                 fence_proxy_async_smem();
@@ -323,63 +327,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
-            if (++ab == ACC_BUFS) { ab = 0; phacc ^= 1; }
         }
         if (lane == 0) bulk_wait_group<0>();
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int s = 0, sa = 0, ab = 0;
-            uint32_t ph = 0, pha = 0, phacc = 0;
-            bool ok = true;
-            const uint32_t sb_addr = smem_addr(sb);
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                if (!mbar_wait(&bar->acc_empty[ab], phacc ^ 1, status)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + ab * BT;
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&bar->full_a[sa], pha, status) ||
-                        !mbar_wait(&bar->full_b[s], ph, status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t bdesc =
-                        smem_desc_kmajor_sw128(sb_addr + (uint32_t)s * B_STAGE_BYTES);
+    } else if (BITS == 4 && warp >= WARP_B4 && warp < WARP_B4 + 4) {
+        // ------------------------------------------------------------------ INT4 B producer
+        // warp w covers tokens 32w .. 32w+31 of the tile; in sub-step i, lane l loads the
+        // 16-byte quarter (l % 4) of token 32w + 8i + l / 4: 8 tokens x 64 B per instruction,
+        // fully used sectors.
+        const int wq = warp & 3;
+        const int q = lane & 3;
+        for (int it = 0; it < total; ++it) {
+            int tile, kb;
+            iter_coords(it, KB, tile, kb);
+            const int s_b = it % B_STAGES;
+            uint4 raw[4];
 #pragma unroll
-                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        mma_i8_ts(d_tmem, tmem + A_COL0 + sa * (BK / 4) + kk * (UMMA_K / 4),
-                                  bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
-                                  (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bar->empty_b[s]);
-                    mma_commit(&bar->empty_a[sa]);
-                    if (++s == B_STAGES) { s = 0; ph ^= 1; }
-                    if (++sa == A_STAGES) { sa = 0; pha ^= 1; }
-                }
-                if (!ok) break;
-                mma_commit(&bar->acc_full[ab]);
-                if (++ab == ACC_BUFS) { ab = 0; phacc ^= 1; }
+            for (int i = 0; i < 4; ++i) {
+                const int row = wq * 32 + 8 * i + (lane >> 2);
+                const int64_t m = (int64_t)(tile / n_wtiles) * BT + row;
+                raw[i] = m < M ? ldg_nc_v4(codes4 + m * (K / 2) + kb * (BK / 2) + q * 16)
+                               : make_uint4(0, 0, 0, 0);
             }
-            // every MMA issued above has finished before TMEM is released
-            mma_commit(&bar->done);
-            mbar_wait(&bar->done, 0, status);
+            if (!warp_wait(&bar->empty_b[s_b], ((uint32_t)(it / B_STAGES) & 1) ^ 1, status, lane))
+                break;
+            uint8_t *dst = sb + (size_t)s_b * B_STAGE_BYTES;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = wq * 32 + 8 * i + (lane >> 2);
+                // 32 codes k = 32q .. 32q+31 -> chunks 2q (words x, y) and 2q+1 (words z, w)
+                const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t w0 = wd[2 * h], w1 = wd[2 * h + 1];
+                    uint4 o;
+                    o.x = sext_nibbles(w0 & 0x0F0F0F0Fu);
+                    o.y = sext_nibbles((w0 >> 4) & 0x0F0F0F0Fu);
+                    o.z = sext_nibbles(w1 & 0x0F0F0F0Fu);
+                    o.w = sext_nibbles((w1 >> 4) & 0x0F0F0F0Fu);
+                    const int c = 2 * q + h;
+                    *reinterpret_cast<uint4 *>(dst + row * 128 + ((c ^ (row & 7)) << 4)) = o;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->full_b[s_b]);
         }
-        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == WARP_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
 template <int BITS, bool OUT_I32>
-static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mo,
-                               int grid, cudaStream_t stream) {
+static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
+                               const CUtensorMap &mo, int grid, cudaStream_t stream) {
     auto kern = ternary_gemm_tc_kernel<BITS, OUT_I32>;
     static bool configured[64] = {};
     int dev = 0;
@@ -390,9 +396,9 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(
-        mc, mo, reinterpret_cast<const uint8_t *>(a.codes), reinterpret_cast<const uint4 *>(a.Wp),
-        a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, (int)a.K, a.status);
+    kern<<<grid, Threads<BITS>::value, SMEM_BYTES, stream>>>(
+        mc, mw, mo, reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum, a.gamma,
+        (int)a.M, (int)a.N, (int)a.K, a.status);
     return cudaGetLastError();
 }
 
@@ -416,23 +422,27 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
     using namespace tc;
     const int64_t tiles = ((a.N + BW - 1) / BW) * ((a.M + BT - 1) / BT);
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    CUtensorMap mc, mo;
+    CUtensorMap mc, mw, mo;
     memset(&mc, 0, sizeof mc);
+    memset(&mw, 0, sizeof mw);
     memset(&mo, 0, sizeof mo);
-    if (a.act_bits == 8) {
-        if (encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)a.K,
-                      (uint64_t)a.M, (uint64_t)a.K, BK, BT,
-                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
+    if (a.act_bits == 8 &&
+        encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)a.K,
+                  (uint64_t)a.M, (uint64_t)a.K, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    // packed weights: [N rows][K/4 bytes], one [128 x 32 B] box per stage
+    if (encode_2d(encode_fn, &mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, (uint64_t)a.K / 4,
+                  (uint64_t)a.N, (uint64_t)a.K / 4, BK / 4, BW,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (a.Y) {
         if (encode_2d(encode_fn, &mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, (uint64_t)a.N,
                       (uint64_t)a.M, (uint64_t)a.N * 2, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mo, grid, stream)
-                            : launch_tc_t<4, false>(a, mc, mo, grid, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, mo, grid, stream)
+                            : launch_tc_t<4, false>(a, mc, mw, mo, grid, stream);
         if (e != cudaSuccess) return e;
     }
     if (a.acc) {
@@ -440,8 +450,8 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
                       (uint64_t)a.M, (uint64_t)a.N * 4, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mo, grid, stream)
-                            : launch_tc_t<4, true>(a, mc, mo, grid, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, mo, grid, stream)
+                            : launch_tc_t<4, true>(a, mc, mw, mo, grid, stream);
     }
     return e;
 }

@@ -43,6 +43,9 @@ _SIGS = {
                                                     ctypes.c_int64, ctypes.c_void_p,
                                                     ctypes.c_void_p, ctypes.c_void_p,
                                                     ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_quantize_pack_weights_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                            ctypes.c_int64, ctypes.c_void_p,
+                                                            ctypes.c_void_p, ctypes.c_void_p]),
     "bitnet_act_codes_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
     "bitnet_act_quant": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                         ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
@@ -156,6 +159,24 @@ def bitnet_quantize_pack_weights(W: torch.Tensor, Wp: torch.Tensor | None = None
     _rc(L.bitnet_quantize_pack_weights(W.data_ptr(), N, K, Wp.data_ptr(), gamma.data_ptr(),
                                        ws.data_ptr(), ws.numel() * ws.element_size(),
                                        _stream(stream)), "bitnet_quantize_pack_weights")
+    return Wp, gamma
+
+
+def bitnet_quantize_pack_weights_noalloc(W: torch.Tensor, Wp: torch.Tensor | None = None,
+                                         gamma: torch.Tensor | None = None, stream=None):
+    """As bitnet_quantize_pack_weights, with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate device memory).  Returns (Wp, gamma)."""
+    L = load_library()
+    _check(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    if Wp is None:
+        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    _rc(L.bitnet_quantize_pack_weights_noalloc(W.data_ptr(), N, K, Wp.data_ptr(),
+                                               gamma.data_ptr(), _stream(stream)),
+        "bitnet_quantize_pack_weights_noalloc")
     return Wp, gamma
 
 

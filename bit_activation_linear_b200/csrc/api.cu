@@ -223,6 +223,35 @@ int bitnet_quantize_pack_weights(const void *W_dev, int64_t N, int64_t K, void *
                     1, "ternarize_pack");
 }
 
+int bitnet_quantize_pack_weights_noalloc(const void *W_dev, int64_t N, int64_t K, void *Wp_dev,
+                                         float *gamma_dev, bitnet_stream_t stream) {
+    int rc = check_shape(1, K, N, false, true);
+    if (rc) return rc;
+    if (!W_dev || !Wp_dev || !gamma_dev) return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(W_dev) || !aligned16(Wp_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    double *scratch = nullptr;
+    size_t scratch_bytes = 0;
+    cudaError_t e = noalloc_partials_address(&scratch, &scratch_bytes);
+    if (e != cudaSuccess)
+        return fail(BITNET_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
+    const int64_t n = N * K;
+    const int P = absmean_num_partials(n);
+    if ((size_t)P * sizeof(double) > scratch_bytes)
+        return fail(BITNET_ERR_UNSUPPORTED,
+                    "%d partial sums need %zu bytes of scratch; the fixed scratch holds %zu", P,
+                    (size_t)P * sizeof(double), scratch_bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // every partial is written before it is read: the scratch needs no clearing
+    if ((rc = launched(launch_absmean_partials(W_dev, n, scratch, P, s), 1, "absmean_partials")))
+        return rc;
+    return launched(launch_ternarize_pack(W_dev, n, scratch, P, static_cast<uint32_t *>(Wp_dev),
+                                          gamma_dev, s),
+                    1, "ternarize_pack");
+}
+
 size_t bitnet_act_codes_bytes(int64_t M, int64_t K, int act_bits) {
     if (M <= 0 || K <= 0) return 0;
     return act_bits == 4 ? (size_t)M * (size_t)K / 2 : (size_t)M * (size_t)K;

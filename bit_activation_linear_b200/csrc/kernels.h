@@ -14,6 +14,8 @@ cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, 
                                     cudaStream_t stream);
 cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partials, int P,
                                   uint32_t *Wp, float *gamma, cudaStream_t stream);
+// Device address (current device) and size of the library's fixed partial-sum scratch.
+cudaError_t noalloc_partials_address(double **ptr, size_t *bytes);
 
 // ---- steps 2-3: activations (actquant.cu) ----
 // Hadamard + quantise (or z output when zout != nullptr).  K = 2^logk, 7 <= logk <= 15.

@@ -14,6 +14,8 @@
 //   ternarize_pack_kernel    every block first sums the P partials in a fixed order (2.4 KB,
 //                            L2-resident), so no third launch or atomic is needed; then each
 //                            thread turns 16 weights into one packed 32-bit word.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -98,6 +100,35 @@ __global__ void __launch_bounds__(kWeightThreads)
         }
         wp[i] = word;
     }
+}
+
+// ------------------------------------------------------------------------------------------
+// Fixed device scratch for callers that cannot allocate device memory.
+//
+// The partial sums of |w| live in this file-scope array instead of caller workspace.  Every GPU
+// that loads the library holds it (9472 bytes) until the process exits.  Host code must not pass
+// the symbol itself to a kernel: the host-side name is only a stand-in, so its device address is
+// looked up once per device with cudaGetSymbolAddress while that device is current.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) double g_noalloc_partials[kMaxPartials];
+
+cudaError_t noalloc_partials_address(double **ptr, size_t *bytes) {
+    static std::mutex mu;
+    static double *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<double *>(p);
+    }
+    *ptr = addr[dev];
+    *bytes = sizeof(g_noalloc_partials);
+    return cudaSuccess;
 }
 
 cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, int P,

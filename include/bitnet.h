@@ -84,6 +84,26 @@ int bitnet_quantize_pack_weights(const void *W_dev, int64_t N, int64_t K, void *
                                  float *gamma_dev, void *ws_dev, size_t ws_bytes,
                                  bitnet_stream_t stream);
 
+/*
+ * bitnet_quantize_pack_weights without a workspace argument, for callers that cannot allocate
+ * device memory themselves -- for example a runtime that hands the library only the tensors it
+ * already owns, or code running where cudaMalloc is not allowed.  (The pages have no counterpart:
+ * this is a convenience of the library, not a step of the method.)
+ * Same inputs, outputs and results as bitnet_quantize_pack_weights; the partial sums of |w| go
+ * to a fixed scratch array inside the library (9472 bytes on every device that loads it, held
+ * until the process exits).  Maximum: the weight count is split into at most 1184 partial sums,
+ * which always fit, so every shape accepted by bitnet_quantize_pack_weights is accepted here;
+ * a shape that needed more scratch would be rejected with BITNET_ERR_UNSUPPORTED.
+ * The first call on a device looks up the scratch address (cudaGetSymbolAddress) with that
+ * device current; make that first call before capturing a stream into a CUDA graph.
+ * All calls share the one scratch array, which keeps the last call's contents (every entry is
+ * rewritten before it is read, so nothing needs clearing): calls that overlap on the GPU --
+ * on different streams without ordering between them -- race and give wrong gamma values.
+ * The call allocates and frees nothing.
+ */
+int bitnet_quantize_pack_weights_noalloc(const void *W_dev, int64_t N, int64_t K, void *Wp_dev,
+                                         float *gamma_dev, bitnet_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------- */
 /* Steps 2 and 3: online Hadamard transform and per-token activation quantisation            */
 /* ---------------------------------------------------------------------------------------- */

@@ -10,9 +10,11 @@ rescale (1 kernel).  Default workload: the Wo-shaped layer of a 2B-class model
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 cuda.synchronize on both sides, timed with CUDA events on the launching stream, max over ranks.
 Inputs are rotated over several copies whose total exceeds twice the L2 cache, so no step finds
-its inputs in L2.  Each copy's step is captured in two CUDA graphs (everything before the product,
-and the product) so that host launch overhead does not starve the GPU; CUDA events recorded
-around the product's replay give its live duration for the roofline figure.
+its inputs in L2.  Each copy's step is captured in two CUDA graphs so that host launch overhead
+does not starve the GPU: the preparation graph runs the weight ternarisation and the activation
+quantisation side by side on two streams (they are independent), the product graph runs the
+tensor-core product; CUDA events recorded around the product's replay give its live duration for
+the roofline figure.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the data
@@ -39,6 +41,7 @@ sys.path.insert(0, ROOT)
 from bit_activation_linear_b200 import synth  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic_wo_2048.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
 METRIC = "H-BitLinear tokens/s and effective int8 TOPS (% of roofline) on 1 B200"
@@ -71,6 +74,24 @@ def kernel_work(wl):
         "ternary_gemm_tc": {"ops": 2 * M * N * K,
                             "bytes": code_bytes + N * K // 4 + 2 * M * N + 8 * M},
     }
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) from the committed ncu capture, or None when the
+    capture is for another workload or the kernel's source changed since it was taken."""
+    import hashlib
+    try:
+        with open(TRAFFIC_FILE) as f:
+            cap = json.load(f)
+    except (OSError, ValueError):
+        return None
+    k = cap.get("kernels", {}).get(kernel)
+    if k is None or not cap.get("workload", "").startswith(workload + " "):
+        return None
+    with open(os.path.join(ROOT, k["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != k["source_sha256_16"]:
+            return None
+    return k["dram_read_bytes"] + k["dram_write_bytes"]
 
 
 # ----------------------------------------------------------------------------------------
@@ -266,8 +287,10 @@ def run_gpu(args, wl, rank, world, device):
         bufs.append(dict(X=X, W=W, Wp=Wp, gamma=gamma, wws=wws, codes=codes, scales=scales,
                          rowsum=rowsum, Y=Y))
 
-    def prep(b):
+    def weights(b):
         B.bitnet_quantize_pack_weights(b["W"], b["Wp"], b["gamma"], b["wws"])
+
+    def quant(b):
         B.bitnet_act_quant(b["X"], wl.hadamard, wl.act_bits, b["codes"], b["scales"],
                            b["rowsum"])
 
@@ -275,30 +298,41 @@ def run_gpu(args, wl, rank, world, device):
         B.bitnet_ternary_gemm(b["codes"], b["scales"], b["rowsum"], K, b["Wp"], b["gamma"],
                               wl.act_bits, want_acc=False, want_y=True, Y=b["Y"])
 
+    phases = (("weights", weights), ("act_quant", quant), ("ternary_gemm", gemm))
+    wstream = torch.cuda.Stream(device)
+
+    def prep(b):
+        # weight ternarisation and activation quantisation are independent: run them side by
+        # side on two streams, join before the product
+        wstream.wait_stream(stream)
+        with torch.cuda.stream(wstream):
+            weights(b)
+        quant(b)
+        stream.wait_stream(wstream)
+
     launches_before = B.bitnet_launch_count()
     for b in bufs:  # eager run once (sets kernel attributes, checks status)
-        prep(b)
-        gemm(b)
+        for _, fn in phases:
+            fn(b)
     B.bitnet_sync_status(stream)
     launches_per_step = (B.bitnet_launch_count() - launches_before) // copies
 
-    g_prep, g_gemm = [], []
+    graphs = []  # graphs[copy] = (prep graph, product graph)
     for b in bufs:
         gp, gg = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(gp, stream=stream):
             prep(b)
         with torch.cuda.graph(gg, stream=stream):
             gemm(b)
-        g_prep.append(gp)
-        g_gemm.append(gg)
+        graphs.append((gp, gg))
     torch.cuda.synchronize(device)
 
     def step(i, ev=None):
-        j = i % copies
-        g_prep[j].replay()
+        gp, gg = graphs[i % copies]
+        gp.replay()
         if ev is not None:
             ev[0].record(stream)
-        g_gemm[j].replay()
+        gg.replay()
         if ev is not None:
             ev[1].record(stream)
 
@@ -337,6 +371,28 @@ def run_gpu(args, wl, rank, world, device):
     gemm_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(k_ev))
     elapsed_ms = aggregate_max(elapsed_ms, device)
     gemm_ms = aggregate_max(gemm_ms, device)
+    # the two preparation phases run side by side inside the step; their own durations are
+    # timed here, one phase at a time, on the same rotated inputs
+    phase_ms = []
+    for _, fn in phases[:2]:
+        gs = []
+        for b in bufs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn(b)
+            gs.append(g)
+        n_iso = min(200, max(20, args.steps // 10))
+        pe = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_iso)]
+        torch.cuda._sleep(int(2e6))
+        for i in range(n_iso):
+            pe[i][0].record(stream)
+            gs[i % copies].replay()
+            pe[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        phase_ms.append(aggregate_max(statistics.mean(a.elapsed_time(b2) for a, b2 in pe), device))
+        del gs
+    phase_ms.append(gemm_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # end to end through the public API: pinned host X and W in, Y out, every step
@@ -347,6 +403,23 @@ def run_gpu(args, wl, rank, world, device):
         work = kernel_work(wl)
         int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
         achieved = work["ternary_gemm_tc"]["ops"] / (gemm_ms * 1e-3) / 1e12
+        hbm = peaks["hbm_gbs"]
+        w_bytes = work["absmean_partials"]["bytes"] + work["ternarize_pack"]["bytes"]
+        q_bytes = work["fwht_quant"]["bytes"]
+        per_kernel = {
+            "weights (absmean_partials + ternarize_pack; alone, outside the timed steps)": {
+                "us": 1e3 * phase_ms[0], "bound": "hbm", "bytes": w_bytes,
+                "achieved_gbs": w_bytes / (phase_ms[0] * 1e-3) / 1e9,
+                "frac": w_bytes / (phase_ms[0] * 1e-3) / 1e9 / hbm},
+            ("fwht_quant" if wl.hadamard else "act_quant_plain") + " (alone, outside the timed steps)": {
+                "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,
+                "achieved_gbs": q_bytes / (phase_ms[1] * 1e-3) / 1e9,
+                "frac": q_bytes / (phase_ms[1] * 1e-3) / 1e9 / hbm},
+            ("ternary_gemm_tc" if M > 8 else "ternary_gemv"): {
+                "us": 1e3 * gemm_ms, "bound": "tensor" if M > 8 else "hbm",
+                "ops": work["ternary_gemm_tc"]["ops"],
+                "achieved_tops": achieved, "frac": achieved / int8_peak},
+        }
         tokens_per_s = world * M / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC,
@@ -369,10 +442,12 @@ def run_gpu(args, wl, rank, world, device):
                              f"({copies * per_copy / 2**20:.0f} MiB > 2 x L2)"},
             "roofline": {"kernel": "ternary_gemm_tc", "bound": "tensor",
                          "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
-                         "frac": achieved / int8_peak, "traffic": None,
+                         "frac": achieved / int8_peak,
+                         "traffic": ncu_traffic("ternary_gemm_tc_kernel", wl.name),
                          "ms_per_launch": gemm_ms,
                          "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x "
                                         f"{INT8_PER_BF16} (nominal int8:bf16 dense ratio)"},
+            "kernels": per_kernel,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,

@@ -42,13 +42,19 @@ struct FwhtPlan {
     static constexpr int L = 1 << L_BITS;  // run length held by one thread in phase B
     static constexpr int COLS = V / L;     // runs per thread
     static constexpr int SHFL_BITS = T_BITS + 1 - L_BITS;  // bits done by lane shuffles
-    static constexpr int TPC_A = 256 / TEAM > 0 ? 256 / TEAM : 1;
-    static constexpr int TPC_B = 16384 / K > 0 ? 16384 / K : 1;  // <= 64 KB of smem per CTA
+    // bf16 rows per team in shared memory: the current one and the next (one for K = 2^15,
+    // where two would not fit next to the 128 KB transpose buffer)
+    static constexpr int RING = K <= 16384 ? 2 : 1;
+    // per team: the fp32 transpose buffer (4K bytes) and RING bf16 rows (2K bytes each)
+    static constexpr int TEAM_BYTES = K * 4 + RING * K * 2;
+    static constexpr int TPC_A = 128 / TEAM > 0 ? 128 / TEAM : 1;
+    static constexpr int TPC_B = 65536 / TEAM_BYTES > 0 ? 65536 / TEAM_BYTES : 1;  // <= 64 KB
     static constexpr int TEAMS = TPC_A < TPC_B ? TPC_A : TPC_B;
     static constexpr int THREADS = TEAMS * TEAM;
     static constexpr int CHUNKS = L / 4;                      // 16-byte chunks per run
     static constexpr int SWZ = (CHUNKS < 8 ? CHUNKS : 8) - 1;  // chunk XOR mask
-    static constexpr size_t SMEM = (size_t)TEAMS * K * sizeof(float) + 64 * sizeof(float);
+    static constexpr size_t SMEM =
+        (size_t)TEAMS * TEAM_BYTES + 64 * sizeof(float) + (size_t)TEAMS * RING * sizeof(uint64_t);
     static_assert(SHFL_BITS >= 0 && SHFL_BITS <= 5, "plan");
     static_assert(L >= 16, "runs must hold 16 codes");
 };
@@ -70,9 +76,9 @@ __device__ __forceinline__ void team_sync(int team) {
 
 template <int LOGK, int BITS, bool ZOUT>
 __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
-    fwht_quant_kernel(const uint32_t *__restrict__ X, int M, float rsqrt_k,
+    fwht_quant_kernel(const uint8_t *__restrict__ X, int M, float rsqrt_k,
                       uint8_t *__restrict__ codes, float *__restrict__ scales,
-                      int32_t *__restrict__ rowsum, float *__restrict__ zout) {
+                      int32_t *__restrict__ rowsum, float *__restrict__ zout, int *status) {
     using P = FwhtPlan<LOGK>;
     constexpr int K = P::K, TEAM = P::TEAM, V = P::V, L = P::L;
     extern __shared__ float4 smem4[];
@@ -82,28 +88,59 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
     const int lane = threadIdx.x & 31;
     float *tbuf = smem + team * K;
     float *red = smem + P::TEAMS * K;  // 64 floats of reduction scratch
+    uint8_t *rows = reinterpret_cast<uint8_t *>(red + 64);  // [TEAMS][RING][K] bf16
+    uint64_t *bars = reinterpret_cast<uint64_t *>(rows + (size_t)P::TEAMS * P::RING * K * 2);
+    uint8_t *ring = rows + (size_t)team * P::RING * K * 2;
+    uint64_t *rbar = bars + team * P::RING;
     const int64_t stride = (int64_t)gridDim.x * P::TEAMS;
+    constexpr uint32_t ROW_BYTES = K * 2;
 
     // Persistent: the team walks rows base + team, base += stride.  The trip count is the same
-    // for every team of the CTA (teams of <= 32 threads share a warp and its __syncwarp).  The
-    // next row's bf16 pairs are loaded while the current row is transformed.
-    uint32_t raw[V / 2];
-    auto load_row = [&](int64_t rw) {
-        const uint32_t *xr = X + rw * (K / 2);
-#pragma unroll
-        for (int c = 0; c < V / 2; ++c) raw[c] = rw < M ? __ldg(xr + c * TEAM + r) : 0u;
+    // for every team of the CTA (teams of <= 32 threads share a warp and its __syncwarp).  Rows
+    // arrive by bulk asynchronous copies into a two-row ring, so the next row is in flight while
+    // the current one is transformed.
+    if (r == 0) {
+        for (int i = 0; i < P::RING; ++i) mbar_init(&rbar[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // slots with a copy issued and not yet waited for, and the parity of that copy's phase
+    uint32_t pending = 0, pend_ph = 0;
+    int issued = 0;  // copies issued so far (sequence number of the next copy)
+    auto issue = [&](int64_t rw, int slot) {
+        if (rw < M) {
+            if (r == 0) {
+                mbar_arrive_expect_tx(&rbar[slot], ROW_BYTES);
+                bulk_load(ring + (size_t)slot * ROW_BYTES, X + rw * ROW_BYTES, ROW_BYTES,
+                          &rbar[slot]);
+            }
+            pending |= 1u << slot;
+            pend_ph = (pend_ph & ~(1u << slot)) | ((uint32_t)(issued / P::RING & 1) << slot);
+        }
+        ++issued;
     };
-    load_row((int64_t)blockIdx.x * P::TEAMS + team);
-    for (int64_t base = (int64_t)blockIdx.x * P::TEAMS; base < M; base += stride) {
+    const int64_t first = (int64_t)blockIdx.x * P::TEAMS;
+#pragma unroll
+    for (int i = 0; i < P::RING; ++i) issue(first + i * stride + team, i);
+    int iter = 0;
+    bool ok = true;
+    for (int64_t base = first; base < M; base += stride, ++iter) {
     const int64_t row = base + team;
     const bool valid = row < M;
+    const int slot = iter % P::RING;
+    if (valid && ok) {
+        if (mbar_wait(&rbar[slot], (uint32_t)(iter / P::RING) & 1, status)) pending &= ~(1u << slot);
+        else ok = false;
+    }
+    const uint32_t *xr = reinterpret_cast<const uint32_t *>(ring + (size_t)slot * ROW_BYTES);
 
     // ---- phase A: bf16 pairs -> fp32, butterflies over register bits ----
     float2 a[V / 2];
 #pragma unroll
-    for (int c = 0; c < V / 2; ++c)
-        a[c] = make_float2(__uint_as_float(raw[c] << 16), __uint_as_float(raw[c] & 0xFFFF0000u));
-    load_row(row + stride);
+    for (int c = 0; c < V / 2; ++c) {
+        const uint32_t w = (valid && ok) ? xr[c * TEAM + r] : 0u;
+        a[c] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
 #pragma unroll
     for (int c = 0; c < V / 2; ++c) {  // index bit 0 (inside the pair)
         float x = a[c].x, y = a[c].y;
@@ -119,7 +156,8 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
             a[c | m] = bfly_sub(x, y);
         }
     }
-    team_sync<TEAM>(team);  // the previous row's phase-B reads of tbuf are done
+    team_sync<TEAM>(team);  // this slot is read and the previous row's tbuf reads are done
+    issue(row + P::RING * stride, slot);  // refill the slot with the row after next
 
     // ---- to shared memory: element j -> run R = j / L, offset o = j % L, chunk-swizzled ----
 #pragma unroll
@@ -273,6 +311,9 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
         }
     }
     }  // row loop
+    // after a time-out, no copy may still be landing in shared memory when the CTA exits
+    for (int i = 0; i < P::RING; ++i)
+        if (pending & (1u << i)) mbar_wait(&rbar[i], (pend_ph >> i) & 1, status);
 }
 
 // ---- plain BitLinear: absmax quantisation without a transform (any K % 128 == 0) ----
@@ -337,7 +378,7 @@ __global__ void __launch_bounds__(256)
 
 template <int LOGK, int BITS, bool ZOUT>
 static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *scales,
-                                 int32_t *rowsum, float *zout, cudaStream_t stream) {
+                                 int32_t *rowsum, float *zout, int *status, cudaStream_t stream) {
     using P = FwhtPlan<LOGK>;
     auto kern = fwht_quant_kernel<LOGK, BITS, ZOUT>;
     static bool configured[64] = {};
@@ -361,33 +402,34 @@ static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *s
     const int64_t blocks = want < cap ? want : cap;
     const float rk = (float)(1.0 / sqrt((double)P::K));
     kern<<<(unsigned)blocks, P::THREADS, P::SMEM, stream>>>(
-        reinterpret_cast<const uint32_t *>(X), (int)M, rk, reinterpret_cast<uint8_t *>(codes),
-        scales, rowsum, zout);
+        reinterpret_cast<const uint8_t *>(X), (int)M, rk, reinterpret_cast<uint8_t *>(codes),
+        scales, rowsum, zout, status);
     return cudaGetLastError();
 }
 
 template <int LOGK>
 static cudaError_t launch_fwht_k(const void *X, int64_t M, int act_bits, void *codes,
-                                 float *scales, int32_t *rowsum, float *zout,
+                                 float *scales, int32_t *rowsum, float *zout, int *status,
                                  cudaStream_t stream) {
-    if (zout) return launch_fwht_t<LOGK, 8, true>(X, M, codes, scales, rowsum, zout, stream);
+    if (zout) return launch_fwht_t<LOGK, 8, true>(X, M, codes, scales, rowsum, zout, status, stream);
     if (act_bits == 4)
-        return launch_fwht_t<LOGK, 4, false>(X, M, codes, scales, rowsum, zout, stream);
-    return launch_fwht_t<LOGK, 8, false>(X, M, codes, scales, rowsum, zout, stream);
+        return launch_fwht_t<LOGK, 4, false>(X, M, codes, scales, rowsum, zout, status, stream);
+    return launch_fwht_t<LOGK, 8, false>(X, M, codes, scales, rowsum, zout, status, stream);
 }
 
 cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
-                              float *scales, int32_t *rowsum, float *zout, cudaStream_t stream) {
+                              float *scales, int32_t *rowsum, float *zout, int *status,
+                              cudaStream_t stream) {
     switch (logk) {
-        case 7: return launch_fwht_k<7>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 8: return launch_fwht_k<8>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 9: return launch_fwht_k<9>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 10: return launch_fwht_k<10>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 11: return launch_fwht_k<11>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 12: return launch_fwht_k<12>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 13: return launch_fwht_k<13>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 14: return launch_fwht_k<14>(X, M, act_bits, codes, scales, rowsum, zout, stream);
-        case 15: return launch_fwht_k<15>(X, M, act_bits, codes, scales, rowsum, zout, stream);
+        case 7: return launch_fwht_k<7>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 8: return launch_fwht_k<8>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 9: return launch_fwht_k<9>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 10: return launch_fwht_k<10>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 11: return launch_fwht_k<11>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 12: return launch_fwht_k<12>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 13: return launch_fwht_k<13>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 14: return launch_fwht_k<14>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        case 15: return launch_fwht_k<15>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -106,15 +106,17 @@ int launched(cudaError_t e, int count, const char *what) {
     return BITNET_OK;
 }
 
-int act_quant_impl(const void *X, int64_t M, int64_t K, int hadamard, int act_bits, void *codes,
-                   float *scales, int32_t *rowsum, float *zout, cudaStream_t stream) {
+int act_quant_impl(DeviceState *st, const void *X, int64_t M, int64_t K, int hadamard,
+                   int act_bits, void *codes, float *scales, int32_t *rowsum, float *zout,
+                   cudaStream_t stream) {
     if (hadamard) {
         const int lk = log2_exact(K);
         if (lk < 7 || lk > 15)
             return fail(BITNET_ERR_UNSUPPORTED,
                         "H-BitLinear needs K to be a power of two in [128, 32768], got %lld",
                         (long long)K);
-        return launched(launch_fwht_quant(X, M, lk, act_bits, codes, scales, rowsum, zout, stream),
+        return launched(launch_fwht_quant(X, M, lk, act_bits, codes, scales, rowsum, zout,
+                                          st->status_word, stream),
                         1, "fwht_quant");
     }
     return launched(launch_act_quant_plain(X, M, K, act_bits, codes, scales, rowsum, stream), 1,
@@ -164,7 +166,7 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
     float *scales = reinterpret_cast<float *>(w + round256(bitnet_act_codes_bytes(M, K, act_bits)));
     int32_t *rowsum = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(scales) +
                                                   round256((size_t)M * sizeof(float)));
-    if ((rc = act_quant_impl(X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr, stream)))
+    if ((rc = act_quant_impl(st, X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr, stream)))
         return rc;
     return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream);
 }
@@ -270,7 +272,7 @@ int bitnet_act_quant(const void *X_dev, int64_t M, int64_t K, int hadamard, int 
         return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
     DeviceState *st = nullptr;
     if ((rc = device_state(&st))) return rc;
-    return act_quant_impl(X_dev, M, K, hadamard, act_bits, codes_dev, scales_dev, rowsum_dev,
+    return act_quant_impl(st, X_dev, M, K, hadamard, act_bits, codes_dev, scales_dev, rowsum_dev,
                           nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -283,7 +285,7 @@ int bitnet_fwht_f32(const void *X_dev, int64_t M, int64_t K, float *Z_dev,
         return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
     DeviceState *st = nullptr;
     if ((rc = device_state(&st))) return rc;
-    return act_quant_impl(X_dev, M, K, 1, 8, nullptr, nullptr, nullptr, Z_dev,
+    return act_quant_impl(st, X_dev, M, K, 1, 8, nullptr, nullptr, nullptr, Z_dev,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 

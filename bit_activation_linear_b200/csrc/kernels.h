@@ -20,7 +20,8 @@ cudaError_t noalloc_partials_address(double **ptr, size_t *bytes);
 // ---- steps 2-3: activations (actquant.cu) ----
 // Hadamard + quantise (or z output when zout != nullptr).  K = 2^logk, 7 <= logk <= 15.
 cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
-                              float *scales, int32_t *rowsum, float *zout, cudaStream_t stream);
+                              float *scales, int32_t *rowsum, float *zout, int *status,
+                              cudaStream_t stream);
 // Quantise without a transform; K % 128 == 0.
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
                                    void *codes, float *scales, int32_t *rowsum,

@@ -11,9 +11,10 @@
 //   absmean_partials_kernel  fixed grid of P blocks (P depends only on the weight count), each
 //                            sums |w| in fp64 over a fixed grid-stride subset and writes one
 //                            partial; the reduction tree is fixed, so gamma is deterministic.
-//   ternarize_pack_kernel    every block first sums the P partials in a fixed order (2.4 KB,
-//                            L2-resident), so no third launch or atomic is needed; then each
-//                            thread turns 16 weights into one packed 32-bit word.
+//   ternarize_pack_kernel    every block first sums the P partials (<= 9.5 KB, L2-resident) in a
+//                            fixed tree, so no third launch or atomic is needed; then each thread
+//                            turns 16 weights into one packed 32-bit word with integer compares
+//                            against a bf16 threshold equivalent to the fp32 division.
 #include <mutex>
 
 #include "common.cuh"
@@ -44,7 +45,21 @@ __global__ void __launch_bounds__(kWeightThreads)
                             double *__restrict__ partials) {
     double acc0 = 0.0, acc1 = 0.0;
     const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
-    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nvec; i += stride) {
+    int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x;
+    // four independent 16-byte loads in flight per thread, then their sums
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ldg_nc_v4(w + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc0 += abs_bf16_pair_sum(v[u].x);
+            acc1 += abs_bf16_pair_sum(v[u].y);
+            acc0 += abs_bf16_pair_sum(v[u].z);
+            acc1 += abs_bf16_pair_sum(v[u].w);
+        }
+    }
+    for (; i < nvec; i += stride) {
         uint4 v = ldg_nc_v4(w + i);
         acc0 += abs_bf16_pair_sum(v.x);
         acc1 += abs_bf16_pair_sum(v.y);
@@ -59,30 +74,50 @@ __global__ void __launch_bounds__(kWeightThreads)
     __syncthreads();
     if (threadIdx.x == 0) {
         double t = 0.0;
-        for (int i = 0; i < kWeightThreads / 32; ++i) t += warp_sums[i];
+        for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
         partials[blockIdx.x] = t;
     }
+}
+
+// Threshold for the ternary decision, as a 15-bit bf16 magnitude pattern.
+// RoundClip(w / gamma, -1, 1) != 0  <=>  fl32(|w| / gamma) > 0.5 (ties to even send 0.5 to 0)
+// <=>  |w| / gamma > 0.5 + 2^-25 (the midpoint between 0.5 and the next float rounds down to
+// 0.5)  <=>  |w| > T with T = gamma * (0.5 + 2^-25), a product that is exact in double.  bf16
+// magnitudes are ordered like their bit patterns, so the decision is |w|_bits >= the pattern of
+// the smallest bf16 strictly above T.  This gives exactly the codes of the fp32 division.
+__device__ __forceinline__ uint32_t ternary_threshold_bits(float gamma) {
+    const double T = (double)gamma * (0.5 + 0x1p-25);
+    const uint32_t f = __float_as_uint(__double2float_ru(T));  // smallest float >= T
+    uint32_t h = (f + 0xFFFFu) >> 16;                          // smallest bf16 >= T
+    if ((double)__uint_as_float(h << 16) == T) h += 1;         // strictly above T
+    return h;
 }
 
 __global__ void __launch_bounds__(kWeightThreads)
     ternarize_pack_kernel(const uint4 *__restrict__ w, int64_t nwords, double n_weights,
                           const double *__restrict__ partials, int P, uint32_t *__restrict__ wp,
                           float *__restrict__ gamma_out) {
-    __shared__ float s_gamma;
-    if (threadIdx.x < 32) {
+    // gamma from the P partial sums: a fixed assignment of partials to threads and a fixed
+    // reduction tree, identical in every block, so gamma does not depend on the launch
+    __shared__ double warp_sums[kWeightThreads / 32];
+    __shared__ uint32_t s_thr;
+    {
         double s = 0.0;
-        for (int i = threadIdx.x; i < P; i += 32) s += partials[i];
+        for (int i = threadIdx.x; i < P; i += kWeightThreads) s += partials[i];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+        __syncthreads();
         if (threadIdx.x == 0) {
-            double mean = s / n_weights;
-            float g = (float)fmax(mean, 1e-5);
-            s_gamma = g;
+            double t = 0.0;
+            for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
+            const float g = (float)fmax(t / n_weights, 1e-5);
+            s_thr = ternary_threshold_bits(g);
             if (blockIdx.x == 0) *gamma_out = g;
         }
+        __syncthreads();
     }
-    __syncthreads();
-    const float g = s_gamma;
+    const uint32_t thr = s_thr;
     const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
     for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nwords; i += stride) {
         // 16 consecutive weights k = 16i + e; weight e = 4p + j goes to bits 8j + 2p as u = q + 1.
@@ -92,10 +127,8 @@ __global__ void __launch_bounds__(kWeightThreads)
         uint32_t word = 0;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            uint32_t bits = (e & 1) ? (h[e >> 1] & 0xFFFF0000u) : (h[e >> 1] << 16);
-            float r = __fdiv_rn(__uint_as_float(bits), g);
-            // clip(rint(r), -1, 1) with ties to even: |r| <= 0.5 gives 0, otherwise sign(r).
-            uint32_t u = r > 0.5f ? 2u : (r < -0.5f ? 0u : 1u);
+            const uint32_t bits = (e & 1) ? (h[e >> 1] >> 16) : (h[e >> 1] & 0xFFFFu);
+            const uint32_t u = (bits & 0x7FFFu) >= thr ? ((bits & 0x8000u) ? 0u : 2u) : 1u;
             word |= u << (8 * (e & 3) + 2 * (e >> 2));
         }
         wp[i] = word;

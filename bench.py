@@ -252,6 +252,12 @@ def aggregate_max(value: float, device) -> float:
     return float(t.item())
 
 
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own tokens_per_rank
+    tokens per step, and ms_per_step is the slowest rank's time (already max-reduced)."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 def barrier():
     if dist.is_available() and dist.is_initialized():
         dist.barrier()
@@ -420,7 +426,7 @@ def run_gpu(args, wl, rank, world, device):
                 "ops": work["ternary_gemm_tc"]["ops"],
                 "achieved_tops": achieved, "frac": achieved / int8_peak},
         }
-        tokens_per_s = world * M / (ms_per_step * 1e-3)
+        tokens_per_s = job_tokens_per_s(world, M, ms_per_step)
         line = {
             "metric": METRIC,
             "value": tokens_per_s,

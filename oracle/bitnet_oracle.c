@@ -34,8 +34,10 @@
  *   (INT8) or Q = 7 (INT4), eps 1e-5, round-half-even, clip to [-Q-1, Q]; output =
  *   bf16_rn(acc * d * gamma) with d = max|z| / Q.
  *
- * Parity pins live in tests/test_oracle_pins.py; the one function without an independent
- * pin is flagged there and in the design notes.
+ * Parity pins live in tests/test_oracle_pins.py: every exported function is checked there
+ * against something independent of it (a page's worked example, a closed form, a library
+ * routine, brute force).  The pins fix the arithmetic of the readings above; the readings
+ * themselves (eps, rounding, the INT4 rule, the 1/sqrt(K) scale) are not printed on the pages.
  */
 #include <math.h>
 #include <stdint.h>

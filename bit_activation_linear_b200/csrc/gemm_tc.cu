@@ -7,34 +7,35 @@
 // cheapest exact "add/subtract" is the int8 tensor-core MMA: the 2-bit weights are unpacked
 // on chip, never in HBM.
 //
-// Tile: 128 output features (MMA M, operand A) x 256 tokens (MMA N, operand B), both operands
-// in shared memory, K in stages of 128 (four 128x256x32 MMAs, 512 tensor cycles).  Measured on
-// B200: a tcgen05.mma issues in ~45 cycles, a commit costs ~50, and an mbarrier test issued after
-// MMAs returns ~180 cycles later, so the MMA thread tests the next stage before issuing the
-// current one and every instruction it issues covers 128 tensor cycles; the tensor core reads
-// its shared-memory operands at full rate while other warps write shared memory.  The two
-// 256-column int32 accumulators fill the 512 TMEM columns, so one tile's epilogue overlaps the
-// next tile's main loop.  A persistent CTA per SM walks its tiles; warp roles:
-//   warp 0       code-tile TMA (INT8): [256 tokens x 128 B] with the 128-byte swizzle (the UMMA
-//                K-major layout), four tiles in flight: under full load a load lands ~1800
-//                cycles after it is issued.
-//   warp 2       weight-tile TMA: packed weights [128 rows x 64 B] (two K stages).
-//   warp 1       MMA issuer (and TMEM owner): tcgen05.mma.kind::i8, A = unsigned bytes
-//                u = q + 1, B = signed codes c, D += u * c; tcgen05.commit frees stages and
-//                publishes finished accumulators; it also frees a weight tile once the A stages
-//                made from it are complete.
-//   warps 4-7/11 A producers (two groups taking alternate stages for INT8, one for INT4):
-//                thread i expands the 32 packed bytes of output feature n0 + i for the stage
-//                (one shift-and-mask per four weights) and stores the 128 int8 bytes in the
-//                swizzled K-major layout.  The 2-bit weights never exist unpacked in HBM.
-//   warps 8-11   (INT4 only) B producers: coalesced 16-byte loads of nibble codes, sign-extended
-//                to int8 in registers and stored in the swizzled K-major layout.
-//   warps 12-19  two epilogue warpgroups, each taking half of the tile's tokens: tcgen05.ld of
-//                the int32 accumulator, subtract the token's code sum (sum_k q*c =
-//                sum_k u*c - sum_k c), scale by d_m * gamma, round to bf16 and store: lane pairs
-//                swap one value so each half-warp writes a contiguous 64-byte row segment.
-// Every wait is bounded: after ~1 s a role records BITNET_ERR_TIMEOUT and stops; in-flight TMA
-// loads and MMAs are drained before TMEM is released.  No cluster multicast is used.
+// A CTA pair (a cluster of two CTAs on neighbouring SMs) computes a tile of 256 tokens x 256
+// output features with tcgen05.mma.cta_group::2: D[256 x 256] += A[256 x 32] * B[256 x 32]^T,
+// A = activation codes (signed), B = weight offset codes u = q + 1 in {0, 1, 2} (unsigned).
+// CTA r of the pair holds tokens 128r .. 128r+127 of A, features 128r .. 128r+127 of B and
+// accumulator rows (tokens) 128r .. 128r+127 for all 256 features.  Against one CTA computing a
+// 128 x 256 tile alone, each SM moves half the activation bytes from L2 and through shared
+// memory per multiply-add: measured on B200, a lone CTA spent ~1050 cycles per 128-deep K stage
+// on 512 cycles of tensor work, its operand traffic (TMA and unpack writes plus tensor-core reads)
+// saturating shared memory and the L2->SM path.
+//
+// K runs in stages of 128 (four K=32 MMAs, 512 tensor cycles).  The two 256-column int32
+// accumulators fill the 512 TMEM columns, so a tile's epilogue overlaps the next tile's MMAs.
+// Warp roles, in both CTAs unless noted:
+//   warp 0       code-tile TMA (INT8): [128 tokens x 128 B] with the 128-byte swizzle (the UMMA
+//                K-major layout); the pair form of the copy completes on the even CTA's barrier,
+//                which expects both halves.
+//   warp 2       packed-weight TMA: [128 features x 64 B] (two K stages) into a local ring.
+//   warp 1       even CTA: MMA issuer (one thread).  Both CTAs: tensor-memory allocation.
+//   warps 4-11   weight unpack (two groups taking alternate stages; one group for INT4): thread i
+//                expands the 32 packed bytes of feature i for the stage (one shift-and-mask per
+//                four weights) into 128 bytes of the swizzled layout, then signals the even CTA.
+//   warps 8-11   (INT4 only) code producers: 16-byte loads of nibble codes, sign-extended to
+//                int8 in registers, stored in the swizzled layout.
+//   warps 12-19  epilogue: thread = token row; tcgen05.ld of 32 features, subtract the token's
+//                code sum (sum_k c*q = sum_k c*u - sum_k c), scale by d_m * gamma, round to bf16,
+//                64 contiguous bytes per thread and chunk.
+// Commits multicast to both CTAs; every wait is bounded: after ~1 s a role records
+// BITNET_ERR_TIMEOUT and stops; in-flight copies and MMAs are drained and both CTAs meet at a
+// cluster barrier before tensor memory is released.  No TMA multicast is used.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,51 +44,53 @@
 namespace bitnet {
 namespace tc {
 
-constexpr int BW = 128;    // output features per tile (MMA M)
-constexpr int BT = 256;    // tokens per tile (MMA N)
-constexpr int BK = 128;    // K per stage: one 128-byte swizzled row of int8
+constexpr int BM = 256;            // tokens per pair tile (MMA M)
+constexpr int BN = 256;            // output features per pair tile (MMA N)
+constexpr int HM = BM / 2;         // tokens held by one CTA
+constexpr int HN = BN / 2;         // features held by one CTA
+constexpr int BK = 128;            // K per stage: one 128-byte swizzled row of int8
 constexpr int UMMA_K = 32;
 constexpr int MMAS = BK / UMMA_K;  // 4 per stage
-constexpr int B_STAGES = 4;        // code tiles in flight (a TMA load takes ~1800 cycles to land)
-constexpr int A_STAGES = 4;        // unpacked A tiles
-constexpr int W_STAGES = 3;        // packed-weight tiles in flight
-constexpr int SPW = 2;             // K stages per packed-weight tile [128 rows x 64 B]
+constexpr int A_STAGES = 6;        // code tiles in flight
+constexpr int B_STAGES = 4;        // unpacked weight tiles
+constexpr int W_STAGES = 4;        // packed-weight tiles in flight
+constexpr int SPW = 2;             // K stages per packed-weight tile [128 features x 64 B]
 constexpr int ACC_BUFS = 2;
 constexpr int TMEM_COLS = 512;
-constexpr int A_STAGE_BYTES = BW * BK;  // 16 KB
-constexpr int B_STAGE_BYTES = BT * BK;  // 32 KB
-constexpr int W_STAGE_BYTES = BW * SPW * BK / 4;
+constexpr int A_STAGE_BYTES = HM * BK;               // 16 KB
+constexpr int B_STAGE_BYTES = HN * BK;               // 16 KB
+constexpr int W_STAGE_BYTES = HN * SPW * BK / 4;     // 8 KB
 constexpr int EPI_WARPS = 8;
-constexpr uint32_t IDESC = idesc_i8_u8s8(BW, BT);
-static_assert(ACC_BUFS * BT <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t IDESC = idesc_i8_s8u8(BM, BN);
+static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM budget");
 
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_A0 = 4, WARP_B4 = 8, WARP_EPI = 12;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_B0 = 4, WARP_A4 = 8, WARP_EPI = 12;
 constexpr int NUM_THREADS = 20 * 32;
 
 struct __align__(8) Barriers {
-    uint64_t full_b[B_STAGES];   // code tile landed
-    uint64_t empty_b[B_STAGES];  // the MMAs that read it have completed
-    uint64_t full_a[A_STAGES];   // unpacked A tile written
-    uint64_t empty_a[A_STAGES];
-    uint64_t full_w[W_STAGES];
-    uint64_t empty_w[W_STAGES];
-    uint64_t acc_full[ACC_BUFS];
-    uint64_t acc_empty[ACC_BUFS];
-    uint64_t done;
+    uint64_t full_a[A_STAGES];     // even CTA: both halves of the code tile are in place
+    uint64_t empty_a[A_STAGES];    // both: the MMAs that read the stage have completed
+    uint64_t full_b[B_STAGES];     // even CTA: the unpack warps of both CTAs wrote the stage
+    uint64_t empty_b[B_STAGES];    // both
+    uint64_t full_w[W_STAGES];     // local packed-weight ring
+    uint64_t empty_w[W_STAGES];    // local; arrived by the MMA thread of the even CTA
+    uint64_t acc_full[ACC_BUFS];   // both
+    uint64_t acc_empty[ACC_BUFS];  // even CTA: the epilogue warps of both CTAs
+    uint64_t done;                 // both: every MMA has completed
     uint32_t tmem_base;
 };
 
+// identical offsets in both CTAs: the pair MMA addresses the peer's operands by the even CTA's
+// shared-memory offsets
 constexpr size_t OFF_A = 0;
 constexpr size_t OFF_B = OFF_A + (size_t)A_STAGES * A_STAGE_BYTES;
 constexpr size_t OFF_W = OFF_B + (size_t)B_STAGES * B_STAGE_BYTES;
-constexpr size_t OFF_SCALE = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;  // [8 warps][BT/2] floats
-constexpr size_t OFF_RSUM = OFF_SCALE + EPI_WARPS * (BT / 2) * sizeof(float);
-constexpr size_t OFF_BAR = OFF_RSUM + EPI_WARPS * (BT / 2) * sizeof(int32_t);
+constexpr size_t OFF_BAR = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + sizeof(Barriers) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, __syncwarp orders the
-// other lanes after the acquire (needed before warp-collective .sync.aligned tcgen05 ops).
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast,
+// __syncwarp orders the other lanes after the acquire (needed before warp-collective tcgen05 ops).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *status, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, status);
@@ -97,7 +100,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *s
 }
 
 template <int BITS, bool OUT_I32>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                            const __grid_constant__ CUtensorMap tmap_w,
                            void *__restrict__ Yout, const uint8_t *__restrict__ codes4,
@@ -110,31 +113,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint8_t *sa = smem + OFF_A;
     uint8_t *sb = smem + OFF_B;
     uint8_t *sw = smem + OFF_W;
-    float *s_scale = reinterpret_cast<float *>(smem + OFF_SCALE);
-    int32_t *s_rsum = reinterpret_cast<int32_t *>(smem + OFF_RSUM);
     Barriers *bar = reinterpret_cast<Barriers *>(smem + OFF_BAR);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_wtiles = (N + BW - 1) / BW;
-    const int n_ttiles = (M + BT - 1) / BT;
-    const int num_tiles = n_wtiles * n_ttiles;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int n_ftiles = (N + BN - 1) / BN;
+    const int n_ttiles = (M + BM - 1) / BM;
+    const int num_tiles = n_ftiles * n_ttiles;
     const int KS = K / BK;                 // stages per tile
-    const int WPT = (KS + SPW - 1) / SPW;  // weight tiles per output tile
-    constexpr int A_GROUPS = BITS == 8 ? 2 : 1;
-    const int my_tiles =
-        (int)blockIdx.x < num_tiles ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const int total = my_tiles * KS;  // (tile, stage) iterations of this CTA
+    const int WPT = (KS + SPW - 1) / SPW;  // packed-weight tiles per output tile
+    constexpr int B_GROUPS = BITS == 8 ? 2 : 1;
+    const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
+    const int total = my_tiles * KS;  // (tile, stage) iterations of this pair
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < B_STAGES; ++s) {
-            // the TMA arrival (INT8) or the four INT4 producer warps
-            mbar_init(&bar->full_b[s], BITS == 8 ? 1 : 4);
-            mbar_init(&bar->empty_b[s], 1);
-        }
         for (int s = 0; s < A_STAGES; ++s) {
-            mbar_init(&bar->full_a[s], 4);
+            // INT8: the even CTA's expect-tx arrival; INT4: the code warps of both CTAs
+            mbar_init(&bar->full_a[s], BITS == 8 ? 1 : 8);
             mbar_init(&bar->empty_a[s], 1);
+        }
+        for (int s = 0; s < B_STAGES; ++s) {
+            mbar_init(&bar->full_b[s], 8);
+            mbar_init(&bar->empty_b[s], 1);
         }
         for (int s = 0; s < W_STAGES; ++s) {
             mbar_init(&bar->full_w[s], 1);
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         for (int s = 0; s < ACC_BUFS; ++s) {
             mbar_init(&bar->acc_full[s], 1);
-            mbar_init(&bar->acc_empty[s], EPI_WARPS);
+            mbar_init(&bar->acc_empty[s], 2 * EPI_WARPS);
         }
         mbar_init(&bar->done, 1);
         fence_mbar_init();
@@ -152,11 +156,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         prefetch_tensormap(&tmap_w);
     }
     if (warp == WARP_MMA) {
-        tmem_alloc(&bar->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised and the tensor memory is allocated
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
@@ -166,20 +170,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t issued = 0, ph = 0;  // for the final drain
             int t = 0, ks = 0;
             for (int it = 0; it < total; ++it) {
-                const int tile = blockIdx.x + t * gridDim.x;
-                const int s = it % B_STAGES;
-                const uint32_t p = (uint32_t)(it / B_STAGES) & 1;
-                if (!mbar_wait(&bar->empty_b[s], p ^ 1, status)) break;
-                mbar_arrive_expect_tx(&bar->full_b[s], B_STAGE_BYTES);
-                tma_load_2d(sb + (size_t)s * B_STAGE_BYTES, &tmap_codes, ks * BK,
-                            (tile / n_wtiles) * BT, &bar->full_b[s]);
+                const int tile = pair + t * npairs;
+                const int s = it % A_STAGES;
+                const uint32_t p = (uint32_t)(it / A_STAGES) & 1;
+                if (!mbar_wait(&bar->empty_a[s], p ^ 1, status)) break;
+                if (leader) mbar_arrive_expect_tx(&bar->full_a[s], 2 * A_STAGE_BYTES);
+                tma_load_2d_pair(sa + (size_t)s * A_STAGE_BYTES, &tmap_codes, ks * BK,
+                                 (tile / n_ftiles) * BM + (int)rank * HM,
+                                 mapa_shared(smem_addr(&bar->full_a[s]), 0));
                 issued |= 1u << s;
                 ph = (ph & ~(1u << s)) | (p << s);
                 if (++ks == KS) { ks = 0; ++t; }
             }
-            // no copy may still be writing shared memory when the CTA exits
-            for (int i = 0; i < B_STAGES; ++i)
-                if (issued & (1u << i)) mbar_wait(&bar->full_b[i], (ph >> i) & 1, status);
+            // no copy may still be writing shared memory when the CTA exits: the even CTA sees
+            // its barrier complete, the odd CTA sees the stage consumed (or gives up)
+            for (int i = 0; i < A_STAGES; ++i)
+                if (issued & (1u << i))
+                    mbar_wait(leader ? &bar->full_a[i] : &bar->empty_a[i], (ph >> i) & 1,
+                                 status);
         }
         __syncwarp();
     } else if (warp == WARP_WTMA) {
@@ -191,10 +199,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int s_w = w % W_STAGES;
                 const uint32_t p_w = (uint32_t)(w / W_STAGES) & 1;
                 if (!mbar_wait(&bar->empty_w[s_w], p_w ^ 1, status)) break;
-                const int tile_w = blockIdx.x + (w / WPT) * gridDim.x;
+                const int tile_w = pair + (w / WPT) * npairs;
                 mbar_arrive_expect_tx(&bar->full_w[s_w], W_STAGE_BYTES);
                 tma_load_2d(sw + (size_t)s_w * W_STAGE_BYTES, &tmap_w, (w % WPT) * SPW * (BK / 4),
-                            (tile_w % n_wtiles) * BW, &bar->full_w[s_w]);
+                            (tile_w % n_ftiles) * BN + (int)rank * HN, &bar->full_w[s_w]);
                 issued |= 1u << s_w;
                 ph = (ph & ~(1u << s_w)) | (p_w << s_w);
             }
@@ -204,10 +212,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else if (warp == WARP_MMA) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (leader && lane == 0) {
             const uint32_t sa_addr = smem_addr(sa);
             const uint32_t sb_addr = smem_addr(sb);
-            bool ok = true;
             bool next_a = total > 0 && mbar_test_wait(&bar->full_a[0], 0);
             bool next_b = total > 0 && mbar_test_wait(&bar->full_b[0], 0);
             int t = 0, ks = 0;
@@ -215,64 +222,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int ab = t & 1;
                 const int sa_i = it % A_STAGES, sb_i = it % B_STAGES;
                 if (ks == 0 &&
-                    !mbar_wait(&bar->acc_empty[ab], ((uint32_t)(t >> 1) & 1) ^ 1, status)) {
-                    ok = false;
+                    !mbar_wait(&bar->acc_empty[ab], ((uint32_t)(t >> 1) & 1) ^ 1, status))
                     break;
-                }
-                if ((!next_a && !mbar_wait(&bar->full_a[sa_i], (uint32_t)(it / A_STAGES) & 1, status)) ||
-                    (!next_b && !mbar_wait(&bar->full_b[sb_i], (uint32_t)(it / B_STAGES) & 1, status))) {
-                    ok = false;
+                if ((!next_a &&
+                     !mbar_wait(&bar->full_a[sa_i], (uint32_t)(it / A_STAGES) & 1, status)) ||
+                    (!next_b &&
+                     !mbar_wait(&bar->full_b[sb_i], (uint32_t)(it / B_STAGES) & 1, status)))
                     break;
-                }
                 tc_fence_after();
                 // ask now whether the next stage is ready: the answers are needed only after this
                 // stage's MMAs have been issued, so their latency is hidden behind them
                 if (it + 1 < total) {
                     next_a = mbar_test_wait(&bar->full_a[(it + 1) % A_STAGES],
-                                            (uint32_t)((it + 1) / A_STAGES) & 1);
+                                               (uint32_t)((it + 1) / A_STAGES) & 1);
                     next_b = mbar_test_wait(&bar->full_b[(it + 1) % B_STAGES],
-                                            (uint32_t)((it + 1) / B_STAGES) & 1);
+                                               (uint32_t)((it + 1) / B_STAGES) & 1);
                 }
-                const uint32_t d_tmem = tmem + ab * BT;
-                const uint64_t adesc = smem_desc_kmajor_sw128(sa_addr + (uint32_t)sa_i * A_STAGE_BYTES);
-                const uint64_t bdesc = smem_desc_kmajor_sw128(sb_addr + (uint32_t)sb_i * B_STAGE_BYTES);
+                const uint32_t d_tmem = tmem + ab * BN;
+                const uint64_t adesc =
+                    smem_desc_kmajor_sw128(sa_addr + (uint32_t)sa_i * A_STAGE_BYTES);
+                const uint64_t bdesc =
+                    smem_desc_kmajor_sw128(sb_addr + (uint32_t)sb_i * B_STAGE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < MMAS; ++kk)
-                    mma_i8_ss(d_tmem, adesc + (uint64_t)(kk * UMMA_K / 16),
-                              bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
-                              (ks | kk) != 0 ? 1u : 0u);
-                mma_commit(&bar->empty_b[sb_i]);
-                mma_commit(&bar->empty_a[sa_i]);
-                // the A tiles made from this weight tile are complete (full_a observed): refill it
-                if (ks % SPW == SPW - 1 || ks == KS - 1)
-                    mbar_arrive(&bar->empty_w[(t * WPT + ks / SPW) % W_STAGES]);
-                if (ks == KS - 1) mma_commit(&bar->acc_full[ab]);
+                    mma_i8_ss_pair(d_tmem, adesc + (uint64_t)(kk * UMMA_K / 16),
+                                   bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
+                                   (ks | kk) != 0 ? 1u : 0u);
+                mma_commit_pair(&bar->empty_a[sa_i], 3);
+                mma_commit_pair(&bar->empty_b[sb_i], 3);
+                // the unpack warps of both CTAs are done with this packed-weight tile (full_b
+                // observed for its last stage): both may refill it
+                if (ks % SPW == SPW - 1 || ks == KS - 1) {
+                    uint64_t *ew = &bar->empty_w[(t * WPT + ks / SPW) % W_STAGES];
+                    mbar_arrive(ew);
+                    mbar_arrive_cluster(mapa_shared(smem_addr(ew), 1));
+                }
+                if (ks == KS - 1) mma_commit_pair(&bar->acc_full[ab], 3);
                 if (++ks == KS) { ks = 0; ++t; }
             }
-            (void)ok;
-            // every MMA issued above has finished before TMEM is released
-            mma_commit(&bar->done);
-            mbar_wait(&bar->done, 0, status);
+            // every MMA issued above has finished before either CTA releases tensor memory
+            mma_commit_pair(&bar->done, 3);
         }
+        if (lane == 0) mbar_wait(&bar->done, 0, status);
         __syncwarp();
-    } else if (warp >= WARP_A0 && warp < WARP_A0 + 4 * A_GROUPS) {
-        // ------------------------------------------------------------------ A producers
-        const int grp = (warp - WARP_A0) >> 2;  // takes iterations it = grp (mod A_GROUPS)
-        const int rr = (warp & 3) * 32 + lane;  // row of the A tile = output feature n0 + rr
-        for (int it = grp; it < total; it += A_GROUPS) {
+    } else if (warp >= WARP_B0 && warp < WARP_B0 + 4 * B_GROUPS) {
+        // ------------------------------------------------------------------ weight unpack
+        const int grp = (warp - WARP_B0) >> 2;  // takes iterations it = grp (mod B_GROUPS)
+        const int rr = (warp & 3) * 32 + lane;  // row of this CTA's B half = feature
+        for (int it = grp; it < total; it += B_GROUPS) {
             const int t = it / KS, ks = it - t * KS;
             const int wseq = t * WPT + ks / SPW;
-            const int s_w = wseq % W_STAGES, s = it % A_STAGES;
+            const int s_w = wseq % W_STAGES, s = it % B_STAGES;
             if (!warp_wait(&bar->full_w[s_w], (uint32_t)(wseq / W_STAGES) & 1, status, lane)) break;
             // row rr of the weight tile: SPW stages x 32 B
             const uint4 *wsrc = reinterpret_cast<const uint4 *>(
                 sw + (size_t)s_w * W_STAGE_BYTES + rr * (SPW * BK / 4) + (ks % SPW) * (BK / 4));
             const uint4 p0 = wsrc[0], p1 = wsrc[1];
             const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            if (!warp_wait(&bar->empty_a[s], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status, lane)) break;
+            if (!warp_wait(&bar->empty_b[s], ((uint32_t)(it / B_STAGES) & 1) ^ 1, status, lane))
+                break;
             // packed word g holds k = 16g .. 16g+15; (w >> 2p) & 0x03030303 is k = 16g+4p .. +3,
             // so word g becomes the 16-byte chunk g of the row, stored at chunk g ^ (rr & 7)
-            uint8_t *arow = sa + (size_t)s * A_STAGE_BYTES + rr * 128;
+            uint8_t *brow = sb + (size_t)s * B_STAGE_BYTES + rr * 128;
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
                 uint4 o;
@@ -280,91 +291,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 o.y = (w[g] >> 2) & 0x03030303u;
                 o.z = (w[g] >> 4) & 0x03030303u;
                 o.w = (w[g] >> 6) & 0x03030303u;
-                *reinterpret_cast<uint4 *>(arow + ((g ^ (rr & 7)) << 4)) = o;
+                *reinterpret_cast<uint4 *>(brow + ((g ^ (rr & 7)) << 4)) = o;
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->full_a[s]);
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full_b[s]), 0));
         }
     } else if (warp >= WARP_EPI && warp < WARP_EPI + EPI_WARPS) {
         // ------------------------------------------------------------------ epilogue
-        const int wq = warp & 3;                  // TMEM lanes 32*wq .. 32*wq+31
-        const int half = (warp - WARP_EPI) >> 2;  // tokens 128*half .. 128*half+127 of the tile
-        const int ew = warp - WARP_EPI;
+        const int wq = warp & 3;                   // TMEM lanes 32*wq .. 32*wq+31 = tokens
+        const int half = (warp - WARP_EPI) >> 2;   // features 128*half .. 128*half+127
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
-        float *w_scale = s_scale + ew * (BT / 2);  // this warp's copy: no cross-warp barrier
-        int32_t *w_rsum = s_rsum + ew * (BT / 2);
         const float gamma = *gamma_ptr;
-        const bool odd = lane & 1;
         for (int t = 0; t < my_tiles; ++t) {
-            const int tile = blockIdx.x + t * gridDim.x;
-            const int nw = tile % n_wtiles;
-            const int mt = tile / n_wtiles;
+            const int tile = pair + t * npairs;
+            const int nf = tile % n_ftiles;
+            const int mt = tile / n_ftiles;
             const int ab = t & 1;
-            __syncwarp();  // the previous tile's scales are no longer read
-#pragma unroll
-            for (int i = 0; i < BT / 64; ++i) {
-                const int ml = i * 32 + lane;
-                const int64_t m = (int64_t)mt * BT + half * (BT / 2) + ml;
-                w_scale[ml] = m < M ? scales[m] * gamma : 0.f;
-                w_rsum[ml] = m < M ? rowsum[m] : 0;
-            }
+            const int64_t m = (int64_t)mt * BM + (int)rank * HM + wq * 32 + lane;
+            const bool m_ok = m < M;
+            const float sc = m_ok ? scales[m] * gamma : 0.f;
+            const int rs = m_ok ? rowsum[m] : 0;
             if (!warp_wait(&bar->acc_full[ab], (uint32_t)(t >> 1) & 1, status, lane)) break;
             tc_fence_after();
-            const int n = nw * BW + wq * 32 + lane;  // this lane's output feature
 #pragma unroll 1
-            for (int ch = 0; ch < BT / 64; ++ch) {
+            for (int ch = 0; ch < HN / 32; ++ch) {
+                const int col = half * HN + ch * 32;
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(t_lane + ab * BT + half * (BT / 2) + ch * 32, v);
+                tmem_ld_32x32b_x32(t_lane + ab * BN + col, v);
                 tmem_wait_ld();
-                const int64_t m_base = (int64_t)mt * BT + half * (BT / 2) + ch * 32;
+                const int n0 = nf * BN + col;
                 if constexpr (OUT_I32) {
-                    int32_t *out = reinterpret_cast<int32_t *>(Yout);
+                    int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int64_t m = m_base + i;
-                        if (m < M && n < N) out[m * N + n] = (int)v[i] - w_rsum[ch * 32 + i];
+                    for (int j = 0; j < 8; ++j) {
+                        const int n = n0 + 4 * j;
+                        if (m_ok && n < N)
+                            *reinterpret_cast<int4 *>(row + n) =
+                                make_int4((int)v[4 * j] - rs, (int)v[4 * j + 1] - rs,
+                                          (int)v[4 * j + 2] - rs, (int)v[4 * j + 3] - rs);
                     }
                 } else {
-                    // this lane holds column n of rows i; lane pairs swap one value so the even
-                    // lane stores row i (n, n+1) and the odd lane row i+1 (n-1, n): each half-warp
-                    // writes one contiguous 64-byte row segment
-                    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(Yout);
-                    const int n_pair = nw * BW + wq * 32 + (lane & ~1);
+                    __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(Yout) + m * N;
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int m0 = ch * 32 + i;
-                        const float2 sc = *reinterpret_cast<const float2 *>(w_scale + m0);
-                        const int2 rs = *reinterpret_cast<const int2 *>(w_rsum + m0);
-                        const float y0 = (float)((int)v[i] - rs.x) * sc.x;
-                        const float y1 = (float)((int)v[i + 1] - rs.y) * sc.y;
-                        const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? y0 : y1, 1);
-                        const __nv_bfloat162 pr =
-                            odd ? __floats2bfloat162_rn(other, y1) : __floats2bfloat162_rn(y0, other);
-                        const int64_t m = m_base + i + (odd ? 1 : 0);
-                        if (m < M && n_pair < N)
-                            *reinterpret_cast<__nv_bfloat162 *>(out + m * N + n_pair) = pr;
+                    for (int i = 0; i < 16; ++i) {
+                        const float y0 = (float)((int)v[2 * i] - rs) * sc;
+                        const float y1 = (float)((int)v[2 * i + 1] - rs) * sc;
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+                        pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int n = n0 + 8 * j;
+                        if (m_ok && n < N)
+                            *reinterpret_cast<uint4 *>(row + n) =
+                                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->acc_empty[ab]);
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->acc_empty[ab]), 0));
         }
-    } else if (BITS == 4 && warp >= WARP_B4 && warp < WARP_B4 + 4) {
-        // ------------------------------------------------------------------ INT4 B producer
-        // warp w covers tokens 64w .. 64w+63 of the tile; in sub-step i, lane l loads the
-        // 16-byte quarter (l % 4) of token 64w + 8i + l / 4: 8 tokens x 64 B per instruction,
+    } else if (BITS == 4 && warp >= WARP_A4 && warp < WARP_A4 + 4) {
+        // ------------------------------------------------------------------ INT4 code producer
+        // warp w covers tokens 32w .. 32w+31 of this CTA's half; in sub-step i, lane l loads the
+        // 16-byte quarter (l % 4) of token 32w + 8i + l / 4: 8 tokens x 64 B per instruction,
         // fully used sectors.  The next stage's bytes are loaded before this one is stored.
-        const int wq = warp - WARP_B4;
+        const int wq = warp - WARP_A4;
         const int q = lane & 3;
-        uint4 nxt[8];
+        uint4 nxt[4];
         auto fetch = [&](int it2) {
             const int t2 = it2 / KS, ks2 = it2 - t2 * KS;
-            const int tile2 = blockIdx.x + t2 * gridDim.x;
-            const int64_t mbase = (int64_t)(tile2 / n_wtiles) * BT + wq * 64 + (lane >> 2);
+            const int tile2 = pair + t2 * npairs;
+            const int64_t mbase =
+                (int64_t)(tile2 / n_ftiles) * BM + (int)rank * HM + wq * 32 + (lane >> 2);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const int64_t m = mbase + 8 * i;
                 nxt[i] = (it2 < total && m < M)
                              ? ldg_nc_v4(codes4 + m * (K / 2) + ks2 * (BK / 2) + q * 16)
@@ -373,17 +377,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         };
         fetch(0);
         for (int it = 0; it < total; ++it) {
-            const int s = it % B_STAGES;
-            uint4 raw[8];
+            const int s = it % A_STAGES;
+            uint4 raw[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) raw[i] = nxt[i];
+            for (int i = 0; i < 4; ++i) raw[i] = nxt[i];
             fetch(it + 1);
-            if (!warp_wait(&bar->empty_b[s], ((uint32_t)(it / B_STAGES) & 1) ^ 1, status, lane))
+            if (!warp_wait(&bar->empty_a[s], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status, lane))
                 break;
-            uint8_t *dst = sb + (size_t)s * B_STAGE_BYTES;
+            uint8_t *dst = sa + (size_t)s * A_STAGE_BYTES;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int row = wq * 64 + 8 * i + (lane >> 2);
+            for (int i = 0; i < 4; ++i) {
+                const int row = wq * 32 + 8 * i + (lane >> 2);
                 // 32 codes k = 32q .. 32q+31 -> chunks 2q (words x, y) and 2q+1 (words z, w)
                 const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
@@ -400,21 +404,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->full_b[s]);
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full_a[s]), 0));
         }
     }
 
+    // neither CTA leaves while the other may still signal its barriers or read its operands
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     if (warp == WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
+}
+
+// Co-resident pairs per device (a persistent grid of one pair per two SMs where the GPU's
+// layout allows it), looked up once per device and kernel instance.
+template <int BITS, bool OUT_I32>
+static int max_pairs(int num_sms) {
+    static int cache[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(num_sms & ~1), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, ternary_gemm_tc_kernel<BITS, OUT_I32>, &cfg) !=
+            cudaSuccess ||
+        clusters < 1) {
+        (void)cudaGetLastError();
+        clusters = num_sms / 2;
+    }
+    if (dev >= 0 && dev < 64) cache[dev] = clusters;
+    return clusters;
 }
 
 template <int BITS, bool OUT_I32>
 static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
-                               void *out, int grid, cudaStream_t stream) {
+                               void *out, int64_t tiles, int num_sms, cudaStream_t stream) {
     auto kern = ternary_gemm_tc_kernel<BITS, OUT_I32>;
     static bool configured[64] = {};
     int dev = 0;
@@ -425,7 +454,9 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(
+    const int pairs_max = max_pairs<BITS, OUT_I32>(num_sms);
+    const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
+    kern<<<2 * pairs, NUM_THREADS, SMEM_BYTES, stream>>>(
         mc, mw, out, reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum, a.gamma,
         (int)a.M, (int)a.N, (int)a.K, a.status);
     return cudaGetLastError();
@@ -449,29 +480,29 @@ static CUresult encode_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream) {
     using namespace tc;
-    const int64_t tiles = ((a.N + BW - 1) / BW) * ((a.M + BT - 1) / BT);
-    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM);
     CUtensorMap mc, mw;
     memset(&mc, 0, sizeof mc);
     memset(&mw, 0, sizeof mw);
+    // codes: [M rows][K bytes], one [128 tokens x 128 B] swizzled box per CTA and stage
     if (a.act_bits == 8 &&
         encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)a.K,
-                  (uint64_t)a.M, (uint64_t)a.K, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+                  (uint64_t)a.M, (uint64_t)a.K, BK, HM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    // packed weights: [N rows][K/4 bytes], one [128 x 64 B] box (two K stages) per tile
+    // packed weights: [N rows][K/4 bytes], one [128 features x 64 B] box (two K stages)
     if (encode_2d(encode_fn, &mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, (uint64_t)a.K / 4,
-                  (uint64_t)a.N, (uint64_t)a.K / 4, SPW * BK / 4, BW,
+                  (uint64_t)a.N, (uint64_t)a.K / 4, SPW * BK / 4, HN,
                   CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (a.Y) {
-        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, a.Y, grid, stream)
-                            : launch_tc_t<4, false>(a, mc, mw, a.Y, grid, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, a.Y, tiles, num_sms, stream)
+                            : launch_tc_t<4, false>(a, mc, mw, a.Y, tiles, num_sms, stream);
         if (e != cudaSuccess) return e;
     }
     if (a.acc) {
-        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, a.acc, grid, stream)
-                            : launch_tc_t<4, true>(a, mc, mw, a.acc, grid, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, a.acc, tiles, num_sms, stream)
+                            : launch_tc_t<4, true>(a, mc, mw, a.acc, tiles, num_sms, stream);
     }
     return e;
 }

@@ -31,10 +31,12 @@
 
 namespace bitnet {
 
-template <int LOGK>
+// Launch plan of the transform for K = 2^LOGK: team of 2^T_BITS threads per row, RING bf16 rows
+// per team in shared memory, TEAMS teams per CTA.
+template <int LOGK, int T_BITS_, int RING_, int TEAMS_>
 struct FwhtPlan {
     static constexpr int K = 1 << LOGK;
-    static constexpr int T_BITS = (LOGK - 7) > ((LOGK - 1) / 2) ? (LOGK - 7) : ((LOGK - 1) / 2);
+    static constexpr int T_BITS = T_BITS_;
     static constexpr int TEAM = 1 << T_BITS;
     static constexpr int V_BITS = LOGK - T_BITS;
     static constexpr int V = 1 << V_BITS;  // values per thread
@@ -42,22 +44,42 @@ struct FwhtPlan {
     static constexpr int L = 1 << L_BITS;  // run length held by one thread in phase B
     static constexpr int COLS = V / L;     // runs per thread
     static constexpr int SHFL_BITS = T_BITS + 1 - L_BITS;  // bits done by lane shuffles
-    // bf16 rows per team in shared memory: the current one and the next (one for K = 2^15,
-    // where two would not fit next to the 128 KB transpose buffer)
-    static constexpr int RING = K <= 16384 ? 2 : 1;
+    // bf16 rows per team in shared memory: the current one, and with RING = 2 the next
+    static constexpr int RING = RING_;
     // per team: the fp32 transpose buffer (4K bytes) and RING bf16 rows (2K bytes each)
     static constexpr int TEAM_BYTES = K * 4 + RING * K * 2;
-    static constexpr int TPC_A = 128 / TEAM > 0 ? 128 / TEAM : 1;
-    static constexpr int TPC_B = 65536 / TEAM_BYTES > 0 ? 65536 / TEAM_BYTES : 1;  // <= 64 KB
-    static constexpr int TEAMS = TPC_A < TPC_B ? TPC_A : TPC_B;
+    static constexpr int TEAMS = TEAMS_;
     static constexpr int THREADS = TEAMS * TEAM;
-    static constexpr int CHUNKS = L / 4;                      // 16-byte chunks per run
+    // resident CTAs per SM the register allocation is sized for: 16 warps per SM
+    static constexpr int MIN_BLOCKS = THREADS >= 512 ? 1 : 512 / THREADS;
+    static constexpr int WARPS_PER_TEAM = TEAM >= 32 ? TEAM / 32 : 1;
+    static constexpr int RED = TEAMS * WARPS_PER_TEAM;         // reduction slots (max, then sum)
+    static constexpr int RED_BYTES = (2 * RED * 4 + 15) / 16 * 16;
+    static constexpr int CHUNKS = L / 4;                       // 16-byte chunks per run
     static constexpr int SWZ = (CHUNKS < 8 ? CHUNKS : 8) - 1;  // chunk XOR mask
     static constexpr size_t SMEM =
-        (size_t)TEAMS * TEAM_BYTES + 64 * sizeof(float) + (size_t)TEAMS * RING * sizeof(uint64_t);
-    static_assert(SHFL_BITS >= 0 && SHFL_BITS <= 5, "plan");
+        (size_t)TEAMS * TEAM_BYTES + RED_BYTES + (size_t)TEAMS * RING * sizeof(uint64_t);
+    static_assert(SHFL_BITS >= 0 && SHFL_BITS <= 5, "plan: shuffle partners inside a warp");
     static_assert(L >= 16, "runs must hold 16 codes");
+    static_assert(V <= 128, "plan: register budget");
+    static_assert(THREADS <= 1024 && THREADS % 32 == 0, "plan: CTA size");
+    static_assert(TEAM <= 32 || TEAMS <= 15, "plan: one named barrier per team");
+    static_assert(SMEM <= 227 * 1024, "plan: shared memory");
 };
+
+// The plan each K runs with.  Values per thread stay <= 64 from K = 2^11 up (<= 96 registers),
+// with one bf16 row per team, so that 16 or more warps per SM keep rows in flight; the bits a
+// thread does not hold in phase B go through lane shuffles.
+template <int LOGK> struct FwhtConfig;
+template <> struct FwhtConfig<7> { using P = FwhtPlan<7, 3, 2, 16>; };
+template <> struct FwhtConfig<8> { using P = FwhtPlan<8, 3, 2, 16>; };
+template <> struct FwhtConfig<9> { using P = FwhtPlan<9, 4, 2, 8>; };
+template <> struct FwhtConfig<10> { using P = FwhtPlan<10, 4, 2, 8>; };
+template <> struct FwhtConfig<11> { using P = FwhtPlan<11, 5, 1, 4>; };
+template <> struct FwhtConfig<12> { using P = FwhtPlan<12, 6, 1, 2>; };
+template <> struct FwhtConfig<13> { using P = FwhtPlan<13, 7, 1, 1>; };
+template <> struct FwhtConfig<14> { using P = FwhtPlan<14, 8, 1, 1>; };
+template <> struct FwhtConfig<15> { using P = FwhtPlan<15, 9, 1, 1>; };
 
 __device__ __forceinline__ float2 bfly_add(float2 a, float2 b) { return add2_rn(a, b); }
 __device__ __forceinline__ float2 bfly_sub(float2 a, float2 b) {
@@ -74,12 +96,11 @@ __device__ __forceinline__ void team_sync(int team) {
     }
 }
 
-template <int LOGK, int BITS, bool ZOUT>
-__global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
+template <class P, int BITS, bool ZOUT>
+__global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     fwht_quant_kernel(const uint8_t *__restrict__ X, int M, float rsqrt_k,
                       uint8_t *__restrict__ codes, float *__restrict__ scales,
                       int32_t *__restrict__ rowsum, float *__restrict__ zout, int *status) {
-    using P = FwhtPlan<LOGK>;
     constexpr int K = P::K, TEAM = P::TEAM, V = P::V, L = P::L;
     extern __shared__ float4 smem4[];
     float *smem = reinterpret_cast<float *>(smem4);
@@ -87,8 +108,8 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
     const int r = threadIdx.x % TEAM;
     const int lane = threadIdx.x & 31;
     float *tbuf = smem + team * K;
-    float *red = smem + P::TEAMS * K;  // 64 floats of reduction scratch
-    uint8_t *rows = reinterpret_cast<uint8_t *>(red + 64);  // [TEAMS][RING][K] bf16
+    float *red = smem + P::TEAMS * K;  // [RED] floats (max), then [RED] ints (code sums)
+    uint8_t *rows = reinterpret_cast<uint8_t *>(red) + P::RED_BYTES;  // [TEAMS][RING][K] bf16
     uint64_t *bars = reinterpret_cast<uint64_t *>(rows + (size_t)P::TEAMS * P::RING * K * 2);
     uint8_t *ring = rows + (size_t)team * P::RING * K * 2;
     uint64_t *rbar = bars + team * P::RING;
@@ -236,11 +257,12 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
         for (int o = W / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
         if constexpr (TEAM > 32) {
             // all warps of this team finished their phase-B reads of tbuf before this barrier
-            if (lane == 0) red[team * 8 + (r >> 5)] = mx;
+            constexpr int WPT = P::WARPS_PER_TEAM;
+            if (lane == 0) red[team * WPT + (r >> 5)] = mx;
             team_sync<TEAM>(team);
-            mx = red[team * 8];
+            mx = red[team * WPT];
 #pragma unroll
-            for (int i = 1; i < TEAM / 32; ++i) mx = fmaxf(mx, red[team * 8 + i]);
+            for (int i = 1; i < WPT; ++i) mx = fmaxf(mx, red[team * WPT + i]);
         }
         constexpr float Q = BITS == 4 ? 7.f : 127.f;
         const float g = fmaxf(mx, 1e-5f);
@@ -298,12 +320,13 @@ __global__ void __launch_bounds__(FwhtPlan<LOGK>::THREADS)
 #pragma unroll
         for (int o = W / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
         if constexpr (TEAM > 32) {
-            int *redi = reinterpret_cast<int *>(red) + 32;
-            if (lane == 0) redi[team * 8 + (r >> 5)] = sum;
+            constexpr int WPT = P::WARPS_PER_TEAM;
+            int *redi = reinterpret_cast<int *>(red) + P::RED;
+            if (lane == 0) redi[team * WPT + (r >> 5)] = sum;
             team_sync<TEAM>(team);
             sum = 0;
 #pragma unroll
-            for (int i = 0; i < TEAM / 32; ++i) sum += redi[team * 8 + i];
+            for (int i = 0; i < WPT; ++i) sum += redi[team * WPT + i];
         }
         if (valid && r == 0) {
             scales[row] = dq;
@@ -376,11 +399,10 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <int LOGK, int BITS, bool ZOUT>
+template <class P, int BITS, bool ZOUT>
 static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *scales,
                                  int32_t *rowsum, float *zout, int *status, cudaStream_t stream) {
-    using P = FwhtPlan<LOGK>;
-    auto kern = fwht_quant_kernel<LOGK, BITS, ZOUT>;
+    auto kern = fwht_quant_kernel<P, BITS, ZOUT>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -411,10 +433,11 @@ template <int LOGK>
 static cudaError_t launch_fwht_k(const void *X, int64_t M, int act_bits, void *codes,
                                  float *scales, int32_t *rowsum, float *zout, int *status,
                                  cudaStream_t stream) {
-    if (zout) return launch_fwht_t<LOGK, 8, true>(X, M, codes, scales, rowsum, zout, status, stream);
+    using P = typename FwhtConfig<LOGK>::P;
+    if (zout) return launch_fwht_t<P, 8, true>(X, M, codes, scales, rowsum, zout, status, stream);
     if (act_bits == 4)
-        return launch_fwht_t<LOGK, 4, false>(X, M, codes, scales, rowsum, zout, status, stream);
-    return launch_fwht_t<LOGK, 8, false>(X, M, codes, scales, rowsum, zout, status, stream);
+        return launch_fwht_t<P, 4, false>(X, M, codes, scales, rowsum, zout, status, stream);
+    return launch_fwht_t<P, 8, false>(X, M, codes, scales, rowsum, zout, status, stream);
 }
 
 cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,

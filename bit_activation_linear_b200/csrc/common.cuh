@@ -49,6 +49,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
         : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive_count(uint64_t *bar, uint32_t count) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+        "r"(count)
+        : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile(
         "{\n\t.reg .b64 st;\n\t"

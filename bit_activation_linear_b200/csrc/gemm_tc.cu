@@ -11,26 +11,30 @@
 // output features with tcgen05.mma.cta_group::2: D[256 x 256] += A[256 x 32] * B[256 x 32]^T,
 // A = activation codes (signed), B = weight offset codes u = q + 1 in {0, 1, 2} (unsigned).
 // CTA r of the pair holds tokens 128r .. 128r+127 of A, features 128r .. 128r+127 of B and
-// accumulator rows (tokens) 128r .. 128r+127 for all 256 features.  Against one CTA computing a
-// 128 x 256 tile alone, each SM moves half the activation bytes from L2 and through shared
-// memory per multiply-add: measured on B200, a lone CTA spent ~1050 cycles per 128-deep K stage
-// on 512 cycles of tensor work, its operand traffic (TMA and unpack writes plus tensor-core reads)
-// saturating shared memory and the L2->SM path.
+// accumulator rows (tokens) 128r .. 128r+127 for all 256 features, so each SM moves half the
+// activation bytes per multiply-add that a lone CTA with a 128 x 256 tile would.
 //
-// K runs in stages of 128 (four K=32 MMAs, 512 tensor cycles).  The two 256-column int32
-// accumulators fill the 512 TMEM columns, so a tile's epilogue overlaps the next tile's MMAs.
-// Warp roles, in both CTAs unless noted:
-//   warp 0       code-tile TMA (INT8): [128 tokens x 128 B] with the 128-byte swizzle (the UMMA
-//                K-major layout); the pair form of the copy completes on the even CTA's barrier,
-//                which expects both halves.
-//   warp 2       packed-weight TMA: [128 features x 64 B] (two K stages) into a local ring.
+// K runs in stages of 256: eight K=32 MMAs (1024 tensor cycles) per readiness test and commit.
+// Measured on B200, issuing one MMA costs ~45-65 cycles and a readiness test ~100, so with
+// 128-deep stages the issuing thread itself used ~900 of every 512 tensor cycles.  A stage
+// holds each operand as two 128-deep sub-tiles [128 rows x 128 B] in the 128-byte-swizzled
+// K-major layout.  The two 256-column int32 accumulators fill the 512 TMEM columns, so a tile's
+// epilogue overlaps the next tile's MMAs.
+// Warp roles, in both CTAs unless noted (warps 5, 9, 13 stay idle so that the scheduler
+// partition of the MMA warp hosts only it and two epilogue warps):
+//   warp 0       code TMA.  INT8: two [128 tokens x 128 B] boxes per stage; the pair form of the
+//                copy completes on the even CTA's stage barrier, which expects all four boxes.
+//                INT4: one [128 tokens x 128 B] box of packed nibbles into the second sub-tile.
+//   warp 2       packed-weight TMA: [128 features x 64 B] (one stage), 64-byte swizzle, into a
+//                local ring.
 //   warp 1       even CTA: MMA issuer (one thread).  Both CTAs: tensor-memory allocation.
-//   warps 4-11   weight unpack (two groups taking alternate stages; one group for INT4): thread i
-//                expands the 32 packed bytes of feature i for the stage (one shift-and-mask per
-//                four weights) into 128 bytes of the swizzled layout, then signals the even CTA.
-//   warps 8-11   (INT4 only) code producers: 16-byte loads of nibble codes, sign-extended to
-//                int8 in registers, stored in the swizzled layout.
-//   warps 12-19  epilogue: thread = token row; tcgen05.ld of 32 features, subtract the token's
+//   unpack warps (two groups of four taking alternate stages; one group for INT4): thread i
+//                expands the 64 packed bytes of feature i for the stage (one shift-and-mask per
+//                four weights) into 256 bytes of the swizzled layout, then signals the even CTA
+//                and releases the packed-weight slot.
+//   code warps   (INT4 only) thread = token row sign-extends its 256 packed codes in place to
+//                int8 in both sub-tiles.
+//   warps 16-23  epilogue: thread = token row; tcgen05.ld of 32 features, subtract the token's
 //                code sum (sum_k c*q = sum_k c*u - sum_k c), scale by d_m * gamma, round to bf16,
 //                64 contiguous bytes per thread and chunk.
 // Commits multicast to both CTAs; every wait is bounded: after ~1 s a role records
@@ -48,32 +52,50 @@ constexpr int BM = 256;            // tokens per pair tile (MMA M)
 constexpr int BN = 256;            // output features per pair tile (MMA N)
 constexpr int HM = BM / 2;         // tokens held by one CTA
 constexpr int HN = BN / 2;         // features held by one CTA
-constexpr int BK = 128;            // K per stage: one 128-byte swizzled row of int8
+constexpr int BK = 256;            // K per stage
+constexpr int SUBK = 128;          // K per sub-tile: one 128-byte swizzled row of int8
 constexpr int UMMA_K = 32;
-constexpr int MMAS = BK / UMMA_K;  // 4 per stage
-constexpr int A_STAGES = 6;        // code tiles in flight
-constexpr int B_STAGES = 4;        // unpacked weight tiles
-constexpr int W_STAGES = 4;        // packed-weight tiles in flight
-constexpr int SPW = 2;             // K stages per packed-weight tile [128 features x 64 B]
+constexpr int MMAS = BK / UMMA_K;  // 8 per stage
+constexpr int STAGES = 3;          // operand stages in flight
+constexpr int W_STAGES = 4;        // packed-weight tiles in flight (one per stage)
 constexpr int ACC_BUFS = 2;
 constexpr int TMEM_COLS = 512;
-constexpr int A_STAGE_BYTES = HM * BK;               // 16 KB
-constexpr int B_STAGE_BYTES = HN * BK;               // 16 KB
-constexpr int W_STAGE_BYTES = HN * SPW * BK / 4;     // 8 KB
+constexpr int SUB_BYTES = 128 * SUBK;                // 16 KB: [128 rows x 128 B]
+constexpr int A_STAGE_BYTES = 2 * SUB_BYTES;         // 32 KB of codes per CTA
+constexpr int B_STAGE_BYTES = 2 * SUB_BYTES;         // 32 KB of unpacked weights per CTA
+constexpr int W_STAGE_BYTES = HN * BK / 4;           // 8 KB of packed weights per CTA
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t IDESC = idesc_i8_s8u8(BM, BN);
 static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM budget");
 
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_B0 = 4, WARP_A4 = 8, WARP_EPI = 12;
-constexpr int NUM_THREADS = 20 * 32;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_EPI = 16;
+constexpr int NUM_THREADS = 24 * 32;
+
+// Unpack / code warps: eight warps outside the MMA warp's scheduler partition (warp % 4 == 1).
+// Returns 0..7, or -1 for every other warp.
+__device__ __forceinline__ int worker_index(int w) {
+    switch (w) {
+        case 4: return 0;
+        case 6: return 1;
+        case 7: return 2;
+        case 8: return 3;
+        case 10: return 4;
+        case 11: return 5;
+        case 12: return 6;
+        case 14: return 7;
+        default: return -1;
+    }
+}
 
 struct __align__(8) Barriers {
-    uint64_t full_a[A_STAGES];     // even CTA: both halves of the code tile are in place
-    uint64_t empty_a[A_STAGES];    // both: the MMAs that read the stage have completed
-    uint64_t full_b[B_STAGES];     // even CTA: the unpack warps of both CTAs wrote the stage
-    uint64_t empty_b[B_STAGES];    // both
+    // even CTA: the stage's code tiles of both CTAs are in place (INT8: the TMA bytes and one
+    // expect-tx arrival; INT4: the code warps of both CTAs) and the unpack warps of both CTAs
+    // have written their weight halves
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];        // both: the MMAs that read the stage have completed
+    uint64_t packed[STAGES];       // local, INT4: the packed codes of the stage have landed
     uint64_t full_w[W_STAGES];     // local packed-weight ring
-    uint64_t empty_w[W_STAGES];    // local; arrived by the MMA thread of the even CTA
+    uint64_t empty_w[W_STAGES];    // local; arrived by this CTA's unpack warps
     uint64_t acc_full[ACC_BUFS];   // both
     uint64_t acc_empty[ACC_BUFS];  // even CTA: the epilogue warps of both CTAs
     uint64_t done;                 // both: every MMA has completed
@@ -83,14 +105,14 @@ struct __align__(8) Barriers {
 // identical offsets in both CTAs: the pair MMA addresses the peer's operands by the even CTA's
 // shared-memory offsets
 constexpr size_t OFF_A = 0;
-constexpr size_t OFF_B = OFF_A + (size_t)A_STAGES * A_STAGE_BYTES;
-constexpr size_t OFF_W = OFF_B + (size_t)B_STAGES * B_STAGE_BYTES;
+constexpr size_t OFF_B = OFF_A + (size_t)STAGES * A_STAGE_BYTES;
+constexpr size_t OFF_W = OFF_B + (size_t)STAGES * B_STAGE_BYTES;
 constexpr size_t OFF_BAR = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + sizeof(Barriers) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast,
-// __syncwarp orders the other lanes after the acquire (needed before warp-collective tcgen05 ops).
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, __syncwarp orders the other
+// lanes after the acquire (needed before warp-collective tcgen05 ops).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *status, int lane) {
     bool ok = true;
     if (lane == 0) ok = mbar_wait(bar, parity, status);
@@ -103,8 +125,7 @@ template <int BITS, bool OUT_I32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                            const __grid_constant__ CUtensorMap tmap_w,
-                           void *__restrict__ Yout, const uint8_t *__restrict__ codes4,
-                           const float *__restrict__ scales,
+                           void *__restrict__ Yout, const float *__restrict__ scales,
                            const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
                            int M, int N, int K, int *status) {
     extern __shared__ uint8_t smem_raw[];
@@ -117,6 +138,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int wi = worker_index(warp);
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int pair = blockIdx.x >> 1;
@@ -124,25 +146,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int n_ftiles = (N + BN - 1) / BN;
     const int n_ttiles = (M + BM - 1) / BM;
     const int num_tiles = n_ftiles * n_ttiles;
-    const int KS = K / BK;                 // stages per tile
-    const int WPT = (KS + SPW - 1) / SPW;  // packed-weight tiles per output tile
+    const int KS = (K + BK - 1) / BK;  // stages per tile (the last one may be half: K % 256 = 128)
     constexpr int B_GROUPS = BITS == 8 ? 2 : 1;
     const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
     const int total = my_tiles * KS;  // (tile, stage) iterations of this pair
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < A_STAGES; ++s) {
-            // INT8: the even CTA's expect-tx arrival; INT4: the code warps of both CTAs
-            mbar_init(&bar->full_a[s], BITS == 8 ? 1 : 8);
-            mbar_init(&bar->empty_a[s], 1);
-        }
-        for (int s = 0; s < B_STAGES; ++s) {
-            mbar_init(&bar->full_b[s], 8);
-            mbar_init(&bar->empty_b[s], 1);
+        for (int s = 0; s < STAGES; ++s) {
+            // 8 unpack-warp arrivals (4 per CTA), plus the even CTA's expect-tx arrival (INT8)
+            // or 8 code-warp arrivals (INT4)
+            mbar_init(&bar->full[s], BITS == 8 ? 9 : 16);
+            mbar_init(&bar->empty[s], 1);
+            mbar_init(&bar->packed[s], 1);
         }
         for (int s = 0; s < W_STAGES; ++s) {
             mbar_init(&bar->full_w[s], 1);
-            mbar_init(&bar->empty_w[s], 1);
+            mbar_init(&bar->empty_w[s], 4);  // the four unpack warps of the stage's group
         }
         for (int s = 0; s < ACC_BUFS; ++s) {
             mbar_init(&bar->acc_full[s], 1);
@@ -152,7 +171,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         fence_mbar_init();
     }
     if (warp == WARP_TMA && lane == 0) {
-        if (BITS == 8) prefetch_tensormap(&tmap_codes);
+        prefetch_tensormap(&tmap_codes);
         prefetch_tensormap(&tmap_w);
     }
     if (warp == WARP_MMA) {
@@ -165,46 +184,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem = bar->tmem_base;
 
     if (warp == WARP_TMA) {
-        // ------------------------------------------------------------------ code-tile TMA
-        if (BITS == 8 && lane == 0) {
+        // ------------------------------------------------------------------ code TMA
+        if (lane == 0) {
             uint32_t issued = 0, ph = 0;  // for the final drain
-            int t = 0, ks = 0;
+            int t = 0, ks = 0, s = 0;
+            uint32_t p = 0;
             for (int it = 0; it < total; ++it) {
                 const int tile = pair + t * npairs;
-                const int s = it % A_STAGES;
-                const uint32_t p = (uint32_t)(it / A_STAGES) & 1;
-                if (!mbar_wait(&bar->empty_a[s], p ^ 1, status)) break;
-                if (leader) mbar_arrive_expect_tx(&bar->full_a[s], 2 * A_STAGE_BYTES);
-                tma_load_2d_pair(sa + (size_t)s * A_STAGE_BYTES, &tmap_codes, ks * BK,
-                                 (tile / n_ftiles) * BM + (int)rank * HM,
-                                 mapa_shared(smem_addr(&bar->full_a[s]), 0));
+                const int m0 = (tile / n_ftiles) * BM + (int)rank * HM;
+                if (!mbar_wait(&bar->empty[s], p ^ 1, status)) break;
+                uint8_t *dst = sa + (size_t)s * A_STAGE_BYTES;
+                if constexpr (BITS == 8) {
+                    if (leader) mbar_arrive_expect_tx(&bar->full[s], 4 * SUB_BYTES);
+                    const uint32_t fb = mapa_shared(smem_addr(&bar->full[s]), 0);
+                    tma_load_2d_pair(dst, &tmap_codes, ks * BK, m0, fb);
+                    tma_load_2d_pair(dst + SUB_BYTES, &tmap_codes, ks * BK + SUBK, m0, fb);
+                } else {
+                    // packed nibbles of the stage (128 B per token) into the second sub-tile,
+                    // widened in place by the code warps
+                    mbar_arrive_expect_tx(&bar->packed[s], SUB_BYTES);
+                    tma_load_2d(dst + SUB_BYTES, &tmap_codes, ks * (BK / 2), m0, &bar->packed[s]);
+                }
                 issued |= 1u << s;
                 ph = (ph & ~(1u << s)) | (p << s);
                 if (++ks == KS) { ks = 0; ++t; }
+                if (++s == STAGES) { s = 0; p ^= 1; }
             }
-            // no copy may still be writing shared memory when the CTA exits: the even CTA sees
-            // its barrier complete, the odd CTA sees the stage consumed (or gives up)
-            for (int i = 0; i < A_STAGES; ++i)
-                if (issued & (1u << i))
-                    mbar_wait(leader ? &bar->full_a[i] : &bar->empty_a[i], (ph >> i) & 1,
-                                 status);
+            // no copy may still be writing shared memory when the CTA exits: each CTA waits
+            // until the stages it loaded have been consumed (or gives up after the time limit)
+            for (int i = 0; i < STAGES; ++i)
+                if (issued & (1u << i)) mbar_wait(&bar->empty[i], (ph >> i) & 1, status);
         }
         __syncwarp();
     } else if (warp == WARP_WTMA) {
         // ------------------------------------------------------------------ weight-tile TMA
         if (lane == 0) {
             uint32_t issued = 0, ph = 0;
-            const int w_total = my_tiles * WPT;
-            for (int w = 0; w < w_total; ++w) {
-                const int s_w = w % W_STAGES;
-                const uint32_t p_w = (uint32_t)(w / W_STAGES) & 1;
+            int t = 0, ks = 0, s_w = 0;
+            uint32_t p_w = 0;
+            for (int it = 0; it < total; ++it) {
+                const int tile = pair + t * npairs;
                 if (!mbar_wait(&bar->empty_w[s_w], p_w ^ 1, status)) break;
-                const int tile_w = pair + (w / WPT) * npairs;
                 mbar_arrive_expect_tx(&bar->full_w[s_w], W_STAGE_BYTES);
-                tma_load_2d(sw + (size_t)s_w * W_STAGE_BYTES, &tmap_w, (w % WPT) * SPW * (BK / 4),
-                            (tile_w % n_ftiles) * BN + (int)rank * HN, &bar->full_w[s_w]);
+                tma_load_2d(sw + (size_t)s_w * W_STAGE_BYTES, &tmap_w, ks * (BK / 4),
+                            (tile % n_ftiles) * BN + (int)rank * HN, &bar->full_w[s_w]);
                 issued |= 1u << s_w;
                 ph = (ph & ~(1u << s_w)) | (p_w << s_w);
+                if (++ks == KS) { ks = 0; ++t; }
+                if (++s_w == W_STAGES) { s_w = 0; p_w ^= 1; }
             }
             for (int i = 0; i < W_STAGES; ++i)
                 if (issued & (1u << i)) mbar_wait(&bar->full_w[i], (ph >> i) & 1, status);
@@ -215,87 +242,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (leader && lane == 0) {
             const uint32_t sa_addr = smem_addr(sa);
             const uint32_t sb_addr = smem_addr(sb);
-            bool next_a = total > 0 && mbar_test_wait(&bar->full_a[0], 0);
-            bool next_b = total > 0 && mbar_test_wait(&bar->full_b[0], 0);
-            int t = 0, ks = 0;
+            bool next = total > 0 && mbar_test_wait(&bar->full[0], 0);
+            int t = 0, ks = 0, s = 0;
+            uint32_t p = 0;
             for (int it = 0; it < total; ++it) {
                 const int ab = t & 1;
-                const int sa_i = it % A_STAGES, sb_i = it % B_STAGES;
                 if (ks == 0 &&
                     !mbar_wait(&bar->acc_empty[ab], ((uint32_t)(t >> 1) & 1) ^ 1, status))
                     break;
-                if ((!next_a &&
-                     !mbar_wait(&bar->full_a[sa_i], (uint32_t)(it / A_STAGES) & 1, status)) ||
-                    (!next_b &&
-                     !mbar_wait(&bar->full_b[sb_i], (uint32_t)(it / B_STAGES) & 1, status)))
-                    break;
+                if (!next && !mbar_wait(&bar->full[s], p, status)) break;
                 tc_fence_after();
-                // ask now whether the next stage is ready: the answers are needed only after this
-                // stage's MMAs have been issued, so their latency is hidden behind them
-                if (it + 1 < total) {
-                    next_a = mbar_test_wait(&bar->full_a[(it + 1) % A_STAGES],
-                                               (uint32_t)((it + 1) / A_STAGES) & 1);
-                    next_b = mbar_test_wait(&bar->full_b[(it + 1) % B_STAGES],
-                                               (uint32_t)((it + 1) / B_STAGES) & 1);
-                }
+                // ask now whether the next stage is ready: the answer is needed only after this
+                // stage's MMAs have been issued
+                const int s1 = s + 1 == STAGES ? 0 : s + 1;
+                next = mbar_test_wait(&bar->full[s1], s1 == 0 ? p ^ 1 : p);
                 const uint32_t d_tmem = tmem + ab * BN;
-                const uint64_t adesc =
-                    smem_desc_kmajor_sw128(sa_addr + (uint32_t)sa_i * A_STAGE_BYTES);
-                const uint64_t bdesc =
-                    smem_desc_kmajor_sw128(sb_addr + (uint32_t)sb_i * B_STAGE_BYTES);
+                const uint32_t a_st = sa_addr + (uint32_t)s * A_STAGE_BYTES;
+                const uint32_t b_st = sb_addr + (uint32_t)s * B_STAGE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < MMAS; ++kk)
-                    mma_i8_ss_pair(d_tmem, adesc + (uint64_t)(kk * UMMA_K / 16),
-                                   bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
-                                   (ks | kk) != 0 ? 1u : 0u);
-                mma_commit_pair(&bar->empty_a[sa_i], 3);
-                mma_commit_pair(&bar->empty_b[sb_i], 3);
-                // the unpack warps of both CTAs are done with this packed-weight tile (full_b
-                // observed for its last stage): both may refill it
-                if (ks % SPW == SPW - 1 || ks == KS - 1) {
-                    uint64_t *ew = &bar->empty_w[(t * WPT + ks / SPW) % W_STAGES];
-                    mbar_arrive(ew);
-                    mbar_arrive_cluster(mapa_shared(smem_addr(ew), 1));
+                for (int sub = 0; sub < 2; ++sub) {
+                    const uint64_t adesc = smem_desc_kmajor_sw128(a_st + sub * SUB_BYTES);
+                    const uint64_t bdesc = smem_desc_kmajor_sw128(b_st + sub * SUB_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < SUBK / UMMA_K; ++kk)
+                        mma_i8_ss_pair(d_tmem, adesc + (uint64_t)(kk * UMMA_K / 16),
+                                       bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
+                                       (ks | sub | kk) != 0 ? 1u : 0u);
                 }
+                mma_commit_pair(&bar->empty[s], 3);
                 if (ks == KS - 1) mma_commit_pair(&bar->acc_full[ab], 3);
                 if (++ks == KS) { ks = 0; ++t; }
+                s = s1;
+                if (s == 0) p ^= 1;
             }
             // every MMA issued above has finished before either CTA releases tensor memory
             mma_commit_pair(&bar->done, 3);
         }
         if (lane == 0) mbar_wait(&bar->done, 0, status);
         __syncwarp();
-    } else if (warp >= WARP_B0 && warp < WARP_B0 + 4 * B_GROUPS) {
+    } else if (wi >= 0 && wi < 4 * B_GROUPS) {
         // ------------------------------------------------------------------ weight unpack
-        const int grp = (warp - WARP_B0) >> 2;  // takes iterations it = grp (mod B_GROUPS)
-        const int rr = (warp & 3) * 32 + lane;  // row of this CTA's B half = feature
+        const int grp = wi >> 2;             // takes iterations it = grp (mod B_GROUPS)
+        const int rr = (wi & 3) * 32 + lane;  // row of this CTA's B half = feature
+        const int sx = (rr >> 1) & 3;
         for (int it = grp; it < total; it += B_GROUPS) {
-            const int t = it / KS, ks = it - t * KS;
-            const int wseq = t * WPT + ks / SPW;
-            const int s_w = wseq % W_STAGES, s = it % B_STAGES;
-            if (!warp_wait(&bar->full_w[s_w], (uint32_t)(wseq / W_STAGES) & 1, status, lane)) break;
-            // row rr of the weight tile: SPW stages x 32 B
-            const uint4 *wsrc = reinterpret_cast<const uint4 *>(
-                sw + (size_t)s_w * W_STAGE_BYTES + rr * (SPW * BK / 4) + (ks % SPW) * (BK / 4));
-            const uint4 p0 = wsrc[0], p1 = wsrc[1];
-            const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            if (!warp_wait(&bar->empty_b[s], ((uint32_t)(it / B_STAGES) & 1) ^ 1, status, lane))
+            const int s = it % STAGES, s_w = it % W_STAGES;
+            if (!warp_wait(&bar->full_w[s_w], (uint32_t)(it / W_STAGES) & 1, status, lane)) break;
+            // row rr of the weight tile: 64 B, 16-byte chunk c stored at chunk c ^ ((rr >> 1) & 3)
+            // (64-byte swizzle: conflict-free reads down the rows)
+            const uint8_t *wrow = sw + (size_t)s_w * W_STAGE_BYTES + rr * (BK / 4);
+            uint32_t w[16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(wrow + ((c ^ sx) << 4));
+                w[4 * c] = v.x;
+                w[4 * c + 1] = v.y;
+                w[4 * c + 2] = v.z;
+                w[4 * c + 3] = v.w;
+            }
+            if (!warp_wait(&bar->empty[s], ((uint32_t)(it / STAGES) & 1) ^ 1, status, lane))
                 break;
             // packed word g holds k = 16g .. 16g+15; (w >> 2p) & 0x03030303 is k = 16g+4p .. +3,
-            // so word g becomes the 16-byte chunk g of the row, stored at chunk g ^ (rr & 7)
-            uint8_t *brow = sb + (size_t)s * B_STAGE_BYTES + rr * 128;
+            // so word g becomes 16-byte chunk g of the row: sub-tile g / 8, stored at chunk
+            // (g % 8) ^ (rr & 7)
+            uint8_t *brow = sb + (size_t)s * B_STAGE_BYTES + rr * SUBK;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) {
+            for (int g = 0; g < 16; ++g) {
                 uint4 o;
                 o.x = w[g] & 0x03030303u;
                 o.y = (w[g] >> 2) & 0x03030303u;
                 o.z = (w[g] >> 4) & 0x03030303u;
                 o.w = (w[g] >> 6) & 0x03030303u;
-                *reinterpret_cast<uint4 *>(brow + ((g ^ (rr & 7)) << 4)) = o;
+                *reinterpret_cast<uint4 *>(brow + (g >> 3) * SUB_BYTES + (((g & 7) ^ (rr & 7)) << 4)) =
+                    o;
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full_b[s]), 0));
+            if (lane == 0) {
+                mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full[s]), 0));
+                mbar_arrive(&bar->empty_w[s_w]);  // the packed tile was consumed above
+            }
         }
     } else if (warp >= WARP_EPI && warp < WARP_EPI + EPI_WARPS) {
         // ------------------------------------------------------------------ epilogue
@@ -354,42 +380,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->acc_empty[ab]), 0));
         }
-    } else if (BITS == 4 && warp >= WARP_A4 && warp < WARP_A4 + 4) {
-        // ------------------------------------------------------------------ INT4 code producer
-        // warp w covers tokens 32w .. 32w+31 of this CTA's half; in sub-step i, lane l loads the
-        // 16-byte quarter (l % 4) of token 32w + 8i + l / 4: 8 tokens x 64 B per instruction,
-        // fully used sectors.  The next stage's bytes are loaded before this one is stored.
-        const int wq = warp - WARP_A4;
-        const int q = lane & 3;
-        uint4 nxt[4];
-        auto fetch = [&](int it2) {
-            const int t2 = it2 / KS, ks2 = it2 - t2 * KS;
-            const int tile2 = pair + t2 * npairs;
-            const int64_t mbase =
-                (int64_t)(tile2 / n_ftiles) * BM + (int)rank * HM + wq * 32 + (lane >> 2);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int64_t m = mbase + 8 * i;
-                nxt[i] = (it2 < total && m < M)
-                             ? ldg_nc_v4(codes4 + m * (K / 2) + ks2 * (BK / 2) + q * 16)
-                             : make_uint4(0, 0, 0, 0);
-            }
-        };
-        fetch(0);
+    } else if (BITS == 4 && wi >= 4) {
+        // ------------------------------------------------------------------ INT4 code widening
+        // thread = token row of this CTA's half: its 128 packed bytes (256 codes) sit in the
+        // second sub-tile; it reads them all, then writes 256 int8 codes over both sub-tiles
+        // (the row's own 128-byte slots, so no other thread's input is overwritten)
+        const int row = (wi - 4) * 32 + lane;
+        const int sx = row & 7;
         for (int it = 0; it < total; ++it) {
-            const int s = it % A_STAGES;
-            uint4 raw[4];
+            const int s = it % STAGES;
+            if (!warp_wait(&bar->packed[s], (uint32_t)(it / STAGES) & 1, status, lane)) break;
+            uint8_t *arow = sa + (size_t)s * A_STAGE_BYTES + row * SUBK;
+            uint4 raw[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) raw[i] = nxt[i];
-            fetch(it + 1);
-            if (!warp_wait(&bar->empty_a[s], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status, lane))
-                break;
-            uint8_t *dst = sa + (size_t)s * A_STAGE_BYTES;
+            for (int c = 0; c < 8; ++c)
+                raw[c] = *reinterpret_cast<const uint4 *>(arow + SUB_BYTES + ((c ^ sx) << 4));
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = wq * 32 + 8 * i + (lane >> 2);
-                // 32 codes k = 32q .. 32q+31 -> chunks 2q (words x, y) and 2q+1 (words z, w)
-                const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+            for (int c = 0; c < 8; ++c) {
+                // 32 codes k = 32c .. 32c+31 -> 16-byte chunks 2c (words x, y) and 2c+1 (z, w)
+                const uint32_t wd[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const uint32_t w0 = wd[2 * h], w1 = wd[2 * h + 1];
@@ -398,13 +407,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     o.y = sext_nibbles((w0 >> 4) & 0x0F0F0F0Fu);
                     o.z = sext_nibbles(w1 & 0x0F0F0F0Fu);
                     o.w = sext_nibbles((w1 >> 4) & 0x0F0F0F0Fu);
-                    const int c = 2 * q + h;
-                    *reinterpret_cast<uint4 *>(dst + row * 128 + ((c ^ (row & 7)) << 4)) = o;
+                    const int oc = 2 * c + h;  // chunk of the 256-byte row: sub-tile oc / 8
+                    *reinterpret_cast<uint4 *>(arow + (oc >> 3) * SUB_BYTES + (((oc & 7) ^ sx) << 4)) =
+                        o;
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full_a[s]), 0));
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->full[s]), 0));
         }
     }
 
@@ -457,8 +467,7 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
     const int pairs_max = max_pairs<BITS, OUT_I32>(num_sms);
     const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     kern<<<2 * pairs, NUM_THREADS, SMEM_BYTES, stream>>>(
-        mc, mw, out, reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum, a.gamma,
-        (int)a.M, (int)a.N, (int)a.K, a.status);
+        mc, mw, out, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, (int)a.K, a.status);
     return cudaGetLastError();
 }
 
@@ -484,15 +493,18 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
     CUtensorMap mc, mw;
     memset(&mc, 0, sizeof mc);
     memset(&mw, 0, sizeof mw);
-    // codes: [M rows][K bytes], one [128 tokens x 128 B] swizzled box per CTA and stage
-    if (a.act_bits == 8 &&
-        encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, (uint64_t)a.K,
-                  (uint64_t)a.M, (uint64_t)a.K, BK, HM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    // codes: INT8 [M rows][K bytes], two [128 tokens x 128 B] boxes per CTA and stage;
+    // INT4 [M rows][K/2 bytes], one [128 tokens x 128 B] box of packed nibbles per CTA and stage;
+    // both with the 128-byte swizzle
+    const uint64_t cb = a.act_bits == 8 ? (uint64_t)a.K : (uint64_t)a.K / 2;
+    if (encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, cb, (uint64_t)a.M, cb,
+                  SUBK, HM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    // packed weights: [N rows][K/4 bytes], one [128 features x 64 B] box (two K stages)
+    // packed weights: [N rows][K/4 bytes], one [128 features x 64 B] box per stage, 64-byte
+    // swizzle
     if (encode_2d(encode_fn, &mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, (uint64_t)a.K / 4,
-                  (uint64_t)a.N, (uint64_t)a.K / 4, SPW * BK / 4, HN,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+                  (uint64_t)a.N, (uint64_t)a.K / 4, BK / 4, HN,
+                  CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (a.Y) {

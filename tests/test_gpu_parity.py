@@ -153,6 +153,7 @@ def staged_product(B, M, K, N, bits, seed):
     (1, 256, 256), (3, 384, 136), (8, 2048, 264),          # decode kernel
     (9, 256, 256), (130, 384, 136), (300, 2048, 264),       # tensor-core kernel, ragged tiles
     (256, 1024, 1024), (513, 128, 8),
+    (1000, 640, 520),                                       # several tiles, 2.5 K stages
 ])
 @pytest.mark.parametrize("bits", [8, 4])
 def test_product_int32_exact_and_bf16(B, M, K, N, bits):

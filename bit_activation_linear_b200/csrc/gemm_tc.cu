@@ -35,8 +35,11 @@
 //   code warps   (INT4 only) thread = token row sign-extends its 256 packed codes in place to
 //                int8 in both sub-tiles.
 //   warps 16-23  epilogue: thread = token row; tcgen05.ld of 32 features, subtract the token's
-//                code sum (sum_k c*q = sum_k c*u - sum_k c), scale by d_m * gamma, round to bf16,
-//                64 contiguous bytes per thread and chunk.
+//                code sum (sum_k c*q = sum_k c*u - sum_k c), scale by d_m * gamma, round to bf16;
+//                each warp stages [32 tokens x 16 features] boxes in shared memory and writes
+//                them with bulk tensor stores.  (Direct stores of one row per thread touch 32
+//                lines per instruction; on B200 they held up the unpack warps' shared-memory
+//                stores for ~6000 cycles per tile.)
 // Commits multicast to both CTAs; every wait is bounded: after ~1 s a role records
 // BITNET_ERR_TIMEOUT and stops; in-flight copies and MMAs are drained and both CTAs meet at a
 // cluster barrier before tensor memory is released.  No TMA multicast is used.
@@ -57,7 +60,7 @@ constexpr int SUBK = 128;          // K per sub-tile: one 128-byte swizzled row 
 constexpr int UMMA_K = 32;
 constexpr int MMAS = BK / UMMA_K;  // 8 per stage
 constexpr int STAGES = 3;          // operand stages in flight
-constexpr int W_STAGES = 4;        // packed-weight tiles in flight (one per stage)
+constexpr int W_STAGES = 3;        // packed-weight tiles in flight (one per stage)
 constexpr int ACC_BUFS = 2;
 constexpr int TMEM_COLS = 512;
 constexpr int SUB_BYTES = 128 * SUBK;                // 16 KB: [128 rows x 128 B]
@@ -65,6 +68,8 @@ constexpr int A_STAGE_BYTES = 2 * SUB_BYTES;         // 32 KB of codes per CTA
 constexpr int B_STAGE_BYTES = 2 * SUB_BYTES;         // 32 KB of unpacked weights per CTA
 constexpr int W_STAGE_BYTES = HN * BK / 4;           // 8 KB of packed weights per CTA
 constexpr int EPI_WARPS = 8;
+constexpr int Y_BOX_N = 16;                          // features per output box (32 B of bf16)
+constexpr int Y_BOX_BYTES = 32 * Y_BOX_N * 2;        // [32 tokens x 16 features] = 1 KB
 constexpr uint32_t IDESC = idesc_i8_s8u8(BM, BN);
 static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM budget");
 
@@ -107,7 +112,8 @@ struct __align__(8) Barriers {
 constexpr size_t OFF_A = 0;
 constexpr size_t OFF_B = OFF_A + (size_t)STAGES * A_STAGE_BYTES;
 constexpr size_t OFF_W = OFF_B + (size_t)STAGES * B_STAGE_BYTES;
-constexpr size_t OFF_BAR = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
+constexpr size_t OFF_Y = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;  // per epilogue warp
+constexpr size_t OFF_BAR = OFF_Y + (size_t)EPI_WARPS * Y_BOX_BYTES;
 constexpr size_t SMEM_BYTES = OFF_BAR + sizeof(Barriers) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
@@ -125,6 +131,7 @@ template <int BITS, bool OUT_I32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                            const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_y,
                            void *__restrict__ Yout, const float *__restrict__ scales,
                            const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
                            int M, int N, int K, int *status) {
@@ -134,6 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint8_t *sa = smem + OFF_A;
     uint8_t *sb = smem + OFF_B;
     uint8_t *sw = smem + OFF_W;
+    uint8_t *sy = smem + OFF_Y;
     Barriers *bar = reinterpret_cast<Barriers *>(smem + OFF_BAR);
 
     const int warp = threadIdx.x >> 5;
@@ -173,6 +181,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (warp == WARP_TMA && lane == 0) {
         prefetch_tensormap(&tmap_codes);
         prefetch_tensormap(&tmap_w);
+        if (!OUT_I32) prefetch_tensormap(&tmap_y);
     }
     if (warp == WARP_MMA) {
         tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
@@ -328,6 +337,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const int wq = warp & 3;                   // TMEM lanes 32*wq .. 32*wq+31 = tokens
         const int half = (warp - WARP_EPI) >> 2;   // features 128*half .. 128*half+127
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
+        uint8_t *ybox = sy + (size_t)(warp - WARP_EPI) * Y_BOX_BYTES;
         const float gamma = *gamma_ptr;
         for (int t = 0; t < my_tiles; ++t) {
             const int tile = pair + t * npairs;
@@ -358,7 +368,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                                           (int)v[4 * j + 2] - rs, (int)v[4 * j + 3] - rs);
                     }
                 } else {
-                    __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(Yout) + m * N;
+                    // bf16 pairs of this token's 32 features, then out through the warp's
+                    // staging box by bulk tensor stores: 16 features x 32 tokens per store, the
+                    // box rows in the 32-byte-swizzled layout (chunk c of row r at c ^ (r >> 2 & 1))
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -367,12 +379,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
                         pk[i] = *reinterpret_cast<const uint32_t *>(&h);
                     }
+                    const int m_w = mt * BM + (int)rank * HM + wq * 32;  // the warp's first token
+                    const int sx = (lane >> 2) & 1;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int n = n0 + 8 * j;
-                        if (m_ok && n < N)
-                            *reinterpret_cast<uint4 *>(row + n) =
-                                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    for (int hb = 0; hb < 2; ++hb) {
+                        if (lane == 0) bulk_wait_group_read<0>();  // the previous box was read
+                        __syncwarp();
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+                            *reinterpret_cast<uint4 *>(ybox + lane * (Y_BOX_N * 2) + ((c ^ sx) << 4)) =
+                                make_uint4(pk[8 * hb + 4 * c], pk[8 * hb + 4 * c + 1],
+                                           pk[8 * hb + 4 * c + 2], pk[8 * hb + 4 * c + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        // rows >= M and features >= N of a box are not written; a box wholly
+                        // outside Y is not issued
+                        if (lane == 0 && m_w < M && n0 + hb * Y_BOX_N < N) {
+                            tma_store_2d(&tmap_y, ybox, n0 + hb * Y_BOX_N, m_w);
+                            bulk_commit_group();
+                        }
                     }
                 }
             }
@@ -380,6 +405,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->acc_empty[ab]), 0));
         }
+        // the staging box stays in use until its last store has completed
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     } else if (BITS == 4 && wi >= 4) {
         // ------------------------------------------------------------------ INT4 code widening
         // thread = token row of this CTA's half: its 128 packed bytes (256 codes) sit in the
@@ -453,7 +481,8 @@ static int max_pairs(int num_sms) {
 
 template <int BITS, bool OUT_I32>
 static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
-                               void *out, int64_t tiles, int num_sms, cudaStream_t stream) {
+                               const CUtensorMap &my, void *out, int64_t tiles, int num_sms,
+                               cudaStream_t stream) {
     auto kern = ternary_gemm_tc_kernel<BITS, OUT_I32>;
     static bool configured[64] = {};
     int dev = 0;
@@ -467,7 +496,7 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
     const int pairs_max = max_pairs<BITS, OUT_I32>(num_sms);
     const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     kern<<<2 * pairs, NUM_THREADS, SMEM_BYTES, stream>>>(
-        mc, mw, out, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, (int)a.K, a.status);
+        mc, mw, my, out, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, (int)a.K, a.status);
     return cudaGetLastError();
 }
 
@@ -490,9 +519,10 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
                                    cudaStream_t stream) {
     using namespace tc;
     const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM);
-    CUtensorMap mc, mw;
+    CUtensorMap mc, mw, my;
     memset(&mc, 0, sizeof mc);
     memset(&mw, 0, sizeof mw);
+    memset(&my, 0, sizeof my);
     // codes: INT8 [M rows][K bytes], two [128 tokens x 128 B] boxes per CTA and stage;
     // INT4 [M rows][K/2 bytes], one [128 tokens x 128 B] box of packed nibbles per CTA and stage;
     // both with the 128-byte swizzle
@@ -508,13 +538,18 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (a.Y) {
-        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, a.Y, tiles, num_sms, stream)
-                            : launch_tc_t<4, false>(a, mc, mw, a.Y, tiles, num_sms, stream);
+        // bf16 output [M rows][N], one [32 tokens x 16 features] box per store, 32-byte swizzle
+        if (encode_2d(encode_fn, &my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, (uint64_t)a.N,
+                      (uint64_t)a.M, (uint64_t)a.N * 2, Y_BOX_N, 32,
+                      CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, my, a.Y, tiles, num_sms, stream)
+                            : launch_tc_t<4, false>(a, mc, mw, my, a.Y, tiles, num_sms, stream);
         if (e != cudaSuccess) return e;
     }
     if (a.acc) {
-        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, a.acc, tiles, num_sms, stream)
-                            : launch_tc_t<4, true>(a, mc, mw, a.acc, tiles, num_sms, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, my, a.acc, tiles, num_sms, stream)
+                            : launch_tc_t<4, true>(a, mc, mw, my, a.acc, tiles, num_sms, stream);
     }
     return e;
 }

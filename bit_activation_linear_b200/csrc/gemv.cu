@@ -7,102 +7,119 @@
 // the matching four activation codes accumulates sum_k u * c exactly; the per-token code sum
 // written by the quantiser removes the offset: sum_k q * c = sum_k u * c - sum_k c.
 //
-// One warp per output feature n; each lane streams 64 weights (one 16-byte load) per step, so a
-// warp reads 2 KB of consecutive packed weights per step.  Activation codes (at most 8 tokens,
-// a few KB) stay in L1/L2.
+// A warp owns R consecutive output features (R = 2 from four tokens up, so that each code load
+// serves two rows).  The K axis is walked in steps of 512 weights: in a step lane l takes the
+// packed word 32s + l of each row (weights k = 512s + 16l .. +15, one coalesced 128-byte load per
+// warp and row) and the 16 matching codes of each token (one coalesced 16-byte load per lane).
+// The weight words of eight steps are loaded before any is used, so every warp keeps 8R loads
+// in flight and the weight stream is requested at full rate.  Activation codes (at most eight
+// tokens) are read through L1, where every warp of the SM finds them.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace bitnet {
 
-template <int BITS, int T>
-__global__ void __launch_bounds__(256)
+constexpr int kGemvSteps = 16;      // 512-weight steps whose weight loads are in flight together
+constexpr int kGemvWarps = 4;       // warps per CTA
+
+template <int BITS, int T, int R>
+__global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                         const int32_t *__restrict__ rowsum, int M, int K,
-                        const uint4 *__restrict__ wp, const float *__restrict__ gamma_ptr, int N,
-                        int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y) {
+                        const uint32_t *__restrict__ wp, const float *__restrict__ gamma_ptr,
+                        int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y) {
     const int lane = threadIdx.x & 31;
-    const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (n >= N) return;
-    const uint4 *wrow = wp + (int64_t)n * (K / 64);  // 64 weights per uint4
-    int acc[T];
+    const int n0 = (blockIdx.x * kGemvWarps + (threadIdx.x >> 5)) * R;
+    if (n0 >= N) return;  // whole warp leaves together
+    const int words = K / 16;  // packed words per row
+    const int steps = (words + 31) / 32;  // the last step may be partial (K % 512 != 0)
+    int acc[R][T];
 #pragma unroll
-    for (int t = 0; t < T; ++t) acc[t] = 0;
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int t = 0; t < T; ++t) acc[r][t] = 0;
 
-    for (int c = lane; c < K / 64; c += 32) {
-        const uint4 w4 = ldg_nc_v4(wrow + c);
-        const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
-        // unpacked offset codes: u[4g + p] holds weights 64c + 16g + 4p .. +3
-        uint32_t u[16];
+    for (int s0 = 0; s0 < steps; s0 += kGemvSteps) {
+        uint32_t w[R][kGemvSteps];
 #pragma unroll
-        for (int g = 0; g < 4; ++g)
+        for (int j = 0; j < kGemvSteps; ++j)
 #pragma unroll
-            for (int p = 0; p < 4; ++p) u[4 * g + p] = (ww[g] >> (2 * p)) & 0x03030303u;
+            for (int r = 0; r < R; ++r)
+                w[r][j] = (32 * (s0 + j) + lane < words && n0 + r < N)
+                              ? __ldg(wp + (int64_t)(n0 + r) * words + 32 * (s0 + j) + lane)
+                              : 0u;
 #pragma unroll
-        for (int t = 0; t < T; ++t) {
-            if (t >= M) break;
-            if constexpr (BITS == 8) {
-                const uint4 *xr = reinterpret_cast<const uint4 *>(codes + (int64_t)t * K) + 4 * c;
+        for (int j = 0; j < kGemvSteps; ++j) {
+            if (s0 + j >= steps) break;
+            const int k0 = 512 * (s0 + j) + 16 * lane;
+            const bool k_in = k0 < K;  // lanes past the end of a partial step add zero
+            // codes k0 .. k0+15 of every token as four words of four int8 (word p = k0+4p .. +3),
+            // all loaded before the dot products (tokens t >= M read nothing and add zero)
+            uint32_t xs[T][4];
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    uint4 x = __ldg(xr + g);
-                    acc[t] = __dp4a((int)u[4 * g + 0], (int)x.x, acc[t]);
-                    acc[t] = __dp4a((int)u[4 * g + 1], (int)x.y, acc[t]);
-                    acc[t] = __dp4a((int)u[4 * g + 2], (int)x.z, acc[t]);
-                    acc[t] = __dp4a((int)u[4 * g + 3], (int)x.w, acc[t]);
-                }
-            } else {
-                // nibble storage: each 32-bit word holds codes k0..k0+3 (low nibbles) and
-                // k0+4..k0+7 (high nibbles)
-                const uint4 *xr =
-                    reinterpret_cast<const uint4 *>(codes + (int64_t)t * (K / 2)) + 2 * c;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint4 x = __ldg(xr + h);
-                    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int word = 4 * h + i;  // codes 8*word .. 8*word+7 of this 64
-                        uint32_t lo = sext_nibbles(xw[i] & 0x0F0F0F0Fu);
-                        uint32_t hi = sext_nibbles((xw[i] >> 4) & 0x0F0F0F0Fu);
-                        acc[t] = __dp4a((int)u[2 * word], (int)lo, acc[t]);
-                        acc[t] = __dp4a((int)u[2 * word + 1], (int)hi, acc[t]);
-                    }
+            for (int t = 0; t < T; ++t) {
+                uint32_t *x = xs[t];
+                if (!k_in || t >= M) {
+                    x[0] = x[1] = x[2] = x[3] = 0u;
+                } else if constexpr (BITS == 8) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(codes + (int64_t)t * K + k0));
+                    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+                } else {
+                    // nibble storage: each word holds codes k..k+3 (low nibbles), k+4..k+7 (high)
+                    const uint2 v =
+                        __ldg(reinterpret_cast<const uint2 *>(codes + (int64_t)t * (K / 2) + k0 / 2));
+                    x[0] = sext_nibbles(v.x & 0x0F0F0F0Fu);
+                    x[1] = sext_nibbles((v.x >> 4) & 0x0F0F0F0Fu);
+                    x[2] = sext_nibbles(v.y & 0x0F0F0F0Fu);
+                    x[3] = sext_nibbles((v.y >> 4) & 0x0F0F0F0Fu);
                 }
             }
+            // packed word: weight k0 + 4p + j at bits 8j + 2p, as offset codes u = q + 1
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const int u = (int)((w[r][j] >> (2 * p)) & 0x03030303u);
+#pragma unroll
+                    for (int t = 0; t < T; ++t) acc[r][t] = __dp4a(u, (int)xs[t][p], acc[r][t]);
+                }
         }
     }
     const float gamma = *gamma_ptr;
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
-        if (t >= M) break;
-        int s = acc[t];
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-        if (lane == t) {
-            const int a = s - rowsum[t];
-            if (acc_out) acc_out[(int64_t)t * N + n] = a;
-            if (Y) Y[(int64_t)t * N + n] = __float2bfloat16_rn((float)a * (scales[t] * gamma));
+        for (int t = 0; t < T; ++t) {
+            if (t >= M) break;
+            int s = acc[r][t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+            const int n = n0 + r;
+            if (lane == r * T + t && n < N) {
+                const int a = s - rowsum[t];
+                if (acc_out) acc_out[(int64_t)t * N + n] = a;
+                if (Y) Y[(int64_t)t * N + n] = __float2bfloat16_rn((float)a * (scales[t] * gamma));
+            }
         }
-    }
 }
 
-template <int BITS, int T>
+template <int BITS, int T, int R>
 static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
-    const unsigned blocks = (unsigned)((a.N + 7) / 8);
-    ternary_gemv_kernel<BITS, T><<<blocks, 256, 0, stream>>>(
+    static_assert(R * T <= 32, "one lane per (row, token) result");
+    const int64_t warps = (a.N + R - 1) / R;
+    const unsigned blocks = (unsigned)((warps + kGemvWarps - 1) / kGemvWarps);
+    ternary_gemv_kernel<BITS, T, R><<<blocks, kGemvWarps * 32, 0, stream>>>(
         reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum, (int)a.M, (int)a.K,
-        reinterpret_cast<const uint4 *>(a.Wp), a.gamma, (int)a.N, a.acc,
-        reinterpret_cast<__nv_bfloat16 *>(a.Y));
+        a.Wp, a.gamma, (int)a.N, a.acc, reinterpret_cast<__nv_bfloat16 *>(a.Y));
     return cudaGetLastError();
 }
 
 template <int BITS>
 static cudaError_t launch_gemv_b(const GemmArgs &a, cudaStream_t stream) {
-    if (a.M <= 1) return launch_gemv_t<BITS, 1>(a, stream);
-    if (a.M <= 2) return launch_gemv_t<BITS, 2>(a, stream);
-    if (a.M <= 4) return launch_gemv_t<BITS, 4>(a, stream);
-    return launch_gemv_t<BITS, 8>(a, stream);
+    if (a.M <= 1) return launch_gemv_t<BITS, 1, 1>(a, stream);
+    if (a.M <= 2) return launch_gemv_t<BITS, 2, 1>(a, stream);
+    if (a.M <= 4) return launch_gemv_t<BITS, 4, 2>(a, stream);
+    return launch_gemv_t<BITS, 8, 2>(a, stream);
 }
 
 cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream) {

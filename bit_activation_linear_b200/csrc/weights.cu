@@ -97,13 +97,21 @@ __global__ void __launch_bounds__(kWeightThreads)
     ternarize_pack_kernel(const uint4 *__restrict__ w, int64_t nwords, double n_weights,
                           const double *__restrict__ partials, int P, uint32_t *__restrict__ wp,
                           float *__restrict__ gamma_out) {
+    // the first 16 weights of this thread do not depend on gamma: their loads are issued before
+    // the reduction below, so the two memory latencies overlap
+    int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (i < nwords) {
+        a = ldg_nc_v4(w + 2 * i);
+        b = ldg_nc_v4(w + 2 * i + 1);
+    }
     // gamma from the P partial sums: a fixed assignment of partials to threads and a fixed
     // reduction tree, identical in every block, so gamma does not depend on the launch
     __shared__ double warp_sums[kWeightThreads / 32];
     __shared__ uint32_t s_thr;
     {
         double s = 0.0;
-        for (int i = threadIdx.x; i < P; i += kWeightThreads) s += partials[i];
+        for (int j = threadIdx.x; j < P; j += kWeightThreads) s += partials[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
         if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
@@ -119,10 +127,12 @@ __global__ void __launch_bounds__(kWeightThreads)
     }
     const uint32_t thr = s_thr;
     const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
-    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nwords; i += stride) {
+    for (bool first = true; i < nwords; i += stride, first = false) {
         // 16 consecutive weights k = 16i + e; weight e = 4p + j goes to bits 8j + 2p as u = q + 1.
-        uint4 a = ldg_nc_v4(w + 2 * i);
-        uint4 b = ldg_nc_v4(w + 2 * i + 1);
+        if (!first) {
+            a = ldg_nc_v4(w + 2 * i);
+            b = ldg_nc_v4(w + 2 * i + 1);
+        }
         const uint32_t h[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
         uint32_t word = 0;
 #pragma unroll

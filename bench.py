@@ -10,11 +10,10 @@ rescale (1 kernel).  Default workload: the Wo-shaped layer of a 2B-class model
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 cuda.synchronize on both sides, timed with CUDA events on the launching stream, max over ranks.
 Inputs are rotated over several copies whose total exceeds twice the L2 cache, so no step finds
-its inputs in L2.  Each copy's step is captured in two CUDA graphs so that host launch overhead
-does not starve the GPU: the preparation graph runs the weight ternarisation and the activation
-quantisation side by side on two streams (they are independent), the product graph runs the
-tensor-core product; CUDA events recorded around the product's replay give its live duration for
-the roofline figure.
+its inputs in L2.  Each copy's step is one CUDA graph, so host launch overhead does not starve
+the GPU: the weight ternarisation and the activation quantisation run side by side on two
+streams (they are independent), then the tensor-core product, bracketed by two timing events
+that are nodes of the same graph; they give the product's live duration for the roofline figure.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the data
@@ -323,34 +322,49 @@ def run_gpu(args, wl, rank, world, device):
     B.bitnet_sync_status(stream)
     launches_per_step = (B.bitnet_launch_count() - launches_before) // copies
 
-    graphs = []  # graphs[copy] = (prep graph, product graph)
+    # One CUDA graph per input copy holds the whole step.  Timing-event nodes inside a graph
+    # cost ~5 us per step on B200, so the timed loop replays event-free graphs, except for its
+    # last copies x SAMPLES steps: each of those replays, once, its own copy of the step graph
+    # whose product is bracketed by two timing events.  Those events give the product's live
+    # duration inside the timed region.
+    SAMPLES = 4
+    graphs, timed = [], []
     for b in bufs:
-        gp, gg = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gp, stream=stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
             prep(b)
-        with torch.cuda.graph(gg, stream=stream):
             gemm(b)
-        graphs.append((gp, gg))
+        graphs.append(g)
+        copy_timed = []
+        for _ in range(SAMPLES):
+            gt = torch.cuda.CUDAGraph()
+            ev = (torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True))
+            with torch.cuda.graph(gt, stream=stream):
+                prep(b)
+                ev[0].record(stream)
+                gemm(b)
+                ev[1].record(stream)
+            copy_timed.append((gt, ev))
+        timed.append(copy_timed)
     torch.cuda.synchronize(device)
+    n_timed = min(args.steps, copies * SAMPLES)
 
-    def step(i, ev=None):
-        gp, gg = graphs[i % copies]
-        gp.replay()
-        if ev is not None:
-            ev[0].record(stream)
-        gg.replay()
-        if ev is not None:
-            ev[1].record(stream)
+    def step(i, sampled=False):
+        if sampled:  # the j-th sampled step of copy i % copies uses that copy's j-th timed graph
+            j = (i - (args.steps - n_timed)) // copies
+            timed[i % copies][j][0].replay()
+        else:
+            graphs[i % copies].replay()
 
     for i in range(args.warmup):
         step(i)
+    for copy_timed in timed:  # first replays upload the sampled graphs outside the timed region
+        for gt, _ in copy_timed:
+            gt.replay()
     torch.cuda.synchronize(device)
     B.bitnet_sync_status(stream)
 
-    n_ev = min(args.steps, 512)
-    every = max(1, args.steps // n_ev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(n_ev)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
 
@@ -361,12 +375,8 @@ def run_gpu(args, wl, rank, world, device):
     # a short device sleep lets the host queue the first replays before the clock starts
     torch.cuda._sleep(int(2e7))
     t_start.record(stream)
-    k_ev = 0
     for i in range(args.steps):
-        use = (i % every == 0) and k_ev < n_ev
-        step(i, evs[k_ev] if use else None)
-        if use:
-            k_ev += 1
+        step(i, sampled=i >= args.steps - n_timed)
     t_end.record(stream)
     torch.cuda.synchronize(device)
     barrier()
@@ -374,7 +384,13 @@ def run_gpu(args, wl, rank, world, device):
     B.bitnet_sync_status(stream)
 
     elapsed_ms = t_start.elapsed_time(t_end)
-    gemm_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(k_ev))
+    # the product's duration in each sampled step (all inside the timed region)
+    samples = []
+    for i in range(args.steps - n_timed, args.steps):
+        j = (i - (args.steps - n_timed)) // copies
+        ev = timed[i % copies][j][1]
+        samples.append(ev[0].elapsed_time(ev[1]))
+    gemm_ms = statistics.mean(samples)
     elapsed_ms = aggregate_max(elapsed_ms, device)
     gemm_ms = aggregate_max(gemm_ms, device)
     # the two preparation phases run side by side inside the step; their own durations are

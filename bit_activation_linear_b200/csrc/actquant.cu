@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     const int64_t stride = (int64_t)gridDim.x * P::TEAMS;
     constexpr uint32_t ROW_BYTES = K * 2;
 
+    // the product that reads these codes may start its own set-up now (it waits for this grid
+    // to complete before it reads anything)
+    pdl_launch_dependents();
     // Persistent: the team walks rows base + team, base += stride.  The trip count is the same
     // for every team of the CTA (teams of <= 32 threads share a warp and its __syncwarp).  Rows
     // arrive by bulk asynchronous copies into a two-row ring, so the next row is in flight while
@@ -348,6 +351,7 @@ __global__ void __launch_bounds__(256)
                            int32_t *__restrict__ rowsum) {
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    pdl_launch_dependents();  // as in fwht_quant_kernel
     if (row >= M) return;  // whole warp leaves together
     const uint4 *xr = X + row * (K / 8);
     const int64_t nchunk = K / 8;

@@ -125,7 +125,7 @@ int act_quant_impl(DeviceState *st, const void *X, int64_t M, int64_t K, int had
 
 int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int32_t *rowsum,
               int64_t M, int64_t K, const void *Wp, const float *gamma, int64_t N, int act_bits,
-              int32_t *acc, void *Y, cudaStream_t stream) {
+              int32_t *acc, void *Y, cudaStream_t stream, bool early_weights = false) {
     GemmArgs a;
     a.codes = codes;
     a.scales = scales;
@@ -139,6 +139,7 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
     a.acc = acc;
     a.Y = Y;
     a.status = st->status_word;
+    a.early_weights = early_weights;
     if (M <= kGemvMaxTokens) return launched(launch_ternary_gemv(a, stream), 1, "ternary_gemv");
     const int n = (acc ? 1 : 0) + (Y ? 1 : 0);
     return launched(launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream), n,
@@ -168,7 +169,9 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
                                                   round256((size_t)M * sizeof(float)));
     if ((rc = act_quant_impl(st, X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr, stream)))
         return rc;
-    return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream);
+    // the quantiser above was launched in stream order after whatever wrote Wp
+    return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream,
+                     true);
 }
 
 }  // namespace

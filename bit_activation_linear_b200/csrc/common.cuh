@@ -153,6 +153,19 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // ------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the previous kernel of its stream is still running; pdl_wait() blocks until that
+// kernel has completed and its memory is visible (a no-op for an ordinary launch).  A kernel
+// calls pdl_launch_dependents() to let the next kernel start early; only kernels whose outputs
+// the next kernel reads after its pdl_wait() do so.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------
 // TMA (bulk tensor copies).  No multicast form is used anywhere in this library.
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y,

@@ -191,6 +191,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     cluster_sync();  // both CTAs' barriers are initialised and the tensor memory is allocated
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+    // everything above overlaps the tail of the kernel that produced the codes (programmatic
+    // dependent launch); nothing is read from global memory before this point
+    pdl_wait();
 
     if (warp == WARP_TMA) {
         // ------------------------------------------------------------------ code TMA
@@ -495,9 +498,18 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
     }
     const int pairs_max = max_pairs<BITS, OUT_I32>(num_sms);
     const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
-    kern<<<2 * pairs, NUM_THREADS, SMEM_BYTES, stream>>>(
-        mc, mw, my, out, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, (int)a.K, a.status);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, mc, mw, my, out, a.scales, a.rowsum, a.gamma, (int)a.M,
+                              (int)a.N, (int)a.K, a.status);
 }
 
 }  // namespace tc

@@ -27,10 +27,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                         const int32_t *__restrict__ rowsum, int M, int K,
                         const uint32_t *__restrict__ wp, const float *__restrict__ gamma_ptr,
-                        int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y) {
+                        int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y,
+                        int early_weights) {
+    if (!early_weights) pdl_wait();
     const int lane = threadIdx.x & 31;
     const int n0 = (blockIdx.x * kGemvWarps + (threadIdx.x >> 5)) * R;
-    if (n0 >= N) return;  // whole warp leaves together
+    if (n0 >= N) return;  // whole warp leaves together (nothing of its own to wait for)
     const int words = K / 16;  // packed words per row
     const int steps = (words + 31) / 32;  // the last step may be partial (K % 512 != 0)
     int acc[R][T];
@@ -48,6 +50,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
                 w[r][j] = (32 * (s0 + j) + lane < words && n0 + r < N)
                               ? __ldg(wp + (int64_t)(n0 + r) * words + 32 * (s0 + j) + lane)
                               : 0u;
+        // With early_weights the packed weights were complete before the kernel that wrote the
+        // codes started, so they are loaded before waiting for that kernel (programmatic
+        // dependent launch); the codes, scales and code sums are always read after the wait.
+        if (early_weights && s0 == 0) pdl_wait();
 #pragma unroll
         for (int j = 0; j < kGemvSteps; ++j) {
             if (s0 + j >= steps) break;
@@ -108,10 +114,19 @@ static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
     static_assert(R * T <= 32, "one lane per (row, token) result");
     const int64_t warps = (a.N + R - 1) / R;
     const unsigned blocks = (unsigned)((warps + kGemvWarps - 1) / kGemvWarps);
-    ternary_gemv_kernel<BITS, T, R><<<blocks, kGemvWarps * 32, 0, stream>>>(
-        reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum, (int)a.M, (int)a.K,
-        a.Wp, a.gamma, (int)a.N, a.acc, reinterpret_cast<__nv_bfloat16 *>(a.Y));
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<BITS, T, R>,
+                              reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum,
+                              (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
+                              reinterpret_cast<__nv_bfloat16 *>(a.Y), a.early_weights ? 1 : 0);
 }
 
 template <int BITS>

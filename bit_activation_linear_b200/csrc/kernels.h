@@ -39,6 +39,10 @@ struct GemmArgs {
     int32_t *acc;           // optional int32 [M][N]
     void *Y;                // optional bf16 [M][N]
     int *status;            // device status word
+    // The packed weights were complete before the kernel that precedes this launch in the
+    // stream started (true when the library's own quantiser runs in between, as in the forward
+    // entries): the decode kernel may then load them before waiting for that kernel.
+    bool early_weights = false;
 };
 
 // Weight-streaming kernel for few tokens (decode).

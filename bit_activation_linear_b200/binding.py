@@ -67,6 +67,7 @@ _SIGS = {
                                                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_size_t, ctypes.c_void_p]),
     "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "bitnet_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -266,6 +267,13 @@ def bitnet_bitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=N
 def bitnet_hbitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=None):
     """Y = H-BitLinear(X): online Hadamard transform, then BitLinear."""
     return _forward("bitnet_hbitlinear_forward", X, Wp, gamma, act_bits, Y, ws, stream)
+
+
+def bitnet_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Enqueue the failure-detection self-test: one bounded wait that runs out after
+    limit_cycles SM cycles and records a time-out for the next bitnet_sync_status()."""
+    st = load_library().bitnet_selftest_wait_timeout(int(limit_cycles), _stream(stream))
+    _rc(st, "bitnet_selftest_wait_timeout")
 
 
 def bitnet_sync_status(stream=None) -> int:

@@ -333,6 +333,18 @@ int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const voi
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+int bitnet_selftest_wait_timeout(int64_t limit_cycles, bitnet_stream_t stream) {
+    if (limit_cycles < 1 || limit_cycles > kWaitLimitCycles)
+        return fail(BITNET_ERR_INVALID, "limit_cycles = %lld must be in 1 .. %lld",
+                    (long long)limit_cycles, (long long)kWaitLimitCycles);
+    DeviceState *st = nullptr;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    return launched(launch_selftest_wait_timeout((long long)limit_cycles, st->status_word,
+                                                 reinterpret_cast<cudaStream_t>(stream)),
+                    1, "selftest_wait_timeout");
+}
+
 int bitnet_sync_status(bitnet_stream_t stream) {
     DeviceState *st = nullptr;
     int rc = device_state(&st);

@@ -109,16 +109,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete.  Returns false (and records a
 // time-out) if it does not complete within kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, int *status,
+                                                long long limit_cycles) {
     if (mbar_test_wait(bar, parity)) return true;
     long long start = clock64();
     while (!mbar_try_wait_sleep(bar, parity)) {
-        if (clock64() - start > kWaitLimitCycles) {
+        if (clock64() - start > limit_cycles) {
             record_status(status, BITNET_ERR_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
+    return mbar_wait_limit(bar, parity, status, kWaitLimitCycles);
 }
 
 // ------------------------------------------------------------------------------------------

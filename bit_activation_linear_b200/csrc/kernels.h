@@ -53,4 +53,8 @@ cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream);
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream);
 
+// ---- failure detection self-test (selftest.cu) ----
+cudaError_t launch_selftest_wait_timeout(long long limit_cycles, int *status,
+                                         cudaStream_t stream);
+
 }  // namespace bitnet

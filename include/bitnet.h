@@ -183,6 +183,17 @@ int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const voi
  * wait since the last call (the flag is cleared), else BITNET_OK. */
 int bitnet_sync_status(bitnet_stream_t stream);
 
+/*
+ * Self-test of the failure detection (a library facility; the pages have no counterpart).
+ * Every wait inside the library's kernels is bounded: a phase that does not complete within
+ * ~1 s makes the kernel record BITNET_ERR_TIMEOUT, wind down and return, and the next
+ * bitnet_sync_status() reports it.  This call enqueues one small kernel that runs that same
+ * bounded wait on a barrier nothing ever arrives on, giving up after limit_cycles SM clock cycles
+ * (1 .. 2e9, else BITNET_ERR_INVALID).  It neither faults nor hangs the GPU; afterwards
+ * bitnet_sync_status(stream) returns BITNET_ERR_TIMEOUT once and the context stays usable.
+ */
+int bitnet_selftest_wait_timeout(int64_t limit_cycles, bitnet_stream_t stream);
+
 /* Number of kernel launches this library has issued in this process (all devices). */
 uint64_t bitnet_launch_count(void);
 

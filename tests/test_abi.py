@@ -108,3 +108,8 @@ def test_binding_raises_without_library(tmp_path):
             "except RuntimeError as e:\n    print('raised', 'no fallback' in str(e).lower())\n")
     out = subprocess.run(["python", "-c", code], capture_output=True, text=True, cwd=ROOT)
     assert "raised True" in out.stdout, out.stdout + out.stderr
+
+
+def test_selftest_rejects_bad_limits_before_touching_the_device(lib):
+    for limit in (0, -5, 3_000_000_000):
+        assert lib.bitnet_selftest_wait_timeout(ctypes.c_int64(limit), None) == -1  # INVALID

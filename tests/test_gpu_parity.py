@@ -227,3 +227,19 @@ def test_errors_are_reported(B):
     Y = B.bitnet_bitlinear_forward(X, Wp, gamma, 8)  # fine without the transform
     B.bitnet_sync_status()
     assert not Y.float().abs().sum().item()
+
+
+# ----------------------------------------------------------------------------------------
+# failure detection: a bounded device wait that runs out is reported, and nothing is lost
+# ----------------------------------------------------------------------------------------
+
+def test_bounded_wait_time_out_is_reported_and_context_survives(B):
+    B.bitnet_sync_status()                       # nothing pending
+    B.bitnet_selftest_wait_timeout(2_000_000)    # ~1 ms of waiting on a barrier nobody arrives on
+    with pytest.raises(B.BitnetError) as err:
+        B.bitnet_sync_status()
+    assert err.value.status == B.ERR_TIMEOUT
+    assert B.bitnet_sync_status() == B.OK        # the flag was cleared
+    # the context is still usable: a small forward matches the oracle
+    wl = synth.WORKLOADS["tiny"]
+    forward_case(B, wl, None)

@@ -63,6 +63,9 @@ def lib():
                 "oracle_pack_base3": (None, [vp, i64, vp]),
                 "oracle_unpack_base3": (None, [vp, i64, vp]),
                 "oracle_fwht": (None, [vp, i64, i64, vp]),
+                "oracle_rmsnorm": (None, [vp, i64, i64, vp, f64, vp]),
+                "oracle_bitlinear_forward_norm": (i32, [vp, i64, i64, vp, i64, i32, i32, i32,
+                                                        vp, f64, vp, vp, vp, vp, vp, vp, vp]),
                 "oracle_quant_act": (None, [vp, i64, i64, i32, vp, vp, vp, vp]),
                 "oracle_pack_int4": (None, [vp, i64, i64, vp]),
                 "oracle_unpack_int4": (None, [vp, i64, i64, vp]),
@@ -159,6 +162,20 @@ def unpack_base3(b: np.ndarray, n: int) -> np.ndarray:
 # Step 2: online Hadamard transform  (BitNet v2 write-up, H-BitLinear paragraphs)
 # --------------------------------------------------------------------------------------
 
+def rmsnorm(x: np.ndarray, gain_bf16: np.ndarray | None = None, eps: float = 1e-5) -> np.ndarray:
+    """y = x * g / sqrt(mean(x^2) + eps) per row, in double (BitNet b1.58 2B4T article, 一.3:
+    subln normalisation; BitNet v2 write-up: RMS normalisation).  x: [M, K] float64; gain: bf16
+    bits [K] or None (unit gain)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if x.ndim == 1:
+        return rmsnorm(x[None, :], gain_bf16, eps)[0]
+    M, K = x.shape
+    y = np.empty_like(x)
+    g = None if gain_bf16 is None else np.ascontiguousarray(gain_bf16, dtype=np.uint16)
+    lib().oracle_rmsnorm(_p(x), M, K, None if g is None else _p(g), float(eps), _p(y))
+    return y
+
+
 def fwht(x: np.ndarray) -> np.ndarray:
     """z = H_K x / sqrt(K) per row, Sylvester order, in double.  x: [M, K] float64."""
     x = np.ascontiguousarray(x, dtype=np.float64)
@@ -251,8 +268,10 @@ def dequant(acc: np.ndarray, d: np.ndarray, gamma) -> np.ndarray:
 # The whole forward
 # --------------------------------------------------------------------------------------
 
-def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bits: int):
-    """Y = (H-)BitLinear(X) from bf16 X [M, K] and latent bf16 W [N, K].
+def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bits: int,
+                      norm_gain: np.ndarray | None = None, norm_eps: float | None = None):
+    """Y = (H-)BitLinear(X) from bf16 X [M, K] and latent bf16 W [N, K].  With norm_eps given,
+    every token row is RMS-normalised first (gain norm_gain, bf16 bits [K], or unit gain).
 
     Returns a dict with every stage: gamma, q, z, codes, d, acc, y (uint16 bf16 bits).
     """
@@ -267,9 +286,11 @@ def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bi
     codes = np.empty((M, K), dtype=np.int8)
     d = np.empty(M, dtype=np.float32)
     acc = np.empty((M, N), dtype=np.int64)
-    rc = lib().oracle_bitlinear_forward(_p(X), M, K, _p(W), N, int(bool(hadamard)), int(bits),
-                                        _p(Y), _p(gamma), _p(q), _p(z), _p(codes), _p(d),
-                                        _p(acc))
+    g = None if norm_gain is None else np.ascontiguousarray(norm_gain, dtype=np.uint16)
+    rc = lib().oracle_bitlinear_forward_norm(
+        _p(X), M, K, _p(W), N, int(bool(hadamard)), int(bits), int(norm_eps is not None),
+        None if g is None else _p(g), float(norm_eps or 0.0),
+        _p(Y), _p(gamma), _p(q), _p(z), _p(codes), _p(d), _p(acc))
     if rc != 0:
         raise MemoryError("oracle_bitlinear_forward could not allocate its buffers")
     return {"gamma": np.float32(gamma[0]), "q": q, "z": z, "codes": codes, "d": d,

@@ -197,6 +197,28 @@ void oracle_unpack_base3(const uint8_t *bytes, int64_t n, uint8_t *digits) {
 }
 
 /* ------------------------------------------------------------------------------------- */
+/* Before step 2: RMS normalisation of each token row  [2B4T 一.3: subln normalisation in  */
+/* place of LayerNorm], [v2: LLaMA-like components with RMS normalisation]                 */
+/* ------------------------------------------------------------------------------------- */
+
+/* y = x * g / sqrt(mean_k(x_k^2) + eps) per row, in double; g is a bf16 gain per feature
+ * (NULL: 1).  The pages name the normalisation only; this is the plainest reading of "RMS
+ * normalisation", applied to the token row right before its quantisation (and before the
+ * Hadamard transform in H-BitLinear). */
+void oracle_rmsnorm(const double *x, int64_t M, int64_t K, const uint16_t *g, double eps,
+                    double *y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const double *row = x + m * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) ss += row[k] * row[k];
+        const double r = 1.0 / sqrt(ss / (double)K + eps);
+        for (int64_t k = 0; k < K; ++k)
+            y[m * K + k] = row[k] * r * (g ? bf16_to_double(g[k]) : 1.0);
+    }
+}
+
+/* ------------------------------------------------------------------------------------- */
 /* Step 2: online Hadamard transform per token  [v2, H-BitLinear], [v2-abs]                */
 /* ------------------------------------------------------------------------------------- */
 
@@ -344,10 +366,27 @@ void oracle_dequant(const int64_t *acc, const float *d, float gamma, int64_t M, 
  * latent bf16 W [N][K].  Optional outputs expose each stage: gamma, ternary q [N][K], the
  * transformed activations z [M][K] (double, before quantisation), codes [M][K], d [M],
  * acc [M][N].  Returns 0, or -1 when a buffer cannot be allocated. */
+int oracle_bitlinear_forward_norm(const uint16_t *X, int64_t M, int64_t K, const uint16_t *W,
+                                  int64_t N, int hadamard, int bits, int norm,
+                                  const uint16_t *norm_gain, double norm_eps, uint16_t *Y,
+                                  float *gamma_out, int8_t *q_out, double *z_out,
+                                  int8_t *codes_out, float *d_out, int64_t *acc_out);
+
 int oracle_bitlinear_forward(const uint16_t *X, int64_t M, int64_t K, const uint16_t *W,
                              int64_t N, int hadamard, int bits, uint16_t *Y,
                              float *gamma_out, int8_t *q_out, double *z_out,
                              int8_t *codes_out, float *d_out, int64_t *acc_out) {
+    return oracle_bitlinear_forward_norm(X, M, K, W, N, hadamard, bits, 0, NULL, 0.0, Y,
+                                         gamma_out, q_out, z_out, codes_out, d_out, acc_out);
+}
+
+/* As oracle_bitlinear_forward; with norm != 0 each token row is RMS-normalised first
+ * (oracle_rmsnorm with norm_gain and norm_eps) and the double result feeds the transform. */
+int oracle_bitlinear_forward_norm(const uint16_t *X, int64_t M, int64_t K, const uint16_t *W,
+                                  int64_t N, int hadamard, int bits, int norm,
+                                  const uint16_t *norm_gain, double norm_eps, uint16_t *Y,
+                                  float *gamma_out, int8_t *q_out, double *z_out,
+                                  int8_t *codes_out, float *d_out, int64_t *acc_out) {
     int rc = -1;
     int8_t *q = malloc((size_t)(N * K));
     double *x = malloc((size_t)(M * K) * sizeof(double));
@@ -362,6 +401,10 @@ int oracle_bitlinear_forward(const uint16_t *X, int64_t M, int64_t K, const uint
     oracle_ternarize(W, N * K, gamma, q);
 
     for (int64_t i = 0; i < M * K; ++i) x[i] = bf16_to_double(X[i]);
+    if (norm) {
+        oracle_rmsnorm(x, M, K, norm_gain, norm_eps, z);
+        memcpy(x, z, (size_t)(M * K) * sizeof(double));
+    }
     if (hadamard) oracle_fwht(x, M, K, z);
     else memcpy(z, x, (size_t)(M * K) * sizeof(double));
     for (int64_t i = 0; i < M * K; ++i) zf[i] = (float)z[i];

@@ -376,3 +376,58 @@ def test_forward_stages_compose():
     np.testing.assert_array_equal(out["codes"], c)
     np.testing.assert_array_equal(out["acc"], acc)
     np.testing.assert_array_equal(out["y"], oracle.dequant(acc, d, g))
+
+
+# ----------------------------------------------------------------------------------------
+# RMS normalisation before the quantiser (BitNet b1.58 2B4T article, 一.3: subln
+# normalisation; BitNet v2 write-up: RMS normalisation)
+# ----------------------------------------------------------------------------------------
+
+def test_rmsnorm_matches_library_rms_norm():
+    rng = np.random.default_rng(3)
+    K = 256
+    x = rng.normal(size=(5, K)) * 3.0
+    g = bf16_bits(rng.uniform(0.5, 1.5, K))
+    for eps in (0.0, 1e-5, 0.1):
+        y = oracle.rmsnorm(x, g, eps)
+        ref = torch.nn.functional.rms_norm(
+            torch.from_numpy(x), (K,), weight=torch.from_numpy(oracle.bf16_to_f64(g)),
+            eps=eps).numpy()
+        np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-15)
+    # no gain = unit gain
+    np.testing.assert_allclose(oracle.rmsnorm(x, None, 1e-5),
+                               oracle.rmsnorm(x, bf16_bits(np.ones(K)), 1e-5), rtol=0, atol=0)
+
+
+def test_rmsnorm_invariants_and_closed_forms():
+    rng = np.random.default_rng(4)
+    x = rng.laplace(size=(4, 128))
+    y = oracle.rmsnorm(x, None, 0.0)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), 1.0, rtol=1e-14)   # unit RMS
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * x, None, 0.0), y, rtol=1e-14)  # scale
+    np.testing.assert_allclose(oracle.rmsnorm(-x, None, 0.0), -y, rtol=0, atol=0)  # odd
+    assert np.all(oracle.rmsnorm(np.zeros((2, 128)), None, 1e-5) == 0.0)            # zero row
+    c, eps = 0.25, 1e-3
+    g = bf16_bits(np.linspace(-2, 2, 128))
+    row = oracle.rmsnorm(np.full((1, 128), c), g, eps)[0]
+    np.testing.assert_allclose(row, c / math.sqrt(c * c + eps) * oracle.bf16_to_f64(g),
+                               rtol=1e-15)
+
+
+@pytest.mark.parametrize("hadamard", [True, False])
+def test_forward_with_norm_composes_from_the_stages(hadamard):
+    rng = np.random.default_rng(5)
+    M, K, N = 6, 256, 64
+    X = synth.sharp_activations(M, K, seed=11)
+    W = synth.latent_weights(N, K, seed=12)
+    g = bf16_bits(rng.uniform(0.5, 1.5, K))
+    ref = oracle.bitlinear_forward(X, W, hadamard, 8, norm_gain=g, norm_eps=1e-5)
+    y = oracle.rmsnorm(oracle.bf16_to_f64(X), g, 1e-5)
+    z = oracle.fwht(y) if hadamard else y
+    np.testing.assert_array_equal(ref["z"], z)
+    codes, d, _, _ = oracle.quant_act(z.astype(np.float32), 8)
+    np.testing.assert_array_equal(ref["codes"], codes)
+    # without norm_eps the forward is the plain one
+    plain = oracle.bitlinear_forward(X, W, hadamard, 8)
+    np.testing.assert_array_equal(
+        plain["z"], oracle.fwht(oracle.bf16_to_f64(X)) if hadamard else oracle.bf16_to_f64(X))

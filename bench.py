@@ -295,7 +295,18 @@ def run_gpu(args, wl, rank, world, device):
     def weights(b):
         B.bitnet_quantize_pack_weights(b["W"], b["Wp"], b["gamma"], b["wws"])
 
+    # with --rmsnorm the token rows are RMS-normalised inside the quantiser (gain of ones
+    # perturbed per feature, eps 1e-5)
+    gain = None
+    if args.rmsnorm:
+        g = np.random.default_rng(7).uniform(0.5, 1.5, K).astype(np.float32)
+        gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
+
     def quant(b):
+        if gain is not None:
+            B.bitnet_act_quant_norm(b["X"], gain, 1e-5, wl.hadamard, wl.act_bits, b["codes"],
+                                    b["scales"], b["rowsum"])
+            return
         B.bitnet_act_quant(b["X"], wl.hadamard, wl.act_bits, b["codes"], b["scales"],
                            b["rowsum"])
 
@@ -433,7 +444,8 @@ def run_gpu(args, wl, rank, world, device):
                 "us": 1e3 * phase_ms[0], "bound": "hbm", "bytes": w_bytes,
                 "achieved_gbs": w_bytes / (phase_ms[0] * 1e-3) / 1e9,
                 "frac": w_bytes / (phase_ms[0] * 1e-3) / 1e9 / hbm},
-            ("fwht_quant" if wl.hadamard else "act_quant_plain") + " (alone, outside the timed steps)": {
+            ("fwht_quant" if wl.hadamard else "act_quant_plain")
+            + ("+rmsnorm" if args.rmsnorm else "") + " (alone, outside the timed steps)": {
                 "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,
                 "achieved_gbs": q_bytes / (phase_ms[1] * 1e-3) / 1e9,
                 "frac": q_bytes / (phase_ms[1] * 1e-3) / 1e9 / hbm},
@@ -458,7 +470,8 @@ def run_gpu(args, wl, rank, world, device):
             "data": "synthetic",
             "effective_tops": world * wl.ops / (ms_per_step * 1e-3) / 1e12,
             "config": {"workload": wl.name, "M": M, "K": K, "N": N, "hadamard": wl.hadamard,
-                       "act_bits": wl.act_bits, "tokens_per_rank": M,
+                       "act_bits": wl.act_bits, "rmsnorm": bool(args.rmsnorm),
+                       "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {copies} copies "
                              f"({copies * per_copy / 2**20:.0f} MiB > 2 x L2)"},
@@ -496,6 +509,13 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
     ws = torch.empty(max(B.bitnet_workspace_bytes(M, K, N, wl.act_bits), 256), dtype=torch.uint8,
                      device=device)
     fwd = B.bitnet_hbitlinear_forward if wl.hadamard else B.bitnet_bitlinear_forward
+    if args.rmsnorm:  # the same gain as the timed steps
+        g = np.random.default_rng(7).uniform(0.5, 1.5, K).astype(np.float32)
+        gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
+
+        def fwd(X, Wp, gamma, act_bits, Y, ws):
+            return B.bitnet_norm_bitlinear_forward(X, gain, 1e-5, wl.hadamard, Wp, gamma,
+                                                   act_bits, Y=Y, ws=ws)
 
     def step():
         Xd.copy_(Xh, non_blocking=True)
@@ -530,6 +550,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--workload", default="wo_2048", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rmsnorm", action="store_true",
+                    help="RMS-normalise the token rows inside the quantiser (fused prologue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()

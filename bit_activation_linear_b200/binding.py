@@ -66,6 +66,19 @@ _SIGS = {
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_act_quant_norm": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_norm_transform_f32": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                 ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
+                                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_norm_bitlinear_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                     ctypes.c_int64, ctypes.c_void_p,
+                                                     ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                                     ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                     ctypes.c_void_p, ctypes.c_void_p,
+                                                     ctypes.c_size_t, ctypes.c_void_p]),
     "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bitnet_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
 }
@@ -267,6 +280,77 @@ def bitnet_bitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=N
 def bitnet_hbitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=None):
     """Y = H-BitLinear(X): online Hadamard transform, then BitLinear."""
     return _forward("bitnet_hbitlinear_forward", X, Wp, gamma, act_bits, Y, ws, stream)
+
+
+def _gain_ptr(gain, K):
+    if gain is None:
+        return None
+    _check(gain, "norm_gain", torch.bfloat16, 1)
+    if gain.numel() != K:
+        raise ValueError(f"norm_gain has {gain.numel()} entries, K = {K}")
+    return gain.data_ptr()
+
+
+def bitnet_act_quant_norm(X: torch.Tensor, norm_gain, eps: float, hadamard: bool, act_bits: int,
+                          codes=None, scales=None, rowsum=None, stream=None):
+    """RMS normalisation (gain norm_gain bf16 [K] or None, eps) fused with per-token
+    (Hadamard +) absmax quantisation.  Returns (codes, scales, rowsum)."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if codes is None:
+        codes = torch.empty((M, K if act_bits == 8 else K // 2),
+                            dtype=torch.int8 if act_bits == 8 else torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=X.device)
+    if rowsum is None:
+        rowsum = torch.empty(M, dtype=torch.int32, device=X.device)
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, act_bits)), "codes")
+    _nbytes_at_least(scales, 4 * M, "scales")
+    _nbytes_at_least(rowsum, 4 * M, "rowsum")
+    _rc(L.bitnet_act_quant_norm(X.data_ptr(), M, K, _gain_ptr(norm_gain, K), float(eps),
+                                int(bool(hadamard)), int(act_bits), codes.data_ptr(),
+                                scales.data_ptr(), rowsum.data_ptr(), _stream(stream)),
+        "bitnet_act_quant_norm")
+    return codes, scales, rowsum
+
+
+def bitnet_norm_transform_f32(X: torch.Tensor, norm_gain, eps: float, hadamard: bool,
+                              Z: torch.Tensor | None = None, stream=None):
+    """The normalised rows (and their Hadamard transform) in fp32 (debug / parity entry)."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if Z is None:
+        Z = torch.empty((M, K), dtype=torch.float32, device=X.device)
+    _rc(L.bitnet_norm_transform_f32(X.data_ptr(), M, K, _gain_ptr(norm_gain, K), float(eps),
+                                    int(bool(hadamard)), Z.data_ptr(), _stream(stream)),
+        "bitnet_norm_transform_f32")
+    return Z
+
+
+def bitnet_norm_bitlinear_forward(X, norm_gain, eps, hadamard, Wp, gamma, act_bits=8, Y=None,
+                                  ws=None, stream=None):
+    """Y = (H-)BitLinear(RMSNorm(X)) with the normalisation fused into the quantiser."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    _check(Wp, "Wp")
+    _check(gamma, "gamma", torch.float32)
+    M, K = X.shape
+    N = Wp.shape[0]
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _nbytes_at_least(Y, 2 * M * N, "Y")
+    need = int(L.bitnet_workspace_bytes(M, K, N, act_bits))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _rc(L.bitnet_norm_bitlinear_forward(X.data_ptr(), M, K, _gain_ptr(norm_gain, K), float(eps),
+                                        int(bool(hadamard)), Wp.data_ptr(), gamma.data_ptr(), N,
+                                        int(act_bits), Y.data_ptr(), ws.data_ptr(),
+                                        ws.numel() * ws.element_size(), _stream(stream)),
+        "bitnet_norm_bitlinear_forward")
+    return Y
 
 
 def bitnet_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

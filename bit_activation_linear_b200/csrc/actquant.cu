@@ -96,9 +96,10 @@ __device__ __forceinline__ void team_sync(int team) {
     }
 }
 
-template <class P, int BITS, bool ZOUT>
+template <class P, int BITS, bool ZOUT, bool NORM>
 __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     fwht_quant_kernel(const uint8_t *__restrict__ X, int M, float rsqrt_k,
+                      const uint32_t *__restrict__ gain2, float eps,
                       uint8_t *__restrict__ codes, float *__restrict__ scales,
                       int32_t *__restrict__ rowsum, float *__restrict__ zout, int *status) {
     constexpr int K = P::K, TEAM = P::TEAM, V = P::V, L = P::L;
@@ -164,6 +165,34 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     for (int c = 0; c < V / 2; ++c) {
         const uint32_t w = (valid && ok) ? xr[c * TEAM + r] : 0u;
         a[c] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+    if constexpr (NORM) {
+        // RMS normalisation of the row before the transform: y = (x * rinv) * g with
+        // rinv = 1 / sqrt(sum(x^2) / K + eps), every operation an IEEE fp32 one
+        float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < V / 2; ++c) ss2 = __ffma2_rn(a[c], a[c], ss2);
+        float ss = ss2.x + ss2.y;
+        constexpr int W = TEAM < 32 ? TEAM : 32;
+#pragma unroll
+        for (int o = W / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        if constexpr (TEAM > 32) {
+            // the previous row's reads of these slots ended before its later barriers
+            constexpr int WPT = P::WARPS_PER_TEAM;
+            if (lane == 0) red[team * WPT + (r >> 5)] = ss;
+            team_sync<TEAM>(team);
+            ss = red[team * WPT];
+#pragma unroll
+            for (int i = 1; i < WPT; ++i) ss += red[team * WPT + i];
+        }
+        const float rinv = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+        const float2 r2 = make_float2(rinv, rinv);
+#pragma unroll
+        for (int c = 0; c < V / 2; ++c) {
+            const uint32_t gw = gain2 ? __ldg(gain2 + c * TEAM + r) : 0x3F803F80u;  // 1.0, 1.0
+            a[c] = mul2_rn(mul2_rn(a[c], r2),
+                           make_float2(__uint_as_float(gw << 16), __uint_as_float(gw & 0xFFFF0000u)));
+        }
     }
 #pragma unroll
     for (int c = 0; c < V / 2; ++c) {  // index bit 0 (inside the pair)
@@ -344,26 +373,71 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
 
 // ---- plain BitLinear: absmax quantisation without a transform (any K % 128 == 0) ----
 // One warp per token row, two passes over the row (the second one hits L1/L2).
-template <int BITS>
+// With NORM each value is first RMS-normalised, y = (x * rinv) * g as in fwht_quant_kernel (an
+// extra pass over the row for sum(x^2)); with ZOUT the kernel writes y in fp32 instead of codes.
+template <int BITS, bool NORM, bool ZOUT>
 __global__ void __launch_bounds__(256)
     act_quant_plain_kernel(const uint4 *__restrict__ X, int64_t M, int64_t K,
+                           const uint4 *__restrict__ gain8, float eps,
                            uint8_t *__restrict__ codes, float *__restrict__ scales,
-                           int32_t *__restrict__ rowsum) {
+                           int32_t *__restrict__ rowsum, float *__restrict__ zout) {
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     pdl_launch_dependents();  // as in fwht_quant_kernel
     if (row >= M) return;  // whole warp leaves together
     const uint4 *xr = X + row * (K / 8);
     const int64_t nchunk = K / 8;
-    float mx = 0.f;
-    for (int64_t c = lane; c < nchunk; c += 32) {
-        uint4 v = __ldg(xr + c);
+    float rinv = 1.f;
+    if constexpr (NORM) {
+        float ss = 0.f;
+        for (int64_t c = lane; c < nchunk; c += 32) {
+            const uint4 v = __ldg(xr + c);
+            const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float x0 = __uint_as_float(h[i] << 16), x1 = __uint_as_float(h[i] & 0xFFFF0000u);
+                ss = __fmaf_rn(x0, x0, ss);
+                ss = __fmaf_rn(x1, x1, ss);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+        rinv = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)K), eps)));
+    }
+    // the eight values of chunk c as four float pairs (normalised with NORM)
+    auto load8 = [&](int64_t c, float2 (&y)[4]) {
+        const uint4 v = __ldg(xr + c);
         const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+        uint32_t gh[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};  // unit gain
+        if (NORM && gain8) {
+            const uint4 gv = __ldg(gain8 + c);
+            gh[0] = gv.x; gh[1] = gv.y; gh[2] = gv.z; gh[3] = gv.w;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            mx = fmaxf(mx, __uint_as_float((h[i] & 0x7FFFu) << 16));
-            mx = fmaxf(mx, __uint_as_float(h[i] & 0x7FFF0000u));
+            y[i] = make_float2(__uint_as_float(h[i] << 16), __uint_as_float(h[i] & 0xFFFF0000u));
+            if constexpr (NORM)
+                y[i] = mul2_rn(mul2_rn(y[i], make_float2(rinv, rinv)),
+                               make_float2(__uint_as_float(gh[i] << 16),
+                                           __uint_as_float(gh[i] & 0xFFFF0000u)));
         }
+    };
+    if constexpr (ZOUT) {
+        for (int64_t c = lane; c < nchunk; c += 32) {
+            float2 y[4];
+            load8(c, y);
+            float4 *zr = reinterpret_cast<float4 *>(zout + row * K + 8 * c);
+            zr[0] = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
+            zr[1] = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
+        }
+        return;
+    }
+    float mx = 0.f;
+    for (int64_t c = lane; c < nchunk; c += 32) {
+        float2 y[4];
+        load8(c, y);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(y[i].x), fabsf(y[i].y)));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
@@ -374,13 +448,13 @@ __global__ void __launch_bounds__(256)
     const float2 magic2 = make_float2(12582912.f, 12582912.f);
     int sum = 0;
     for (int64_t c = lane; c < nchunk; c += 32) {
-        uint4 v = __ldg(xr + c);
-        const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+        float2 y[4];
+        load8(c, y);
         uint32_t f[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            float2 x = make_float2(__uint_as_float(h[i] << 16), __uint_as_float(h[i] & 0xFFFF0000u));
-            float2 u = __fadd2_rn(make_float2(__fmul_rn(x.x, s), __fmul_rn(x.y, s)), magic2);
+            // __fmul_rn is never contracted with the following add (see fwht_quant_kernel)
+            float2 u = __fadd2_rn(make_float2(__fmul_rn(y[i].x, s), __fmul_rn(y[i].y, s)), magic2);
             f[2 * i] = __float_as_uint(u.x);
             f[2 * i + 1] = __float_as_uint(u.y);
         }
@@ -403,10 +477,11 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <class P, int BITS, bool ZOUT>
-static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *scales,
-                                 int32_t *rowsum, float *zout, int *status, cudaStream_t stream) {
-    auto kern = fwht_quant_kernel<P, BITS, ZOUT>;
+template <class P, int BITS, bool ZOUT, bool NORM>
+static cudaError_t launch_fwht_t(const void *X, int64_t M, const NormArgs &nrm, void *codes,
+                                 float *scales, int32_t *rowsum, float *zout, int *status,
+                                 cudaStream_t stream) {
+    auto kern = fwht_quant_kernel<P, BITS, ZOUT, NORM>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -428,52 +503,80 @@ static cudaError_t launch_fwht_t(const void *X, int64_t M, void *codes, float *s
     const int64_t blocks = want < cap ? want : cap;
     const float rk = (float)(1.0 / sqrt((double)P::K));
     kern<<<(unsigned)blocks, P::THREADS, P::SMEM, stream>>>(
-        reinterpret_cast<const uint8_t *>(X), (int)M, rk, reinterpret_cast<uint8_t *>(codes),
-        scales, rowsum, zout, status);
+        reinterpret_cast<const uint8_t *>(X), (int)M, rk,
+        reinterpret_cast<const uint32_t *>(nrm.gain), nrm.eps,
+        reinterpret_cast<uint8_t *>(codes), scales, rowsum, zout, status);
     return cudaGetLastError();
+}
+
+template <int LOGK, bool NORM>
+static cudaError_t launch_fwht_n(const void *X, int64_t M, int act_bits, const NormArgs &nrm,
+                                 void *codes, float *scales, int32_t *rowsum, float *zout,
+                                 int *status, cudaStream_t stream) {
+    using P = typename FwhtConfig<LOGK>::P;
+    if (zout)
+        return launch_fwht_t<P, 8, true, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
+                                               stream);
+    if (act_bits == 4)
+        return launch_fwht_t<P, 4, false, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
+                                                stream);
+    return launch_fwht_t<P, 8, false, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
+                                            stream);
 }
 
 template <int LOGK>
-static cudaError_t launch_fwht_k(const void *X, int64_t M, int act_bits, void *codes,
-                                 float *scales, int32_t *rowsum, float *zout, int *status,
-                                 cudaStream_t stream) {
-    using P = typename FwhtConfig<LOGK>::P;
-    if (zout) return launch_fwht_t<P, 8, true>(X, M, codes, scales, rowsum, zout, status, stream);
-    if (act_bits == 4)
-        return launch_fwht_t<P, 4, false>(X, M, codes, scales, rowsum, zout, status, stream);
-    return launch_fwht_t<P, 8, false>(X, M, codes, scales, rowsum, zout, status, stream);
+static cudaError_t launch_fwht_k(const void *X, int64_t M, int act_bits, const NormArgs &nrm,
+                                 void *codes, float *scales, int32_t *rowsum, float *zout,
+                                 int *status, cudaStream_t stream) {
+    return nrm.on ? launch_fwht_n<LOGK, true>(X, M, act_bits, nrm, codes, scales, rowsum, zout,
+                                              status, stream)
+                  : launch_fwht_n<LOGK, false>(X, M, act_bits, nrm, codes, scales, rowsum, zout,
+                                               status, stream);
 }
 
-cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
-                              float *scales, int32_t *rowsum, float *zout, int *status,
-                              cudaStream_t stream) {
+cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
+                              const NormArgs &nrm, void *codes, float *scales, int32_t *rowsum,
+                              float *zout, int *status, cudaStream_t stream) {
+#define BITNET_FWHT_CASE(L) \
+    case L: return launch_fwht_k<L>(X, M, act_bits, nrm, codes, scales, rowsum, zout, status, stream)
     switch (logk) {
-        case 7: return launch_fwht_k<7>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 8: return launch_fwht_k<8>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 9: return launch_fwht_k<9>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 10: return launch_fwht_k<10>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 11: return launch_fwht_k<11>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 12: return launch_fwht_k<12>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 13: return launch_fwht_k<13>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 14: return launch_fwht_k<14>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
-        case 15: return launch_fwht_k<15>(X, M, act_bits, codes, scales, rowsum, zout, status, stream);
+        BITNET_FWHT_CASE(7);
+        BITNET_FWHT_CASE(8);
+        BITNET_FWHT_CASE(9);
+        BITNET_FWHT_CASE(10);
+        BITNET_FWHT_CASE(11);
+        BITNET_FWHT_CASE(12);
+        BITNET_FWHT_CASE(13);
+        BITNET_FWHT_CASE(14);
+        BITNET_FWHT_CASE(15);
         default: return cudaErrorInvalidValue;
     }
+#undef BITNET_FWHT_CASE
+}
+
+template <int BITS, bool NORM, bool ZOUT>
+static cudaError_t launch_plain_t(const void *X, int64_t M, int64_t K, const NormArgs &nrm,
+                                  void *codes, float *scales, int32_t *rowsum, float *zout,
+                                  cudaStream_t stream) {
+    const int64_t blocks = (M + 7) / 8;
+    act_quant_plain_kernel<BITS, NORM, ZOUT><<<(unsigned)blocks, 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<const uint4 *>(nrm.gain),
+        nrm.eps, reinterpret_cast<uint8_t *>(codes), scales, rowsum, zout);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
-                                   void *codes, float *scales, int32_t *rowsum,
-                                   cudaStream_t stream) {
-    const int64_t blocks = (M + 7) / 8;
-    if (act_bits == 4)
-        act_quant_plain_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(
-            reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<uint8_t *>(codes),
-            scales, rowsum);
-    else
-        act_quant_plain_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(
-            reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<uint8_t *>(codes),
-            scales, rowsum);
-    return cudaGetLastError();
+                                   const NormArgs &nrm, void *codes, float *scales,
+                                   int32_t *rowsum, float *zout, cudaStream_t stream) {
+    if (zout)  // the normalised rows themselves (the parity entry); only with a norm
+        return launch_plain_t<8, true, true>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
+    if (nrm.on)
+        return act_bits == 4
+                   ? launch_plain_t<4, true, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream)
+                   : launch_plain_t<8, true, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
+    return act_bits == 4
+               ? launch_plain_t<4, false, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream)
+               : launch_plain_t<8, false, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
 }
 
 }  // namespace bitnet

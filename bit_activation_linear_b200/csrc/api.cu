@@ -108,19 +108,20 @@ int launched(cudaError_t e, int count, const char *what) {
 
 int act_quant_impl(DeviceState *st, const void *X, int64_t M, int64_t K, int hadamard,
                    int act_bits, void *codes, float *scales, int32_t *rowsum, float *zout,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, const NormArgs &nrm = NormArgs()) {
     if (hadamard) {
         const int lk = log2_exact(K);
         if (lk < 7 || lk > 15)
             return fail(BITNET_ERR_UNSUPPORTED,
                         "H-BitLinear needs K to be a power of two in [128, 32768], got %lld",
                         (long long)K);
-        return launched(launch_fwht_quant(X, M, lk, act_bits, codes, scales, rowsum, zout,
+        return launched(launch_fwht_quant(X, M, lk, act_bits, nrm, codes, scales, rowsum, zout,
                                           st->status_word, stream),
                         1, "fwht_quant");
     }
-    return launched(launch_act_quant_plain(X, M, K, act_bits, codes, scales, rowsum, stream), 1,
-                    "act_quant_plain");
+    return launched(launch_act_quant_plain(X, M, K, act_bits, nrm, codes, scales, rowsum, zout,
+                                           stream),
+                    1, "act_quant_plain");
 }
 
 int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int32_t *rowsum,
@@ -148,7 +149,7 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
 
 int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const float *gamma,
                  int64_t N, int act_bits, void *Y, void *ws, size_t ws_bytes, int hadamard,
-                 cudaStream_t stream) {
+                 cudaStream_t stream, const NormArgs &nrm = NormArgs()) {
     int rc = check_shape(M, K, N, true, true);
     if (rc) return rc;
     if (act_bits != 8 && act_bits != 4)
@@ -167,7 +168,8 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
     float *scales = reinterpret_cast<float *>(w + round256(bitnet_act_codes_bytes(M, K, act_bits)));
     int32_t *rowsum = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(scales) +
                                                   round256((size_t)M * sizeof(float)));
-    if ((rc = act_quant_impl(st, X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr, stream)))
+    if ((rc = act_quant_impl(st, X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr,
+                             stream, nrm)))
         return rc;
     // the quantiser above was launched in stream order after whatever wrote Wp
     return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream,
@@ -290,6 +292,69 @@ int bitnet_fwht_f32(const void *X_dev, int64_t M, int64_t K, float *Z_dev,
     if ((rc = device_state(&st))) return rc;
     return act_quant_impl(st, X_dev, M, K, 1, 8, nullptr, nullptr, nullptr, Z_dev,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+namespace {
+int norm_args(const void *gain_dev, float eps, NormArgs *out) {
+    if (!(eps > 0.f) || !std::isfinite(eps))
+        return fail(BITNET_ERR_INVALID, "eps = %g must be finite and > 0", (double)eps);
+    if (gain_dev && !aligned16(gain_dev))
+        return fail(BITNET_ERR_INVALID, "the norm gain must be 16-byte aligned");
+    out->on = true;
+    out->gain = gain_dev;
+    out->eps = eps;
+    return BITNET_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int bitnet_act_quant_norm(const void *X_dev, int64_t M, int64_t K, const void *norm_gain_dev,
+                          float eps, int hadamard, int act_bits, void *codes_dev,
+                          float *scales_dev, int32_t *rowsum_dev, bitnet_stream_t stream) {
+    int rc = check_shape(M, K, 8, true, false);
+    if (rc) return rc;
+    if (act_bits != 8 && act_bits != 4)
+        return fail(BITNET_ERR_INVALID, "act_bits = %d must be 8 or 4", act_bits);
+    if (!X_dev || !codes_dev || !scales_dev || !rowsum_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(X_dev) || !aligned16(codes_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    NormArgs nrm;
+    if ((rc = norm_args(norm_gain_dev, eps, &nrm))) return rc;
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    return act_quant_impl(st, X_dev, M, K, hadamard, act_bits, codes_dev, scales_dev, rowsum_dev,
+                          nullptr, reinterpret_cast<cudaStream_t>(stream), nrm);
+}
+
+int bitnet_norm_transform_f32(const void *X_dev, int64_t M, int64_t K, const void *norm_gain_dev,
+                              float eps, int hadamard, float *Z_dev, bitnet_stream_t stream) {
+    int rc = check_shape(M, K, 8, true, false);
+    if (rc) return rc;
+    if (!X_dev || !Z_dev) return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(X_dev) || !aligned16(Z_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    NormArgs nrm;
+    if ((rc = norm_args(norm_gain_dev, eps, &nrm))) return rc;
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    return act_quant_impl(st, X_dev, M, K, hadamard, 8, nullptr, nullptr, nullptr, Z_dev,
+                          reinterpret_cast<cudaStream_t>(stream), nrm);
+}
+
+int bitnet_norm_bitlinear_forward(const void *X_dev, int64_t M, int64_t K,
+                                  const void *norm_gain_dev, float eps, int hadamard,
+                                  const void *Wp_dev, const float *gamma_dev, int64_t N,
+                                  int act_bits, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                  bitnet_stream_t stream) {
+    NormArgs nrm;
+    int rc = norm_args(norm_gain_dev, eps, &nrm);
+    if (rc) return rc;
+    return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, act_bits, Y_dev, ws_dev, ws_bytes,
+                        hadamard ? 1 : 0, reinterpret_cast<cudaStream_t>(stream), nrm);
 }
 
 int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,

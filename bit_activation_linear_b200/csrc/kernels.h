@@ -18,14 +18,22 @@ cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partia
 cudaError_t noalloc_partials_address(double **ptr, size_t *bytes);
 
 // ---- steps 2-3: activations (actquant.cu) ----
+// Optional RMS normalisation of each row before the transform / quantisation:
+// y = (x * rinv) * g, rinv = 1 / sqrt(sum(x^2) / K + eps), g bf16 [K] (nullptr: unit gain).
+struct NormArgs {
+    bool on = false;
+    const void *gain = nullptr;
+    float eps = 0.f;
+};
 // Hadamard + quantise (or z output when zout != nullptr).  K = 2^logk, 7 <= logk <= 15.
-cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits, void *codes,
-                              float *scales, int32_t *rowsum, float *zout, int *status,
-                              cudaStream_t stream);
-// Quantise without a transform; K % 128 == 0.
+cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
+                              const NormArgs &nrm, void *codes, float *scales, int32_t *rowsum,
+                              float *zout, int *status, cudaStream_t stream);
+// Quantise without a transform; K % 128 == 0.  zout != nullptr (with nrm.on) writes the
+// normalised rows in fp32 instead of codes.
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
-                                   void *codes, float *scales, int32_t *rowsum,
-                                   cudaStream_t stream);
+                                   const NormArgs &nrm, void *codes, float *scales,
+                                   int32_t *rowsum, float *zout, cudaStream_t stream);
 
 // ---- step 4: product (gemv.cu, gemm_tc.cu) ----
 struct GemmArgs {

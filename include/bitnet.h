@@ -134,6 +134,25 @@ int bitnet_act_quant(const void *X_dev, int64_t M, int64_t K, int hadamard, int 
 int bitnet_fwht_f32(const void *X_dev, int64_t M, int64_t K, float *Z_dev,
                     bitnet_stream_t stream);
 
+/*
+ * RMS normalisation fused in front of steps 2 and 3.  The pages name this normalisation without a
+ * formula: BitNet b1.58 2B4T article, section 一.3 (subln normalisation in place of LayerNorm);
+ * BitNet v2 write-up (RMS normalisation among the model's LLaMA-like components).  Per token row:
+ *   y = (x * rinv) * g,  rinv = 1 / sqrt(sum_k x_k^2 / K + eps)   (each an IEEE fp32 operation),
+ * then exactly bitnet_act_quant on y (hadamard != 0: z = (1/sqrt(K)) H_K y).
+ * norm_gain_dev  bf16 [K] per-feature gain, 16-byte aligned, or NULL for unit gain.
+ * eps            finite and > 0, else BITNET_ERR_INVALID.
+ * Other arguments, layouts and errors as bitnet_act_quant.
+ */
+int bitnet_act_quant_norm(const void *X_dev, int64_t M, int64_t K, const void *norm_gain_dev,
+                          float eps, int hadamard, int act_bits, void *codes_dev,
+                          float *scales_dev, int32_t *rowsum_dev, bitnet_stream_t stream);
+
+/* Debug / parity entry: Z = y (hadamard == 0) or (1/sqrt(K)) H_K y (hadamard != 0), float
+ * [M, K], with y the normalised rows of bitnet_act_quant_norm (same kernels and arithmetic). */
+int bitnet_norm_transform_f32(const void *X_dev, int64_t M, int64_t K, const void *norm_gain_dev,
+                              float eps, int hadamard, float *Z_dev, bitnet_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------- */
 /* Step 4: ternary x integer product and rescale                                             */
 /* ---------------------------------------------------------------------------------------- */
@@ -173,6 +192,15 @@ int bitnet_bitlinear_forward(const void *X_dev, int64_t M, int64_t K, const void
 int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
                               const float *gamma_dev, int64_t N, int act_bits, void *Y_dev,
                               void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
+
+/* Y = BitLinear(RMSNorm(X)) (hadamard == 0) or H-BitLinear(RMSNorm(X)) (hadamard != 0): the
+ * layer with the normalisation of bitnet_act_quant_norm fused into its quantiser.  Arguments
+ * as bitnet_act_quant_norm and bitnet_bitlinear_forward; the same workspace size. */
+int bitnet_norm_bitlinear_forward(const void *X_dev, int64_t M, int64_t K,
+                                  const void *norm_gain_dev, float eps, int hadamard,
+                                  const void *Wp_dev, const float *gamma_dev, int64_t N,
+                                  int act_bits, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                  bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* Status                                                                                   */

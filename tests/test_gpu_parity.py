@@ -243,3 +243,87 @@ def test_bounded_wait_time_out_is_reported_and_context_survives(B):
     # the context is still usable: a small forward matches the oracle
     wl = synth.WORKLOADS["tiny"]
     forward_case(B, wl, None)
+
+
+# ----------------------------------------------------------------------------------------
+# RMS normalisation fused into the quantiser (2B4T article, 一.3: subln normalisation;
+# BitNet v2 write-up: RMS normalisation).  The normalised rows are fp32 on the GPU and double
+# in the oracle, so they are held to the transform's tolerance; codes are then exact on the
+# GPU's own rows.
+# ----------------------------------------------------------------------------------------
+
+NORM_EPS = 1e-5
+
+
+def gain_bits(K, seed):
+    g = np.random.default_rng(seed).uniform(0.5, 1.5, K).astype(np.float32)
+    return synth.f32_to_bf16_bits(g)
+
+
+def dev_gain(bits):
+    return None if bits is None else synth.to_torch_bf16(bits).cuda()
+
+
+NORM_CASES = [(128, True), (2048, True), (8192, True), (16384, True),
+              (384, False), (2048, False)]
+
+
+@pytest.mark.parametrize("K,hadamard", NORM_CASES)
+@pytest.mark.parametrize("with_gain", [True, False])
+def test_norm_transform_matches_oracle(B, K, hadamard, with_gain):
+    M = 29 if K <= 8192 else 7
+    X = synth.sharp_activations(M, K, seed=K + 5)
+    g = gain_bits(K, K) if with_gain else None
+    Z = B.bitnet_norm_transform_f32(dev_bf16(X), dev_gain(g), NORM_EPS, hadamard)
+    Z = Z.cpu().numpy().astype(np.float64)
+    ref = oracle.rmsnorm(oracle.bf16_to_f64(X), g, NORM_EPS)
+    if hadamard:
+        ref = oracle.fwht(ref)
+    err = np.abs(Z - ref).max(axis=1) / np.abs(ref).max(axis=1)
+    assert err.max() <= FWHT_REL, err.max()
+
+
+@pytest.mark.parametrize("K,hadamard", NORM_CASES)
+@pytest.mark.parametrize("bits", [8, 4])
+def test_norm_quant_codes_exact_on_the_gpu_rows(B, K, hadamard, bits):
+    M = 33 if K <= 8192 else 9
+    X = synth.sharp_activations(M, K, seed=7 * K + bits)
+    g = gain_bits(K, K + 1)
+    Xd, gd = dev_bf16(X), dev_gain(g)
+    z = B.bitnet_norm_transform_f32(Xd, gd, NORM_EPS, hadamard).cpu().numpy()
+    codes, scales, rowsum = B.bitnet_act_quant_norm(Xd, gd, NORM_EPS, hadamard, bits)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
+    c = codes.cpu().numpy()
+    c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+    assert check_codes(c, c_ref, pre) == 0
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
+
+
+@pytest.mark.parametrize("name,hadamard,rows", [
+    ("wo_2048", True, 48), ("wdown_8192", True, 16), ("decode_m8_k8192", True, None),
+    ("tiny", False, None), ("decode_m32_k2048", False, None),
+])
+def test_norm_forward_end_to_end(B, name, hadamard, rows):
+    wl = synth.WORKLOADS[name]
+    X, W = wl.activations(seed=1), wl.weights(seed=1)
+    g = gain_bits(wl.K, 99)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    Y = B.bitnet_norm_bitlinear_forward(dev_bf16(X), dev_gain(g), NORM_EPS, hadamard, Wp, gamma,
+                                        wl.act_bits)
+    B.bitnet_sync_status()
+    sel = np.arange(wl.M) if rows is None else np.sort(
+        np.random.default_rng(1).choice(wl.M, size=rows, replace=False))
+    ref = oracle.bitlinear_forward(X[sel], W, hadamard, wl.act_bits, norm_gain=g,
+                                   norm_eps=NORM_EPS)
+    y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
+    y_ref = oracle.bf16_to_f64(ref["y"])
+    assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
+
+
+def test_norm_rejects_bad_eps(B):
+    X = dev_bf16(synth.sharp_activations(4, 256, seed=1))
+    for eps in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(B.BitnetError) as err:
+            B.bitnet_act_quant_norm(X, None, eps, True, 8)
+        assert err.value.status == B.ERR_INVALID

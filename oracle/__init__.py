@@ -72,6 +72,7 @@ def lib():
                 "oracle_gemm_i64": (None, [vp, vp, i64, i64, i64, vp]),
                 "oracle_gemm_addsub": (None, [vp, vp, i64, i64, i64, vp]),
                 "oracle_dequant": (None, [vp, vp, f32, i64, i64, vp]),
+                "oracle_dequant_act": (None, [vp, vp, f32, i64, i64, i32, vp]),
                 "oracle_bitlinear_forward": (i32, [vp, i64, i64, vp, i64, i32, i32, vp,
                                                    vp, vp, vp, vp, vp, vp]),
             }
@@ -267,6 +268,20 @@ def dequant(acc: np.ndarray, d: np.ndarray, gamma) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # The whole forward
 # --------------------------------------------------------------------------------------
+
+RELU2, SWIGLU = 1, 2
+
+
+def dequant_act(acc: np.ndarray, d: np.ndarray, gamma, act: int) -> np.ndarray:
+    """Rescale then activation (2B4T article, 一.3: squared ReLU; BitNet v2 write-up: SwishGLU),
+    rounded to bf16 bits.  act RELU2: [M, N]; SWIGLU: rows interleaved gate/up, [M, N/2]."""
+    acc = np.ascontiguousarray(acc, dtype=np.int64)
+    d = np.ascontiguousarray(d, dtype=np.float32)
+    M, N = acc.shape
+    Y = np.empty((M, N if act == RELU2 else N // 2), dtype=np.uint16)
+    lib().oracle_dequant_act(_p(acc), _p(d), float(np.float32(gamma)), M, N, int(act), _p(Y))
+    return Y
+
 
 def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bits: int,
                       norm_gain: np.ndarray | None = None, norm_eps: float | None = None):

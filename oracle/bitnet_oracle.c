@@ -358,6 +358,33 @@ void oracle_dequant(const int64_t *acc, const float *d, float gamma, int64_t M, 
             Y[m * N + n] = double_to_bf16_rn((double)acc[m * N + n] * (double)d[m] * (double)gamma);
 }
 
+/* Activations fused after the rescale, for the up / gate projections that feed the FFN
+ * [2B4T 一.3: squared ReLU activation], [v2: SwishGLU activation].  v = acc * d * gamma in
+ * double, then
+ *   act 1 (squared ReLU): Y[m][n] = bf16(max(v, 0)^2), N columns;
+ *   act 2 (SwiGLU on interleaved rows, feature 2j the gate and 2j+1 the up projection):
+ *         Y[m][j] = bf16(silu(v[2j]) * v[2j+1]), silu(x) = x / (1 + exp(-x)), N/2 columns.
+ * The pages name the activations only; the interleaving is this library's layout. */
+void oracle_dequant_act(const int64_t *acc, const float *d, float gamma, int64_t M, int64_t N,
+                        int act, uint16_t *Y) {
+    for (int64_t m = 0; m < M; ++m) {
+        const double s = (double)d[m] * (double)gamma;
+        if (act == 1) {
+            for (int64_t n = 0; n < N; ++n) {
+                const double v = (double)acc[m * N + n] * s;
+                const double r = v > 0.0 ? v : 0.0;
+                Y[m * N + n] = double_to_bf16_rn(r * r);
+            }
+        } else {
+            for (int64_t j = 0; j < N / 2; ++j) {
+                const double g = (double)acc[m * N + 2 * j] * s;
+                const double u = (double)acc[m * N + 2 * j + 1] * s;
+                Y[m * (N / 2) + j] = double_to_bf16_rn(g / (1.0 + exp(-g)) * u);
+            }
+        }
+    }
+}
+
 /* ------------------------------------------------------------------------------------- */
 /* The whole forward, step by step                                                         */
 /* ------------------------------------------------------------------------------------- */

@@ -431,3 +431,42 @@ def test_forward_with_norm_composes_from_the_stages(hadamard):
     plain = oracle.bitlinear_forward(X, W, hadamard, 8)
     np.testing.assert_array_equal(
         plain["z"], oracle.fwht(oracle.bf16_to_f64(X)) if hadamard else oracle.bf16_to_f64(X))
+
+
+# ----------------------------------------------------------------------------------------
+# Activations after the rescale (2B4T article, 一.3: squared ReLU; BitNet v2 write-up:
+# SwishGLU), fused into the product's epilogue
+# ----------------------------------------------------------------------------------------
+
+def test_squared_relu_closed_forms():
+    # d * gamma = 0.5 exactly, so v = acc / 2 and v^2 are exact in bf16
+    acc = np.arange(-6, 7, dtype=np.int64).reshape(1, -1)
+    y = oracle.bf16_to_f64(oracle.dequant_act(acc, np.array([0.25], np.float32), 2.0,
+                                              oracle.RELU2))
+    expect = np.where(acc > 0, (acc / 2.0) ** 2, 0.0)
+    np.testing.assert_array_equal(y, expect)
+
+
+def test_swiglu_against_library_silu():
+    rng = np.random.default_rng(9)
+    M, N = 7, 64
+    acc = rng.integers(-3000, 3000, size=(M, N)).astype(np.int64)
+    d = rng.uniform(1e-4, 3e-3, size=M).astype(np.float32)
+    gamma = np.float32(0.4375)
+    y = oracle.bf16_to_f64(oracle.dequant_act(acc, d, gamma, oracle.SWIGLU))
+    v = torch.from_numpy(acc.astype(np.float64) * d.astype(np.float64)[:, None] * float(gamma))
+    ref = (torch.nn.functional.silu(v[:, 0::2]) * v[:, 1::2]).numpy()
+    ref_bf16 = oracle.bf16_to_f64(oracle.f64_to_bf16(ref))
+    ulp = np.abs(ref_bf16) * 2.0 ** -7
+    assert np.all(np.abs(y - ref_bf16) <= ulp + 1e-30)
+    assert y.shape == (M, N // 2)
+
+
+def test_swiglu_limits():
+    acc = np.array([[0, 5, 400, 3, -400, 7]], dtype=np.int64)  # (gate, up) pairs
+    y = oracle.bf16_to_f64(oracle.dequant_act(acc, np.array([0.1], np.float32), 1.0,
+                                              oracle.SWIGLU))[0]
+    s = float(np.float32(0.1))
+    assert y[0] == 0.0                                   # silu(0) = 0
+    assert y[1] == oracle.bf16_to_f64(oracle.f64_to_bf16(np.array([400 * s * 3 * s])))[0]
+    assert abs(y[2]) < 1e-15                             # silu(-40) ~ -1.7e-16

@@ -310,7 +310,13 @@ def run_gpu(args, wl, rank, world, device):
         B.bitnet_act_quant(b["X"], wl.hadamard, wl.act_bits, b["codes"], b["scales"],
                            b["rowsum"])
 
+    act = {"none": 0, "relu2": B.ACT_RELU2, "swiglu": B.ACT_SWIGLU}[args.activation]
+
     def gemm(b):
+        if act:  # the activation in the product's epilogue (Y's first M x N' elements)
+            B.bitnet_ternary_gemm_act(b["codes"], b["scales"], b["rowsum"], K, b["Wp"],
+                                      b["gamma"], wl.act_bits, act, Y=b["Y"])
+            return
         B.bitnet_ternary_gemm(b["codes"], b["scales"], b["rowsum"], K, b["Wp"], b["gamma"],
                               wl.act_bits, want_acc=False, want_y=True, Y=b["Y"])
 
@@ -471,6 +477,7 @@ def run_gpu(args, wl, rank, world, device):
             "effective_tops": world * wl.ops / (ms_per_step * 1e-3) / 1e12,
             "config": {"workload": wl.name, "M": M, "K": K, "N": N, "hadamard": wl.hadamard,
                        "act_bits": wl.act_bits, "rmsnorm": bool(args.rmsnorm),
+                       "activation": args.activation,
                        "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {copies} copies "
@@ -550,6 +557,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--workload", default="wo_2048", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--activation", default="none", choices=["none", "relu2", "swiglu"],
+                    help="activation in the product's epilogue (squared ReLU, SwiGLU)")
     ap.add_argument("--rmsnorm", action="store_true",
                     help="RMS-normalise the token rows inside the quantiser (fused prologue)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -20,6 +20,7 @@ _lock = threading.Lock()
 _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+ACT_RELU2, ACT_SWIGLU = 1, 2  # bitnet_activation
 
 
 class BitnetError(RuntimeError):
@@ -79,6 +80,16 @@ _SIGS = {
                                                      ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
                                                      ctypes.c_void_p, ctypes.c_void_p,
                                                      ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_ternary_gemm_act": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_bitlinear_forward_act": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                    ctypes.c_int64, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                    ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_size_t,
+                                                    ctypes.c_void_p]),
     "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bitnet_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
 }
@@ -280,6 +291,56 @@ def bitnet_bitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=N
 def bitnet_hbitlinear_forward(X, Wp, gamma, act_bits=8, Y=None, ws=None, stream=None):
     """Y = H-BitLinear(X): online Hadamard transform, then BitLinear."""
     return _forward("bitnet_hbitlinear_forward", X, Wp, gamma, act_bits, Y, ws, stream)
+
+
+def _act_cols(N: int, activation: int) -> int:
+    return N // 2 if activation == ACT_SWIGLU else N
+
+
+def bitnet_ternary_gemm_act(codes, scales, rowsum, K: int, Wp, gamma, act_bits: int,
+                            activation: int, Y=None, stream=None):
+    """Y = activation(rescaled product): squared ReLU [M, N] or SwiGLU over interleaved gate/up
+    features [M, N/2] (bf16)."""
+    L = load_library()
+    for t, n in ((codes, "codes"), (scales, "scales"), (rowsum, "rowsum"), (Wp, "Wp"),
+                 (gamma, "gamma")):
+        _check(t, n)
+    M = scales.numel()
+    N = Wp.shape[0]
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, act_bits)), "codes")
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if Y is None:
+        Y = torch.empty((M, _act_cols(N, activation)), dtype=torch.bfloat16, device=Wp.device)
+    _nbytes_at_least(Y, 2 * M * _act_cols(N, activation), "Y")
+    _rc(L.bitnet_ternary_gemm_act(codes.data_ptr(), scales.data_ptr(), rowsum.data_ptr(), M, K,
+                                  Wp.data_ptr(), gamma.data_ptr(), N, int(act_bits),
+                                  int(activation), Y.data_ptr(), _stream(stream)),
+        "bitnet_ternary_gemm_act")
+    return Y
+
+
+def bitnet_bitlinear_forward_act(X, Wp, gamma, act_bits, hadamard, activation, Y=None, ws=None,
+                                 stream=None):
+    """Y = activation((H-)BitLinear(X)) with the activation in the product's epilogue."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    _check(Wp, "Wp")
+    _check(gamma, "gamma", torch.float32)
+    M, K = X.shape
+    N = Wp.shape[0]
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if Y is None:
+        Y = torch.empty((M, _act_cols(N, activation)), dtype=torch.bfloat16, device=X.device)
+    _nbytes_at_least(Y, 2 * M * _act_cols(N, activation), "Y")
+    need = int(L.bitnet_workspace_bytes(M, K, N, act_bits))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _rc(L.bitnet_bitlinear_forward_act(X.data_ptr(), M, K, Wp.data_ptr(), gamma.data_ptr(), N,
+                                       int(act_bits), int(bool(hadamard)), int(activation),
+                                       Y.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                       _stream(stream)),
+        "bitnet_bitlinear_forward_act")
+    return Y
 
 
 def _gain_ptr(gain, K):

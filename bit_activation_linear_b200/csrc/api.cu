@@ -126,7 +126,8 @@ int act_quant_impl(DeviceState *st, const void *X, int64_t M, int64_t K, int had
 
 int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int32_t *rowsum,
               int64_t M, int64_t K, const void *Wp, const float *gamma, int64_t N, int act_bits,
-              int32_t *acc, void *Y, cudaStream_t stream, bool early_weights = false) {
+              int32_t *acc, void *Y, cudaStream_t stream, bool early_weights = false,
+              int activation = 0) {
     GemmArgs a;
     a.codes = codes;
     a.scales = scales;
@@ -141,6 +142,7 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
     a.Y = Y;
     a.status = st->status_word;
     a.early_weights = early_weights;
+    a.activation = activation;
     if (M <= kGemvMaxTokens) return launched(launch_ternary_gemv(a, stream), 1, "ternary_gemv");
     const int n = (acc ? 1 : 0) + (Y ? 1 : 0);
     return launched(launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream), n,
@@ -149,7 +151,7 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
 
 int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const float *gamma,
                  int64_t N, int act_bits, void *Y, void *ws, size_t ws_bytes, int hadamard,
-                 cudaStream_t stream, const NormArgs &nrm = NormArgs()) {
+                 cudaStream_t stream, const NormArgs &nrm = NormArgs(), int activation = 0) {
     int rc = check_shape(M, K, N, true, true);
     if (rc) return rc;
     if (act_bits != 8 && act_bits != 4)
@@ -173,7 +175,7 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
         return rc;
     // the quantiser above was launched in stream order after whatever wrote Wp
     return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream,
-                     true);
+                     true, activation);
 }
 
 }  // namespace
@@ -355,6 +357,51 @@ int bitnet_norm_bitlinear_forward(const void *X_dev, int64_t M, int64_t K,
     if (rc) return rc;
     return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, act_bits, Y_dev, ws_dev, ws_bytes,
                         hadamard ? 1 : 0, reinterpret_cast<cudaStream_t>(stream), nrm);
+}
+
+}  // extern "C"
+
+namespace {
+int check_activation(int activation, int64_t N) {
+    if (activation != BITNET_ACT_RELU2 && activation != BITNET_ACT_SWIGLU)
+        return fail(BITNET_ERR_INVALID, "activation = %d must be %d (squared ReLU) or %d (SwiGLU)",
+                    activation, (int)BITNET_ACT_RELU2, (int)BITNET_ACT_SWIGLU);
+    if (activation == BITNET_ACT_SWIGLU && N % 16 != 0)
+        return fail(BITNET_ERR_INVALID, "SwiGLU needs N %% 16 == 0, got N = %lld", (long long)N);
+    return BITNET_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int bitnet_ternary_gemm_act(const void *codes_dev, const float *scales_dev,
+                            const int32_t *rowsum_dev, int64_t M, int64_t K, const void *Wp_dev,
+                            const float *gamma_dev, int64_t N, int act_bits, int activation,
+                            void *Y_dev, bitnet_stream_t stream) {
+    int rc = check_shape(M, K, N, true, true);
+    if (rc) return rc;
+    if ((rc = check_activation(activation, N))) return rc;
+    if (act_bits != 8 && act_bits != 4)
+        return fail(BITNET_ERR_INVALID, "act_bits = %d must be 8 or 4", act_bits);
+    if (!codes_dev || !scales_dev || !rowsum_dev || !Wp_dev || !gamma_dev || !Y_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(codes_dev) || !aligned16(Wp_dev) || !aligned16(Y_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    return gemm_impl(st, codes_dev, scales_dev, rowsum_dev, M, K, Wp_dev, gamma_dev, N, act_bits,
+                     nullptr, Y_dev, reinterpret_cast<cudaStream_t>(stream), false, activation);
+}
+
+int bitnet_bitlinear_forward_act(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                                 const float *gamma_dev, int64_t N, int act_bits, int hadamard,
+                                 int activation, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                 bitnet_stream_t stream) {
+    int rc = check_activation(activation, N);
+    if (rc) return rc;
+    return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, act_bits, Y_dev, ws_dev, ws_bytes,
+                        hadamard ? 1 : 0, reinterpret_cast<cudaStream_t>(stream), NormArgs(),
+                        activation);
 }
 
 int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,

@@ -74,6 +74,11 @@ constexpr uint32_t IDESC = idesc_i8_s8u8(BM, BN);
 static_assert(ACC_BUFS * BN <= TMEM_COLS, "TMEM budget");
 
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_EPI = 16;
+
+// What the epilogue writes: the int32 accumulators (parity entry), the rescaled bf16 output, or
+// the rescaled output through an activation (squared ReLU; SwiGLU over interleaved gate/up
+// features, half as many columns).
+enum OutMode { OUT_ACC = 0, OUT_BF16 = 1, OUT_RELU2 = 2, OUT_SWIGLU = 3 };
 constexpr int NUM_THREADS = 24 * 32;
 
 // Unpack / code warps: eight warps outside the MMA warp's scheduler partition (warp % 4 == 1).
@@ -127,7 +132,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *s
     return ok;
 }
 
-template <int BITS, bool OUT_I32>
+template <int BITS, int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ternary_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                            const __grid_constant__ CUtensorMap tmap_w,
@@ -181,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (warp == WARP_TMA && lane == 0) {
         prefetch_tensormap(&tmap_codes);
         prefetch_tensormap(&tmap_w);
-        if (!OUT_I32) prefetch_tensormap(&tmap_y);
+        if (MODE != OUT_ACC) prefetch_tensormap(&tmap_y);
     }
     if (warp == WARP_MMA) {
         tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
@@ -360,7 +365,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_32x32b_x32(t_lane + ab * BN + col, v);
                 tmem_wait_ld();
                 const int n0 = nf * BN + col;
-                if constexpr (OUT_I32) {
+                if constexpr (MODE == OUT_ACC) {
                     int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -374,18 +379,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     // bf16 pairs of this token's 32 features, then out through the warp's
                     // staging box by bulk tensor stores: 16 features x 32 tokens per store, the
                     // box rows in the 32-byte-swizzled layout (chunk c of row r at c ^ (r >> 2 & 1))
+                    // (SwiGLU: pair i of the chunk is (gate, up) = features 2i, 2i+1; its 16
+                    // outputs fill one box at output column n0 / 2)
+                    constexpr int BOXES = MODE == OUT_SWIGLU ? 1 : 2;
                     uint32_t pk[16];
+                    if constexpr (MODE == OUT_SWIGLU) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float y0 = (float)((int)v[2 * i] - rs) * sc;
-                        const float y1 = (float)((int)v[2 * i + 1] - rs) * sc;
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-                        pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+                        for (int i = 0; i < 8; ++i) {
+                            float o[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float g = (float)((int)v[4 * i + 2 * e] - rs) * sc;
+                                const float u = (float)((int)v[4 * i + 2 * e + 1] - rs) * sc;
+                                o[e] = __fdiv_rn(g, 1.f + expf(-g)) * u;
+                            }
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
+                            pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float y0 = (float)((int)v[2 * i] - rs) * sc;
+                            float y1 = (float)((int)v[2 * i + 1] - rs) * sc;
+                            if constexpr (MODE == OUT_RELU2) {
+                                y0 = y0 > 0.f ? y0 * y0 : 0.f;
+                                y1 = y1 > 0.f ? y1 * y1 : 0.f;
+                            }
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+                            pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+                        }
                     }
                     const int m_w = mt * BM + (int)rank * HM + wq * 32;  // the warp's first token
                     const int sx = (lane >> 2) & 1;
+                    const int nx0 = MODE == OUT_SWIGLU ? n0 / 2 : n0;  // first output column
+                    const int n_out = MODE == OUT_SWIGLU ? N / 2 : N;
 #pragma unroll
-                    for (int hb = 0; hb < 2; ++hb) {
+                    for (int hb = 0; hb < BOXES; ++hb) {
                         if (lane == 0) bulk_wait_group_read<0>();  // the previous box was read
                         __syncwarp();
 #pragma unroll
@@ -397,8 +426,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         __syncwarp();
                         // rows >= M and features >= N of a box are not written; a box wholly
                         // outside Y is not issued
-                        if (lane == 0 && m_w < M && n0 + hb * Y_BOX_N < N) {
-                            tma_store_2d(&tmap_y, ybox, n0 + hb * Y_BOX_N, m_w);
+                        if (lane == 0 && m_w < M && nx0 + hb * Y_BOX_N < n_out) {
+                            tma_store_2d(&tmap_y, ybox, nx0 + hb * Y_BOX_N, m_w);
                             bulk_commit_group();
                         }
                     }
@@ -461,7 +490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
 // Co-resident pairs per device (a persistent grid of one pair per two SMs where the GPU's
 // layout allows it), looked up once per device and kernel instance.
-template <int BITS, bool OUT_I32>
+template <int BITS, int MODE>
 static int max_pairs(int num_sms) {
     static int cache[64] = {};
     int dev = 0;
@@ -472,7 +501,7 @@ static int max_pairs(int num_sms) {
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, ternary_gemm_tc_kernel<BITS, OUT_I32>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&clusters, ternary_gemm_tc_kernel<BITS, MODE>, &cfg) !=
             cudaSuccess ||
         clusters < 1) {
         (void)cudaGetLastError();
@@ -482,11 +511,11 @@ static int max_pairs(int num_sms) {
     return clusters;
 }
 
-template <int BITS, bool OUT_I32>
+template <int BITS, int MODE>
 static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
                                const CUtensorMap &my, void *out, int64_t tiles, int num_sms,
                                cudaStream_t stream) {
-    auto kern = ternary_gemm_tc_kernel<BITS, OUT_I32>;
+    auto kern = ternary_gemm_tc_kernel<BITS, MODE>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -496,7 +525,7 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    const int pairs_max = max_pairs<BITS, OUT_I32>(num_sms);
+    const int pairs_max = max_pairs<BITS, MODE>(num_sms);
     const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
@@ -550,18 +579,26 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (a.Y) {
-        // bf16 output [M rows][N], one [32 tokens x 16 features] box per store, 32-byte swizzle
-        if (encode_2d(encode_fn, &my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, (uint64_t)a.N,
-                      (uint64_t)a.M, (uint64_t)a.N * 2, Y_BOX_N, 32,
-                      CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+        // bf16 output [M rows][N] (N/2 with SwiGLU), one [32 tokens x 16 features] box per
+        // store, 32-byte swizzle
+        const uint64_t n_out = a.activation == 2 ? (uint64_t)a.N / 2 : (uint64_t)a.N;
+        if (encode_2d(encode_fn, &my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, n_out, (uint64_t)a.M,
+                      n_out * 2, Y_BOX_N, 32, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-        e = a.act_bits == 8 ? launch_tc_t<8, false>(a, mc, mw, my, a.Y, tiles, num_sms, stream)
-                            : launch_tc_t<4, false>(a, mc, mw, my, a.Y, tiles, num_sms, stream);
+        switch (a.activation * 2 + (a.act_bits == 8 ? 1 : 0)) {
+            case 0: e = launch_tc_t<4, OUT_BF16>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            case 1: e = launch_tc_t<8, OUT_BF16>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            case 2: e = launch_tc_t<4, OUT_RELU2>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            case 3: e = launch_tc_t<8, OUT_RELU2>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            case 4: e = launch_tc_t<4, OUT_SWIGLU>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            case 5: e = launch_tc_t<8, OUT_SWIGLU>(a, mc, mw, my, a.Y, tiles, num_sms, stream); break;
+            default: return cudaErrorInvalidValue;
+        }
         if (e != cudaSuccess) return e;
     }
     if (a.acc) {
-        e = a.act_bits == 8 ? launch_tc_t<8, true>(a, mc, mw, my, a.acc, tiles, num_sms, stream)
-                            : launch_tc_t<4, true>(a, mc, mw, my, a.acc, tiles, num_sms, stream);
+        e = a.act_bits == 8 ? launch_tc_t<8, OUT_ACC>(a, mc, mw, my, a.acc, tiles, num_sms, stream)
+                            : launch_tc_t<4, OUT_ACC>(a, mc, mw, my, a.acc, tiles, num_sms, stream);
     }
     return e;
 }

@@ -22,7 +22,9 @@ namespace bitnet {
 constexpr int kGemvSteps = 16;      // 512-weight steps whose weight loads are in flight together
 constexpr int kGemvWarps = 4;       // warps per CTA
 
-template <int BITS, int T, int R>
+// ACT: 0 rescaled output, 1 squared ReLU of it, 2 SwiGLU over the warp's two rows (gate, up =
+// features 2j, 2j+1; output column j; needs R == 2).
+template <int BITS, int T, int R, int ACT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                         const int32_t *__restrict__ rowsum, int M, int K,
@@ -92,24 +94,46 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
         }
     }
     const float gamma = *gamma_ptr;
+    static_assert(ACT != 2 || R == 2, "SwiGLU needs the gate and up rows in one warp");
+    int sums[R][T];  // full sums, the same in every lane
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-            if (t >= M) break;
             int s = acc[r][t];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-            const int n = n0 + r;
-            if (lane == r * T + t && n < N) {
-                const int a = s - rowsum[t];
-                if (acc_out) acc_out[(int64_t)t * N + n] = a;
-                if (Y) Y[(int64_t)t * N + n] = __float2bfloat16_rn((float)a * (scales[t] * gamma));
+            sums[r][t] = s;
+        }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        if (t >= M) break;
+        const float sc = scales[t] * gamma;
+        if constexpr (ACT == 2) {
+            if (lane == t && n0 + 1 < N) {
+                const float g = (float)(sums[0][t] - rowsum[t]) * sc;
+                const float u = (float)(sums[1][t] - rowsum[t]) * sc;
+                Y[(int64_t)t * (N / 2) + n0 / 2] = __float2bfloat16_rn(__fdiv_rn(g, 1.f + expf(-g)) * u);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int n = n0 + r;
+                if (lane == r * T + t && n < N) {
+                    const int a = sums[r][t] - rowsum[t];
+                    if (acc_out) acc_out[(int64_t)t * N + n] = a;
+                    if (Y) {
+                        float y = (float)a * sc;
+                        if constexpr (ACT == 1) y = y > 0.f ? y * y : 0.f;
+                        Y[(int64_t)t * N + n] = __float2bfloat16_rn(y);
+                    }
+                }
             }
         }
+    }
 }
 
-template <int BITS, int T, int R>
+template <int BITS, int T, int R, int ACT>
 static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
     static_assert(R * T <= 32, "one lane per (row, token) result");
     const int64_t warps = (a.N + R - 1) / R;
@@ -123,18 +147,26 @@ static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<BITS, T, R>,
+    return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<BITS, T, R, ACT>,
                               reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum,
                               (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
                               reinterpret_cast<__nv_bfloat16 *>(a.Y), a.early_weights ? 1 : 0);
 }
 
+template <int BITS, int ACT>
+static cudaError_t launch_gemv_a(const GemmArgs &a, cudaStream_t stream) {
+    constexpr int R_SMALL = ACT == 2 ? 2 : 1;  // SwiGLU keeps the row pair in one warp
+    if (a.M <= 1) return launch_gemv_t<BITS, 1, R_SMALL, ACT>(a, stream);
+    if (a.M <= 2) return launch_gemv_t<BITS, 2, R_SMALL, ACT>(a, stream);
+    if (a.M <= 4) return launch_gemv_t<BITS, 4, 2, ACT>(a, stream);
+    return launch_gemv_t<BITS, 8, 2, ACT>(a, stream);
+}
+
 template <int BITS>
 static cudaError_t launch_gemv_b(const GemmArgs &a, cudaStream_t stream) {
-    if (a.M <= 1) return launch_gemv_t<BITS, 1, 1>(a, stream);
-    if (a.M <= 2) return launch_gemv_t<BITS, 2, 1>(a, stream);
-    if (a.M <= 4) return launch_gemv_t<BITS, 4, 2>(a, stream);
-    return launch_gemv_t<BITS, 8, 2>(a, stream);
+    if (a.acc || a.activation == 0) return launch_gemv_a<BITS, 0>(a, stream);
+    return a.activation == 1 ? launch_gemv_a<BITS, 1>(a, stream)
+                             : launch_gemv_a<BITS, 2>(a, stream);
 }
 
 cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream) {

@@ -51,6 +51,9 @@ struct GemmArgs {
     // stream started (true when the library's own quantiser runs in between, as in the forward
     // entries): the decode kernel may then load them before waiting for that kernel.
     bool early_weights = false;
+    // 0: Y = rescaled output; 1: squared ReLU of it; 2: SwiGLU over interleaved gate/up
+    // features (Y has N/2 columns)
+    int activation = 0;
 };
 
 // Weight-streaming kernel for few tokens (decode).

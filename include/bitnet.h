@@ -170,6 +170,23 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
                         const float *gamma_dev, int64_t N, int act_bits, int32_t *acc_dev,
                         void *Y_dev, bitnet_stream_t stream);
 
+/*
+ * Activations fused into the product's epilogue, for the up / gate projections that feed the
+ * FFN (BitNet b1.58 2B4T article, section 一.3: squared ReLU; BitNet v2 write-up: SwishGLU).
+ * With y = float(acc) * (scales[m] * gamma) as in bitnet_ternary_gemm:
+ *   BITNET_ACT_RELU2   Y[m, n] = bf16_rn(max(y, 0) * max(y, 0))                Y bf16 [M, N]
+ *   BITNET_ACT_SWIGLU  Y[m, j] = bf16_rn(silu(y[m, 2j]) * y[m, 2j + 1])         Y bf16 [M, N/2]
+ * silu(x) = x / (1 + exp(-x)).  For SwiGLU the weight rows are interleaved: feature 2j is the
+ * gate projection and 2j + 1 the up projection of output j, and N % 16 == 0.  Other arguments
+ * as bitnet_ternary_gemm (only the bf16 output); an unknown activation is BITNET_ERR_INVALID.
+ */
+typedef enum { BITNET_ACT_RELU2 = 1, BITNET_ACT_SWIGLU = 2 } bitnet_activation;
+
+int bitnet_ternary_gemm_act(const void *codes_dev, const float *scales_dev,
+                            const int32_t *rowsum_dev, int64_t M, int64_t K, const void *Wp_dev,
+                            const float *gamma_dev, int64_t N, int act_bits, int activation,
+                            void *Y_dev, bitnet_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------- */
 /* The whole layer                                                                          */
 /* ---------------------------------------------------------------------------------------- */
@@ -201,6 +218,13 @@ int bitnet_norm_bitlinear_forward(const void *X_dev, int64_t M, int64_t K,
                                   const void *Wp_dev, const float *gamma_dev, int64_t N,
                                   int act_bits, void *Y_dev, void *ws_dev, size_t ws_bytes,
                                   bitnet_stream_t stream);
+
+/* Y = act(BitLinear(X)) (hadamard == 0) or act(H-BitLinear(X)): the layer with the activation of
+ * bitnet_ternary_gemm_act in its epilogue.  Y is bf16 [M, N] or [M, N/2] (SwiGLU). */
+int bitnet_bitlinear_forward_act(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                                 const float *gamma_dev, int64_t N, int act_bits, int hadamard,
+                                 int activation, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                 bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* Status                                                                                   */

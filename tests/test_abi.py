@@ -113,3 +113,15 @@ def test_binding_raises_without_library(tmp_path):
 def test_selftest_rejects_bad_limits_before_touching_the_device(lib):
     for limit in (0, -5, 3_000_000_000):
         assert lib.bitnet_selftest_wait_timeout(ctypes.c_int64(limit), None) == -1  # INVALID
+
+
+def test_activation_entries_reject_bad_arguments_before_the_device(lib):
+    p = ctypes.c_void_p(16)
+    # unknown activation
+    rc = lib.bitnet_ternary_gemm_act(p, p, p, 8, 256, p, p, 256, 8, 3, p, None)
+    assert rc == -1
+    # SwiGLU needs N % 16 == 0
+    rc = lib.bitnet_ternary_gemm_act(p, p, p, 8, 256, p, p, 264, 8, 2, p, None)
+    assert rc == -1
+    rc = lib.bitnet_bitlinear_forward_act(p, 8, 256, p, p, 264, 8, 0, 2, p, p, 1 << 20, None)
+    assert rc == -1

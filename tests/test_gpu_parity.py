@@ -327,3 +327,59 @@ def test_norm_rejects_bad_eps(B):
         with pytest.raises(B.BitnetError) as err:
             B.bitnet_act_quant_norm(X, None, eps, True, 8)
         assert err.value.status == B.ERR_INVALID
+
+
+# ----------------------------------------------------------------------------------------
+# activations fused into the product's epilogue (2B4T article, 一.3: squared ReLU; BitNet v2
+# write-up: SwishGLU), staged on the GPU's codes and end to end
+# ----------------------------------------------------------------------------------------
+
+def check_act(Y, y_ref_bits):
+    y = oracle.bf16_to_f64(to_np_bits(Y))
+    y_ref = oracle.bf16_to_f64(y_ref_bits)
+    assert y.shape == y_ref.shape
+    rel = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), 1e-30)
+    assert np.all((rel <= Y_REL) | (y_ref == 0)), rel.max()
+    # squared ReLU: zeros exactly where the accumulator is <= 0; SwiGLU: silu(0) * u = 0
+    assert np.all(np.abs(y[y_ref == 0]) <= 1e-30)
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (1, 256, 256), (5, 2048, 272), (8, 384, 528),               # decode kernel
+    (9, 256, 256), (300, 2048, 272), (1000, 640, 528),          # tensor-core kernel
+])
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("act", [1, 2])
+def test_product_activation_matches_oracle(B, M, K, N, bits, act):
+    X = synth.sharp_activations(M, K, seed=M + K)
+    W = synth.latent_weights(N, K, seed=N + 3)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    hadamard = (K & (K - 1)) == 0
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), hadamard, bits)
+    acc, _ = B.bitnet_ternary_gemm(codes, scales, rowsum, K, Wp, gamma, bits, want_acc=True,
+                                   want_y=False)
+    Y = B.bitnet_ternary_gemm_act(codes, scales, rowsum, K, Wp, gamma, bits, act)
+    B.bitnet_sync_status()
+    c = codes.cpu().numpy()
+    c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+    q, _ = oracle.unpack_ternary(Wp.cpu().numpy().view(np.uint32), K)
+    acc_ref = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(acc.cpu().numpy().astype(np.int64), acc_ref)
+    check_act(Y, oracle.dequant_act(acc_ref, scales.cpu().numpy(), np.float32(gamma.item()), act))
+
+
+@pytest.mark.parametrize("name,act", [("up_7b", 1), ("up_7b", 2), ("tiny", 2),
+                                      ("decode_m8_k2048", 1), ("decode_m1_k8192", 2)])
+def test_forward_activation_end_to_end(B, name, act):
+    wl = synth.WORKLOADS[name]
+    rows = 24 if wl.M > 64 else None
+    X, W = wl.activations(seed=2), wl.weights(seed=2)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    Y = B.bitnet_bitlinear_forward_act(dev_bf16(X), Wp, gamma, wl.act_bits, wl.hadamard, act)
+    B.bitnet_sync_status()
+    sel = np.arange(wl.M) if rows is None else np.sort(
+        np.random.default_rng(2).choice(wl.M, size=rows, replace=False))
+    ref = oracle.bitlinear_forward(X[sel], W, wl.hadamard, wl.act_bits)
+    y_ref = oracle.bf16_to_f64(oracle.dequant_act(ref["acc"], ref["d"], ref["gamma"], act))
+    y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
+    assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL

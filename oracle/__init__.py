@@ -61,6 +61,8 @@ def lib():
                 "oracle_pack_ternary": (None, [vp, i64, i64, vp]),
                 "oracle_unpack_ternary": (i64, [vp, i64, i64, vp]),
                 "oracle_pack_base3": (None, [vp, i64, vp]),
+                "oracle_pack_ternary_base3": (None, [vp, i64, i64, vp]),
+                "oracle_unpack_ternary_base3": (i64, [vp, i64, i64, vp]),
                 "oracle_unpack_base3": (None, [vp, i64, vp]),
                 "oracle_fwht": (None, [vp, i64, i64, vp]),
                 "oracle_rmsnorm": (None, [vp, i64, i64, vp, f64, vp]),
@@ -162,6 +164,25 @@ def unpack_base3(b: np.ndarray, n: int) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # Step 2: online Hadamard transform  (BitNet v2 write-up, H-BitLinear paragraphs)
 # --------------------------------------------------------------------------------------
+
+def pack_ternary_base3(q: np.ndarray) -> np.ndarray:
+    """Ternary int8 [N, K] -> base-3 rows, uint32 [N, ceil(K/20)] (BitNet b1.58 2B4T article,
+    一.1: five ternary weights per byte; this library's row layout for the decode product)."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N, K = q.shape
+    out = np.zeros((N, (K + 19) // 20), dtype=np.uint32)
+    lib().oracle_pack_ternary_base3(_p(q), N, K, _p(out))
+    return out
+
+
+def unpack_ternary_base3(words: np.ndarray, K: int):
+    """Inverse of pack_ternary_base3: (q int8 [N, K], count of invalid bytes or padding)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    N = words.shape[0]
+    q = np.empty((N, K), dtype=np.int8)
+    bad = lib().oracle_unpack_ternary_base3(_p(words), N, K, _p(q))
+    return q, int(bad)
+
 
 def rmsnorm(x: np.ndarray, gain_bf16: np.ndarray | None = None, eps: float = 1e-5) -> np.ndarray:
     """y = x * g / sqrt(mean(x^2) + eps) per row, in double (BitNet b1.58 2B4T article, 一.3:

@@ -196,6 +196,42 @@ void oracle_unpack_base3(const uint8_t *bytes, int64_t n, uint8_t *digits) {
     }
 }
 
+/* Base-3 storage of a ternary matrix for the decode product, built on oracle_pack_base3
+ * [2B4T 一.1]: row n is ceil(K/20) 32-bit little-endian words; byte i of word w holds the offset
+ * codes u = q + 1 of weights k = 20w + 5i .. 20w + 5i + 4 as one base-3 number, first weight
+ * most significant; weights k >= K are stored as u = 1 (q = 0).  1.6 bits per weight. */
+void oracle_pack_ternary_base3(const int8_t *q, int64_t N, int64_t K, uint32_t *out) {
+    const int64_t words = (K + 19) / 20;
+    uint8_t *dig = malloc((size_t)(words * 20));
+    if (!dig) return;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < words * 20; ++k)
+            dig[k] = k < K ? (uint8_t)(q[n * K + k] + 1) : 1u;
+        oracle_pack_base3(dig, words * 20, (uint8_t *)(out + n * words));
+    }
+    free(dig);
+}
+
+/* Inverse of oracle_pack_ternary_base3.  Returns the number of bytes that are not valid base-3
+ * numbers (>= 243) plus the number of padding weights not stored as u = 1. */
+int64_t oracle_unpack_ternary_base3(const uint32_t *in, int64_t N, int64_t K, int8_t *q) {
+    const int64_t words = (K + 19) / 20;
+    uint8_t *dig = malloc((size_t)(words * 20));
+    if (!dig) return -1;
+    int64_t bad = 0;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t *bytes = (const uint8_t *)(in + n * words);
+        for (int64_t b = 0; b < words * 4; ++b) bad += bytes[b] >= 243;
+        oracle_unpack_base3(bytes, words * 20, dig);
+        for (int64_t k = 0; k < words * 20; ++k) {
+            if (k < K) q[n * K + k] = (int8_t)((int)dig[k] - 1);
+            else bad += dig[k] != 1;
+        }
+    }
+    free(dig);
+    return bad;
+}
+
 /* ------------------------------------------------------------------------------------- */
 /* Before step 2: RMS normalisation of each token row  [2B4T 一.3: subln normalisation in  */
 /* place of LayerNorm], [v2: LLaMA-like components with RMS normalisation]                 */

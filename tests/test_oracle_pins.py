@@ -470,3 +470,35 @@ def test_swiglu_limits():
     assert y[0] == 0.0                                   # silu(0) = 0
     assert y[1] == oracle.bf16_to_f64(oracle.f64_to_bf16(np.array([400 * s * 3 * s])))[0]
     assert abs(y[2]) < 1e-15                             # silu(-40) ~ -1.7e-16
+
+
+# ----------------------------------------------------------------------------------------
+# Base-3 rows for the decode product (2B4T article, 一.1: five ternary weights per byte)
+# ----------------------------------------------------------------------------------------
+
+def test_base3_rows_carry_the_page_example():
+    # the first five weights of a row with offset codes 2,0,1,2,1 (q = 1,-1,0,1,0): byte 178
+    q = np.zeros((2, 40), np.int8)
+    q[1, :5] = [1, -1, 0, 1, 0]
+    words = oracle.pack_ternary_base3(q)
+    assert words.shape == (2, 2)
+    assert words[1, 0] & 0xFF == 178
+    # all-zero weights are offset code 1 everywhere: 1,1,1,1,1 -> 81+27+9+3+1 = 121 per byte
+    assert words[0, 0] == 121 * 0x01010101
+
+
+@pytest.mark.parametrize("K", [128, 2048, 8192, 384])
+def test_base3_rows_round_trip_and_size(K):
+    rng = np.random.default_rng(K)
+    q = rng.integers(-1, 2, size=(5, K)).astype(np.int8)
+    words = oracle.pack_ternary_base3(q)
+    assert words.shape == (5, (K + 19) // 20)                 # 1.6 bits per weight, rounded up
+    bytes_ = words.view(np.uint8)
+    assert bytes_.max() < 243
+    back, bad = oracle.unpack_ternary_base3(words, K)
+    assert bad == 0
+    np.testing.assert_array_equal(back, q)
+    # brute force on one row: each byte is sum u_i 3^(4-i) over its five weights
+    row = np.concatenate([q[2] + 1, np.ones((-K) % 20, np.int64)])
+    expect = (row.reshape(-1, 5) * np.array([81, 27, 9, 3, 1])).sum(axis=1)
+    np.testing.assert_array_equal(words[2].view(np.uint8), expect.astype(np.uint8))

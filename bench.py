@@ -59,19 +59,26 @@ def load_peaks():
 # algorithmic work per kernel (bytes at the stored widths, ops of the product)
 # ----------------------------------------------------------------------------------------
 
-def kernel_work(wl):
+def weight_bytes(N: int, K: int, base3: bool) -> int:
+    """Bytes of stored ternary weights: 2 bits a weight, or rows of ceil(K/20) 32-bit words of
+    five base-3 weights a byte."""
+    return N * 4 * ((K + 19) // 20) if base3 else N * K // 4
+
+
+def kernel_work(wl, base3: bool = False):
     M, K, N = wl.M, wl.K, wl.N
     code_bytes = M * K if wl.act_bits == 8 else M * K // 2
+    wb = weight_bytes(N, K, base3)
     return {
         # read W (bf16) once
         "absmean_partials": {"bytes": 2 * N * K},
-        # read W (bf16) once, write the 2-bit weights
-        "ternarize_pack": {"bytes": 2 * N * K + N * K // 4},
+        # read W (bf16) once, write the stored weights
+        "ternarize_pack": {"bytes": 2 * N * K + wb},
         # read X (bf16), write codes + scale + code sum per token
         "fwht_quant": {"bytes": 2 * M * K + code_bytes + 8 * M},
         # product: 2 M N K integer ops; bytes = codes + 2-bit weights + bf16 Y
         "ternary_gemm_tc": {"ops": 2 * M * N * K,
-                            "bytes": code_bytes + N * K // 4 + 2 * M * N + 8 * M},
+                            "bytes": code_bytes + wb + 2 * M * N + 8 * M},
     }
 
 
@@ -270,7 +277,7 @@ def run_gpu(args, wl, rank, world, device):
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     M, K, N = wl.M, wl.K, wl.N
     code_bytes = M * K if wl.act_bits == 8 else M * K // 2
-    per_copy = 2 * M * K + 2 * N * K + N * K // 4 + code_bytes + 2 * M * N
+    per_copy = 2 * M * K + 2 * N * K + weight_bytes(N, K, args.base3) + code_bytes + 2 * M * N
     copies = max(2, math.ceil(2 * l2 / per_copy) + 1)
 
     # inputs: one batch per rank (seed = rank), rotated copies of X and W
@@ -280,7 +287,8 @@ def run_gpu(args, wl, rank, world, device):
     for i in range(copies):
         X = X0.to(device, non_blocking=False).clone()
         W = W0.to(device).clone()
-        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=device)
+        Wp = torch.empty((N, weight_bytes(N, K, args.base3) // N), dtype=torch.uint8,
+                         device=device)
         gamma = torch.empty(1, dtype=torch.float32, device=device)
         wws = torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
                           device=device)
@@ -293,6 +301,9 @@ def run_gpu(args, wl, rank, world, device):
                          rowsum=rowsum, Y=Y))
 
     def weights(b):
+        if args.base3:
+            B.bitnet_quantize_pack_weights_base3(b["W"], b["Wp"], b["gamma"], b["wws"])
+            return
         B.bitnet_quantize_pack_weights(b["W"], b["Wp"], b["gamma"], b["wws"])
 
     # with --rmsnorm the token rows are RMS-normalised inside the quantiser (gain of ones
@@ -313,6 +324,10 @@ def run_gpu(args, wl, rank, world, device):
     act = {"none": 0, "relu2": B.ACT_RELU2, "swiglu": B.ACT_SWIGLU}[args.activation]
 
     def gemm(b):
+        if args.base3:  # decode product on base-3 weights (Y's first M x N' elements)
+            B.bitnet_ternary_gemv_base3(b["codes"], b["scales"], b["rowsum"], K, b["Wp"],
+                                        b["gamma"], act, Y=b["Y"])
+            return
         if act:  # the activation in the product's epilogue (Y's first M x N' elements)
             B.bitnet_ternary_gemm_act(b["codes"], b["scales"], b["rowsum"], K, b["Wp"],
                                       b["gamma"], wl.act_bits, act, Y=b["Y"])
@@ -439,7 +454,7 @@ def run_gpu(args, wl, rank, world, device):
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
-        work = kernel_work(wl)
+        work = kernel_work(wl, args.base3)
         int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
         achieved = work["ternary_gemm_tc"]["ops"] / (gemm_ms * 1e-3) / 1e12
         hbm = peaks["hbm_gbs"]
@@ -455,11 +470,33 @@ def run_gpu(args, wl, rank, world, device):
                 "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,
                 "achieved_gbs": q_bytes / (phase_ms[1] * 1e-3) / 1e9,
                 "frac": q_bytes / (phase_ms[1] * 1e-3) / 1e9 / hbm},
-            ("ternary_gemm_tc" if M > 8 else "ternary_gemv"): {
-                "us": 1e3 * gemm_ms, "bound": "tensor" if M > 8 else "hbm",
-                "ops": work["ternary_gemm_tc"]["ops"],
-                "achieved_tops": achieved, "frac": achieved / int8_peak},
         }
+        prod_bytes = work["ternary_gemm_tc"]["bytes"]
+        prod_gbs = prod_bytes / (gemm_ms * 1e-3) / 1e9
+        if M > 8:
+            per_kernel["ternary_gemm_tc"] = {
+                "us": 1e3 * gemm_ms, "bound": "tensor", "ops": work["ternary_gemm_tc"]["ops"],
+                "achieved_tops": achieved, "frac": achieved / int8_peak}
+            roofline = {"kernel": "ternary_gemm_tc", "bound": "tensor",
+                        "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
+                        "frac": achieved / int8_peak,
+                        "traffic": ncu_traffic("ternary_gemm_tc_kernel", wl.name),
+                        "ms_per_launch": gemm_ms,
+                        "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x "
+                                       f"{INT8_PER_BF16} (nominal int8:bf16 dense ratio)"}
+        else:
+            # a few tokens: the product streams the stored weights once (bytes = weights +
+            # codes + bf16 Y), so HBM bounds it
+            gemv = "ternary_gemv_base3" if args.base3 else "ternary_gemv"
+            per_kernel[gemv] = {
+                "us": 1e3 * gemm_ms, "bound": "hbm", "bytes": prod_bytes,
+                "achieved_gbs": prod_gbs, "frac": prod_gbs / hbm,
+                "ops": work["ternary_gemm_tc"]["ops"], "achieved_tops": achieved}
+            roofline = {"kernel": gemv, "bound": "hbm", "achieved": prod_gbs, "peak": hbm,
+                        "unit": "GB/s", "frac": prod_gbs / hbm,
+                        "traffic": ncu_traffic(gemv + "_kernel", wl.name),
+                        "ms_per_launch": gemm_ms,
+                        "peak_source": f"{peak_kind} HBM copy bandwidth"}
         tokens_per_s = job_tokens_per_s(world, M, ms_per_step)
         line = {
             "metric": METRIC,
@@ -478,17 +515,12 @@ def run_gpu(args, wl, rank, world, device):
             "config": {"workload": wl.name, "M": M, "K": K, "N": N, "hadamard": wl.hadamard,
                        "act_bits": wl.act_bits, "rmsnorm": bool(args.rmsnorm),
                        "activation": args.activation,
+                       "weights": "base3" if args.base3 else "2bit",
                        "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {copies} copies "
                              f"({copies * per_copy / 2**20:.0f} MiB > 2 x L2)"},
-            "roofline": {"kernel": "ternary_gemm_tc", "bound": "tensor",
-                         "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
-                         "frac": achieved / int8_peak,
-                         "traffic": ncu_traffic("ternary_gemm_tc_kernel", wl.name),
-                         "ms_per_launch": gemm_ms,
-                         "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x "
-                                        f"{INT8_PER_BF16} (nominal int8:bf16 dense ratio)"},
+            "roofline": roofline,
             "kernels": per_kernel,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
@@ -518,7 +550,8 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
             Yh=torch.empty((M, n_out), dtype=torch.bfloat16).pin_memory(),
             Xd=torch.empty_like(Xh, device=device), Wd=torch.empty_like(Wh, device=device),
             Yd=torch.empty((M, n_out), dtype=torch.bfloat16, device=device),
-            Wp=torch.empty((N, K // 4), dtype=torch.uint8, device=device),
+            Wp=torch.empty((N, weight_bytes(N, K, args.base3) // N), dtype=torch.uint8,
+                           device=device),
             gamma=torch.empty(1, dtype=torch.float32, device=device),
             wws=torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
                             device=device),
@@ -530,7 +563,10 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
         gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
 
     def fwd(b):
-        if gain is not None:
+        if args.base3:
+            B.bitnet_bitlinear_forward_base3(b["Xd"], b["Wp"], b["gamma"], wl.hadamard, act,
+                                             Y=b["Yd"], ws=b["ws"])
+        elif gain is not None:
             B.bitnet_norm_bitlinear_forward(b["Xd"], gain, 1e-5, wl.hadamard, b["Wp"], b["gamma"],
                                             wl.act_bits, Y=b["Yd"], ws=b["ws"])
         elif act:
@@ -560,7 +596,9 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
             ev_in[k].record(s_in)
         with torch.cuda.stream(s_c):
             s_c.wait_event(ev_in[k])
-            B.bitnet_quantize_pack_weights(b["Wd"], b["Wp"], b["gamma"], b["wws"])
+            pack = (B.bitnet_quantize_pack_weights_base3 if args.base3
+                    else B.bitnet_quantize_pack_weights)
+            pack(b["Wd"], b["Wp"], b["gamma"], b["wws"])
             fwd(b)
             ev_c[k].record(s_c)
         with torch.cuda.stream(s_out):
@@ -600,6 +638,9 @@ def main():
                     help="activation in the product's epilogue (squared ReLU, SwiGLU)")
     ap.add_argument("--rmsnorm", action="store_true",
                     help="RMS-normalise the token rows inside the quantiser (fused prologue)")
+    ap.add_argument("--base3", action="store_true",
+                    help="store the weights five to a byte (base 3) for the decode product "
+                         "(at most 8 tokens, INT8 activations)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -610,6 +651,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = synth.WORKLOADS[args.workload]
+    if args.base3 and (wl.M > 8 or wl.act_bits != 8 or args.rmsnorm):
+        ap.error("--base3 serves workloads of at most 8 tokens with INT8 activations, "
+                 "without --rmsnorm")
 
     if args.impl == "reference":
         run_reference(args, wl, rank, world)

@@ -90,6 +90,22 @@ _SIGS = {
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                                     ctypes.c_void_p, ctypes.c_size_t,
                                                     ctypes.c_void_p]),
+    "bitnet_base3_weight_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "bitnet_quantize_pack_weights_base3": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                          ctypes.c_int64, ctypes.c_void_p,
+                                                          ctypes.c_void_p, ctypes.c_void_p,
+                                                          ctypes.c_size_t, ctypes.c_void_p]),
+    "bitnet_ternary_gemv_base3": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                 ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p]),
+    "bitnet_bitlinear_forward_base3": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                      ctypes.c_int64, ctypes.c_void_p,
+                                                      ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                                      ctypes.c_int, ctypes.c_void_p,
+                                                      ctypes.c_void_p, ctypes.c_size_t,
+                                                      ctypes.c_void_p]),
     "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bitnet_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
 }
@@ -411,6 +427,84 @@ def bitnet_norm_bitlinear_forward(X, norm_gain, eps, hadamard, Wp, gamma, act_bi
                                         int(act_bits), Y.data_ptr(), ws.data_ptr(),
                                         ws.numel() * ws.element_size(), _stream(stream)),
         "bitnet_norm_bitlinear_forward")
+    return Y
+
+
+def bitnet_base3_weight_bytes(N: int, K: int) -> int:
+    return int(load_library().bitnet_base3_weight_bytes(N, K))
+
+
+def bitnet_quantize_pack_weights_base3(W: torch.Tensor, Wp3: torch.Tensor | None = None,
+                                       gamma: torch.Tensor | None = None,
+                                       ws: torch.Tensor | None = None, stream=None):
+    """absmean-ternarise bf16 W [N, K] into base-3 rows (five weights a byte).
+    Returns (Wp3 uint8 [N, 4 * ceil(K/20)], gamma float [1])."""
+    L = load_library()
+    _check(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    if Wp3 is None:
+        Wp3 = torch.empty((N, 4 * ((K + 19) // 20)), dtype=torch.uint8, device=W.device)
+    _nbytes_at_least(Wp3, int(L.bitnet_base3_weight_bytes(N, K)), "Wp3")
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    need = int(L.bitnet_weight_workspace_bytes(N, K))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    _rc(L.bitnet_quantize_pack_weights_base3(W.data_ptr(), N, K, Wp3.data_ptr(),
+                                             gamma.data_ptr(), ws.data_ptr(),
+                                             ws.numel() * ws.element_size(), _stream(stream)),
+        "bitnet_quantize_pack_weights_base3")
+    return Wp3, gamma
+
+
+def bitnet_ternary_gemv_base3(codes, scales, rowsum, K: int, Wp3, gamma, activation: int = 0,
+                              want_acc=False, want_y=True, acc=None, Y=None, stream=None):
+    """Product of INT8 codes (M <= 8 tokens) with base-3 weights Wp3 [N, 4 * ceil(K/20)].
+    Returns (acc int32 [M, N] or None, Y bf16 [M, N] ([M, N/2] for SwiGLU) or None)."""
+    L = load_library()
+    for t, n in ((codes, "codes"), (scales, "scales"), (rowsum, "rowsum"), (Wp3, "Wp3"),
+                 (gamma, "gamma")):
+        _check(t, n)
+    M = scales.numel()
+    N = Wp3.shape[0]
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, 8)), "codes")
+    _nbytes_at_least(rowsum, 4 * M, "rowsum")
+    _nbytes_at_least(Wp3, int(L.bitnet_base3_weight_bytes(N, K)), "Wp3")
+    if want_acc and acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=codes.device)
+    if want_y and Y is None:
+        Y = torch.empty((M, _act_cols(N, activation)), dtype=torch.bfloat16, device=codes.device)
+    if Y is not None:
+        _nbytes_at_least(Y, 2 * M * _act_cols(N, activation), "Y")
+    _rc(L.bitnet_ternary_gemv_base3(codes.data_ptr(), scales.data_ptr(), rowsum.data_ptr(), M, K,
+                                    Wp3.data_ptr(), gamma.data_ptr(), N, int(activation),
+                                    acc.data_ptr() if acc is not None else None,
+                                    Y.data_ptr() if Y is not None else None, _stream(stream)),
+        "bitnet_ternary_gemv_base3")
+    return acc, Y
+
+
+def bitnet_bitlinear_forward_base3(X, Wp3, gamma, hadamard: bool, activation: int = 0, Y=None,
+                                   ws=None, stream=None):
+    """Y = activation((H-)BitLinear(X)) for M <= 8 tokens on base-3 weights, INT8 activations."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    _check(Wp3, "Wp3")
+    _check(gamma, "gamma", torch.float32)
+    M, K = X.shape
+    N = Wp3.shape[0]
+    _nbytes_at_least(Wp3, int(L.bitnet_base3_weight_bytes(N, K)), "Wp3")
+    if Y is None:
+        Y = torch.empty((M, _act_cols(N, activation)), dtype=torch.bfloat16, device=X.device)
+    _nbytes_at_least(Y, 2 * M * _act_cols(N, activation), "Y")
+    need = int(L.bitnet_workspace_bytes(M, K, N, 8))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _rc(L.bitnet_bitlinear_forward_base3(X.data_ptr(), M, K, Wp3.data_ptr(), gamma.data_ptr(), N,
+                                         int(bool(hadamard)), int(activation), Y.data_ptr(),
+                                         ws.data_ptr(), ws.numel() * ws.element_size(),
+                                         _stream(stream)),
+        "bitnet_bitlinear_forward_base3")
     return Y
 
 

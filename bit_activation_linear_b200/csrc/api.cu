@@ -445,6 +445,124 @@ int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const voi
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t bitnet_base3_weight_bytes(int64_t N, int64_t K) {
+    return (N > 0 && K > 0) ? (size_t)N * (size_t)((K + 19) / 20) * 4 : 0;
+}
+
+int bitnet_quantize_pack_weights_base3(const void *W_dev, int64_t N, int64_t K, void *Wp3_dev,
+                                       float *gamma_dev, void *ws_dev, size_t ws_bytes,
+                                       bitnet_stream_t stream) {
+    int rc = check_shape(1, K, N, false, true);
+    if (rc) return rc;
+    if (!W_dev || !Wp3_dev || !gamma_dev || !ws_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(W_dev) || !aligned16(Wp3_dev) || !aligned16(ws_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    const size_t need = bitnet_weight_workspace_bytes(N, K);
+    if (ws_bytes < need)
+        return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    const int P = absmean_num_partials(N * K);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    double *partials = static_cast<double *>(ws_dev);
+    if ((rc = launched(launch_absmean_partials(W_dev, N * K, partials, P, s), 1,
+                       "absmean_partials")))
+        return rc;
+    return launched(launch_ternarize_pack_base3(W_dev, N, K, partials, P,
+                                                static_cast<uint32_t *>(Wp3_dev), gamma_dev, s),
+                    1, "ternarize_pack_base3");
+}
+
+}  // extern "C"
+
+namespace {
+int check_base3(int64_t M, int64_t K, int64_t N, int activation) {
+    int rc = check_shape(M, K, N, true, true);
+    if (rc) return rc;
+    if (M > kGemvMaxTokens)
+        return fail(BITNET_ERR_UNSUPPORTED, "base-3 weights serve M <= %d tokens, got M = %lld",
+                    kGemvMaxTokens, (long long)M);
+    if (activation != 0) return check_activation(activation, N);
+    return BITNET_OK;
+}
+
+int gemv_base3_impl(DeviceState *st, const void *codes, const float *scales,
+                    const int32_t *rowsum, int64_t M, int64_t K, const void *Wp3,
+                    const float *gamma, int64_t N, int activation, int32_t *acc, void *Y,
+                    bool early_weights, cudaStream_t stream) {
+    GemmArgs a;
+    a.codes = codes;
+    a.scales = scales;
+    a.rowsum = rowsum;
+    a.Wp = reinterpret_cast<const uint32_t *>(Wp3);
+    a.gamma = gamma;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.act_bits = 8;
+    a.acc = acc;
+    a.Y = Y;
+    a.status = st->status_word;
+    a.early_weights = early_weights;
+    a.activation = activation;
+    return launched(launch_ternary_gemv_base3(a, stream), 1, "ternary_gemv_base3");
+}
+}  // namespace
+
+extern "C" {
+
+int bitnet_ternary_gemv_base3(const void *codes_dev, const float *scales_dev,
+                              const int32_t *rowsum_dev, int64_t M, int64_t K,
+                              const void *Wp3_dev, const float *gamma_dev, int64_t N,
+                              int activation, int32_t *acc_dev, void *Y_dev,
+                              bitnet_stream_t stream) {
+    int rc = check_base3(M, K, N, activation);
+    if (rc) return rc;
+    if (!codes_dev || !scales_dev || !rowsum_dev || !Wp3_dev || !gamma_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!acc_dev && !Y_dev) return fail(BITNET_ERR_INVALID, "neither acc nor Y requested");
+    if (acc_dev && activation != 0)
+        return fail(BITNET_ERR_INVALID, "acc is the product before the activation: pass "
+                                        "activation 0 with acc");
+    if (!aligned16(codes_dev) || !aligned16(Wp3_dev) || (acc_dev && !aligned16(acc_dev)) ||
+        (Y_dev && !aligned16(Y_dev)))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    return gemv_base3_impl(st, codes_dev, scales_dev, rowsum_dev, M, K, Wp3_dev, gamma_dev, N,
+                           activation, acc_dev, Y_dev, false,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_bitlinear_forward_base3(const void *X_dev, int64_t M, int64_t K, const void *Wp3_dev,
+                                   const float *gamma_dev, int64_t N, int hadamard,
+                                   int activation, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                   bitnet_stream_t stream) {
+    int rc = check_base3(M, K, N, activation);
+    if (rc) return rc;
+    if (!X_dev || !Wp3_dev || !gamma_dev || !Y_dev || !ws_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(X_dev) || !aligned16(Wp3_dev) || !aligned16(Y_dev) || !aligned16(ws_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    const size_t need = bitnet_workspace_bytes(M, K, N, 8);
+    if (ws_bytes < need)
+        return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *w = static_cast<uint8_t *>(ws_dev);
+    float *scales = reinterpret_cast<float *>(w + round256(bitnet_act_codes_bytes(M, K, 8)));
+    int32_t *rowsum = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(scales) +
+                                                  round256((size_t)M * sizeof(float)));
+    if ((rc = act_quant_impl(st, X_dev, M, K, hadamard ? 1 : 0, 8, w, scales, rowsum, nullptr,
+                             s)))
+        return rc;
+    // the quantiser was launched in stream order after whatever wrote Wp3
+    return gemv_base3_impl(st, w, scales, rowsum, M, K, Wp3_dev, gamma_dev, N, activation,
+                           nullptr, Y_dev, true, s);
+}
+
 int bitnet_selftest_wait_timeout(int64_t limit_cycles, bitnet_stream_t stream) {
     if (limit_cycles < 1 || limit_cycles > kWaitLimitCycles)
         return fail(BITNET_ERR_INVALID, "limit_cycles = %lld must be in 1 .. %lld",

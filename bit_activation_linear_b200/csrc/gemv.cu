@@ -22,8 +22,55 @@ namespace bitnet {
 constexpr int kGemvSteps = 16;      // 512-weight steps whose weight loads are in flight together
 constexpr int kGemvWarps = 4;       // warps per CTA
 
-// ACT: 0 rescaled output, 1 squared ReLU of it, 2 SwiGLU over the warp's two rows (gate, up =
-// features 2j, 2j+1; output column j; needs R == 2).
+// Reduce the lanes' partial sums, remove the weight offset with the code sums and write the
+// results: lane r*T + t stores (row n0 + r, token t).  ACT: 0 rescaled output, 1 squared ReLU of
+// it, 2 SwiGLU over the warp's two rows (gate, up = features 2j, 2j+1; output column j; R == 2).
+template <int T, int R, int ACT>
+__device__ __forceinline__ void gemv_epilogue(const int (&acc)[R][T], int lane, int n0, int M,
+                                              int N, const float *__restrict__ scales,
+                                              const int32_t *__restrict__ rowsum, float gamma,
+                                              int32_t *__restrict__ acc_out,
+                                              __nv_bfloat16 *__restrict__ Y) {
+    static_assert(ACT != 2 || R == 2, "SwiGLU needs the gate and up rows in one warp");
+    int sums[R][T];  // full sums, the same in every lane
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            int s = acc[r][t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+            sums[r][t] = s;
+        }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        if (t >= M) break;
+        const float sc = scales[t] * gamma;
+        if constexpr (ACT == 2) {
+            if (lane == t && n0 + 1 < N) {
+                const float g = (float)(sums[0][t] - rowsum[t]) * sc;
+                const float u = (float)(sums[1][t] - rowsum[t]) * sc;
+                Y[(int64_t)t * (N / 2) + n0 / 2] = __float2bfloat16_rn(__fdiv_rn(g, 1.f + expf(-g)) * u);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int n = n0 + r;
+                if (lane == r * T + t && n < N) {
+                    const int a = sums[r][t] - rowsum[t];
+                    if (acc_out) acc_out[(int64_t)t * N + n] = a;
+                    if (Y) {
+                        float y = (float)a * sc;
+                        if constexpr (ACT == 1) y = y > 0.f ? y * y : 0.f;
+                        Y[(int64_t)t * N + n] = __float2bfloat16_rn(y);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// ACT as in gemv_epilogue.
 template <int BITS, int T, int R, int ACT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
@@ -93,44 +140,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
                 }
         }
     }
-    const float gamma = *gamma_ptr;
-    static_assert(ACT != 2 || R == 2, "SwiGLU needs the gate and up rows in one warp");
-    int sums[R][T];  // full sums, the same in every lane
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int t = 0; t < T; ++t) {
-            int s = acc[r][t];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-            sums[r][t] = s;
-        }
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-        if (t >= M) break;
-        const float sc = scales[t] * gamma;
-        if constexpr (ACT == 2) {
-            if (lane == t && n0 + 1 < N) {
-                const float g = (float)(sums[0][t] - rowsum[t]) * sc;
-                const float u = (float)(sums[1][t] - rowsum[t]) * sc;
-                Y[(int64_t)t * (N / 2) + n0 / 2] = __float2bfloat16_rn(__fdiv_rn(g, 1.f + expf(-g)) * u);
-            }
-        } else {
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int n = n0 + r;
-                if (lane == r * T + t && n < N) {
-                    const int a = sums[r][t] - rowsum[t];
-                    if (acc_out) acc_out[(int64_t)t * N + n] = a;
-                    if (Y) {
-                        float y = (float)a * sc;
-                        if constexpr (ACT == 1) y = y > 0.f ? y * y : 0.f;
-                        Y[(int64_t)t * N + n] = __float2bfloat16_rn(y);
-                    }
-                }
-            }
-        }
-    }
+    gemv_epilogue<T, R, ACT>(acc, lane, n0, M, N, scales, rowsum, *gamma_ptr, acc_out, Y);
 }
 
 template <int BITS, int T, int R, int ACT>
@@ -172,6 +182,130 @@ static cudaError_t launch_gemv_b(const GemmArgs &a, cudaStream_t stream) {
 cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream) {
     if (a.M > kGemvMaxTokens) return cudaErrorInvalidValue;
     return a.act_bits == 4 ? launch_gemv_b<4>(a, stream) : launch_gemv_b<8>(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------
+// Base-3 weights (2B4T article, section 一.1: five ternary weights in one byte, 1.6 bits a
+// weight).  Row n is ceil(K/20) 32-bit words; byte i of word w is the base-3 number of the offset
+// codes of weights 20w + 5i .. +4, first weight most significant.  A 256-entry table in shared
+// memory turns a byte into its five offset codes, one per byte of a 64-bit entry; the four entries
+// of a word are spliced into five dp4a words of four codes each, matching the 20 activation codes
+// k = 20w .. 20w + 19.  Same K walk as the 2-bit kernel with steps of 640 weights: lane l takes
+// word 32s + l of each row.  INT8 codes only (the 20-code groups do not fall on the 8-code
+// groups of the INT4 nibble layout).
+
+template <int T, int R, int ACT>
+__global__ void __launch_bounds__(kGemvWarps * 32)
+    ternary_gemv_base3_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
+                              const int32_t *__restrict__ rowsum, int M, int K,
+                              const uint32_t *__restrict__ wp3, const float *__restrict__ gamma_ptr,
+                              int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y,
+                              int early_weights) {
+    __shared__ unsigned long long digits[256];
+    for (int v = threadIdx.x; v < 256; v += kGemvWarps * 32) {
+        // byte 4 - j of the entry = base-3 digit j of v (digit 0 least significant); bytes
+        // 243..255 never occur in a stored row
+        unsigned long long e = 0;
+        int x = v;
+#pragma unroll
+        for (int b = 4; b >= 0; --b) {
+            e |= (unsigned long long)(x % 3) << (8 * b);
+            x /= 3;
+        }
+        digits[v] = e;
+    }
+    __syncthreads();
+    if (!early_weights) pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const int n0 = (blockIdx.x * kGemvWarps + (threadIdx.x >> 5)) * R;
+    if (n0 >= N) return;  // whole warp leaves together (after the block's only barrier)
+    const int words = (K + 19) / 20;
+    const int steps = (words + 31) / 32;
+    int acc[R][T];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int t = 0; t < T; ++t) acc[r][t] = 0;
+
+    for (int s0 = 0; s0 < steps; s0 += kGemvSteps) {
+        uint32_t w[R][kGemvSteps];
+#pragma unroll
+        for (int j = 0; j < kGemvSteps; ++j)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+                w[r][j] = (32 * (s0 + j) + lane < words && n0 + r < N)
+                              ? __ldg(wp3 + (int64_t)(n0 + r) * words + 32 * (s0 + j) + lane)
+                              : 0u;  // byte 0 decodes to u = 0: adds nothing
+        if (early_weights && s0 == 0) pdl_wait();
+#pragma unroll
+        for (int j = 0; j < kGemvSteps; ++j) {
+            if (s0 + j >= steps) break;
+            const int k0 = 20 * (32 * (s0 + j) + lane);
+            // codes k0 + 4p .. +3 of every token (K % 4 == 0: a group is wholly in or out)
+            uint32_t xs[T][5];
+#pragma unroll
+            for (int t = 0; t < T; ++t)
+#pragma unroll
+                for (int p = 0; p < 5; ++p)
+                    xs[t][p] = (t < M && k0 + 4 * p < K)
+                                   ? __ldg(reinterpret_cast<const uint32_t *>(
+                                         codes + (int64_t)t * K + k0 + 4 * p))
+                                   : 0u;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const uint32_t v = w[r][j];
+                const unsigned long long L0 = digits[v & 0xFFu], L1 = digits[(v >> 8) & 0xFFu],
+                                         L2 = digits[(v >> 16) & 0xFFu], L3 = digits[v >> 24];
+                // offset codes of weights k0 .. k0+19, four per word in k order
+                const uint32_t u[5] = {(uint32_t)L0,
+                                       (uint32_t)(L0 >> 32) | (uint32_t)(L1 << 8),
+                                       (uint32_t)(L1 >> 24) | (uint32_t)(L2 << 16),
+                                       (uint32_t)(L2 >> 16) | (uint32_t)(L3 << 24),
+                                       (uint32_t)(L3 >> 8)};
+#pragma unroll
+                for (int p = 0; p < 5; ++p)
+#pragma unroll
+                    for (int t = 0; t < T; ++t)
+                        acc[r][t] = __dp4a((int)u[p], (int)xs[t][p], acc[r][t]);
+            }
+        }
+    }
+    gemv_epilogue<T, R, ACT>(acc, lane, n0, M, N, scales, rowsum, *gamma_ptr, acc_out, Y);
+}
+
+template <int T, int R, int ACT>
+static cudaError_t launch_gemv3_t(const GemmArgs &a, cudaStream_t stream) {
+    static_assert(R * T <= 32, "one lane per (row, token) result");
+    const int64_t warps = (a.N + R - 1) / R;
+    const unsigned blocks = (unsigned)((warps + kGemvWarps - 1) / kGemvWarps);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ternary_gemv_base3_kernel<T, R, ACT>,
+                              reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum,
+                              (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
+                              reinterpret_cast<__nv_bfloat16 *>(a.Y), a.early_weights ? 1 : 0);
+}
+
+template <int ACT>
+static cudaError_t launch_gemv3_a(const GemmArgs &a, cudaStream_t stream) {
+    constexpr int R_SMALL = ACT == 2 ? 2 : 1;
+    if (a.M <= 1) return launch_gemv3_t<1, R_SMALL, ACT>(a, stream);
+    if (a.M <= 2) return launch_gemv3_t<2, R_SMALL, ACT>(a, stream);
+    if (a.M <= 4) return launch_gemv3_t<4, 2, ACT>(a, stream);
+    return launch_gemv3_t<8, 2, ACT>(a, stream);
+}
+
+cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream) {
+    if (a.M > kGemvMaxTokens || a.act_bits != 8) return cudaErrorInvalidValue;
+    if (a.acc || a.activation == 0) return launch_gemv3_a<0>(a, stream);
+    return a.activation == 1 ? launch_gemv3_a<1>(a, stream) : launch_gemv3_a<2>(a, stream);
 }
 
 }  // namespace bitnet

@@ -14,6 +14,10 @@ cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, 
                                     cudaStream_t stream);
 cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partials, int P,
                                   uint32_t *Wp, float *gamma, cudaStream_t stream);
+// Base-3 rows (five weights per byte, ceil(K/20) 32-bit words per row) for the decode product.
+cudaError_t launch_ternarize_pack_base3(const void *W, int64_t N, int64_t K,
+                                        const double *partials, int P, uint32_t *Wp3,
+                                        float *gamma, cudaStream_t stream);
 // Device address (current device) and size of the library's fixed partial-sum scratch.
 cudaError_t noalloc_partials_address(double **ptr, size_t *bytes);
 
@@ -59,6 +63,10 @@ struct GemmArgs {
 // Weight-streaming kernel for few tokens (decode).
 constexpr int kGemvMaxTokens = 8;
 cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream);
+
+// Weight-streaming kernel on base-3 rows (INT8 codes, M <= kGemvMaxTokens); a.Wp points at the
+// base-3 words.
+cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream);
 
 // tcgen05 tensor-core kernel (prefill).  encode is cuTensorMapEncodeTiled.
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,

@@ -93,6 +93,35 @@ __device__ __forceinline__ uint32_t ternary_threshold_bits(float gamma) {
     return h;
 }
 
+// gamma from the P partial sums, then its decision threshold; every block computes it the same
+// way (a fixed assignment of partials to threads and a fixed reduction tree), so gamma does not
+// depend on the launch.  Block 0 writes gamma.  Contains __syncthreads.
+__device__ __forceinline__ uint32_t block_threshold(const double *__restrict__ partials, int P,
+                                                    double n_weights, float *__restrict__ gamma_out) {
+    __shared__ double warp_sums[kWeightThreads / 32];
+    __shared__ uint32_t s_thr;
+    double s = 0.0;
+    for (int j = threadIdx.x; j < P; j += kWeightThreads) s += partials[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
+        const float g = (float)fmax(t / n_weights, 1e-5);
+        s_thr = ternary_threshold_bits(g);
+        if (blockIdx.x == 0) *gamma_out = g;
+    }
+    __syncthreads();
+    return s_thr;
+}
+
+// Offset code u = q + 1 of one bf16 weight against the threshold (see ternary_threshold_bits).
+__device__ __forceinline__ uint32_t offset_code(uint32_t bits, uint32_t thr) {
+    return (bits & 0x7FFFu) >= thr ? ((bits & 0x8000u) ? 0u : 2u) : 1u;
+}
+
 __global__ void __launch_bounds__(kWeightThreads)
     ternarize_pack_kernel(const uint4 *__restrict__ w, int64_t nwords, double n_weights,
                           const double *__restrict__ partials, int P, uint32_t *__restrict__ wp,
@@ -105,27 +134,7 @@ __global__ void __launch_bounds__(kWeightThreads)
         a = ldg_nc_v4(w + 2 * i);
         b = ldg_nc_v4(w + 2 * i + 1);
     }
-    // gamma from the P partial sums: a fixed assignment of partials to threads and a fixed
-    // reduction tree, identical in every block, so gamma does not depend on the launch
-    __shared__ double warp_sums[kWeightThreads / 32];
-    __shared__ uint32_t s_thr;
-    {
-        double s = 0.0;
-        for (int j = threadIdx.x; j < P; j += kWeightThreads) s += partials[j];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-        if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double t = 0.0;
-            for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
-            const float g = (float)fmax(t / n_weights, 1e-5);
-            s_thr = ternary_threshold_bits(g);
-            if (blockIdx.x == 0) *gamma_out = g;
-        }
-        __syncthreads();
-    }
-    const uint32_t thr = s_thr;
+    const uint32_t thr = block_threshold(partials, P, n_weights, gamma_out);
     const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
     for (bool first = true; i < nwords; i += stride, first = false) {
         // 16 consecutive weights k = 16i + e; weight e = 4p + j goes to bits 8j + 2p as u = q + 1.
@@ -138,11 +147,72 @@ __global__ void __launch_bounds__(kWeightThreads)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const uint32_t bits = (e & 1) ? (h[e >> 1] >> 16) : (h[e >> 1] & 0xFFFFu);
-            const uint32_t u = (bits & 0x7FFFu) >= thr ? ((bits & 0x8000u) ? 0u : 2u) : 1u;
+            const uint32_t u = offset_code(bits, thr);
             word |= u << (8 * (e & 3) + 2 * (e >> 2));
         }
         wp[i] = word;
     }
+}
+
+// Base-3 storage for the decode product (2B4T article, section 一.1: five ternary weights in one
+// byte): row n is ceil(K/20) 32-bit words; byte i of word w holds the offset codes of weights
+// k = 20w + 5i .. +4 as the base-3 number u0*81 + u1*27 + u2*9 + u3*3 + u4 (first weight most
+// significant); weights k >= K are stored as u = 1.  The decisions are those of
+// ternarize_pack_kernel (same gamma, same threshold).  One thread per word.
+__global__ void __launch_bounds__(kWeightThreads)
+    ternarize_pack_base3_kernel(const uint16_t *__restrict__ w, int64_t N, int64_t K,
+                                double n_weights, const double *__restrict__ partials, int P,
+                                uint32_t *__restrict__ wp3, float *__restrict__ gamma_out) {
+    const int64_t words = (K + 19) / 20;
+    const int64_t total = N * words;
+    const uint32_t thr = block_threshold(partials, P, n_weights, gamma_out);
+    const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < total; i += stride) {
+        const int64_t n = i / words, wd = i - n * words;
+        const int64_t k0 = 20 * wd;
+        const uint16_t *src = w + n * K + k0;
+        uint32_t h[20];
+        if (k0 + 20 <= K) {
+            // 40 bytes at an 8-byte-aligned address (K % 128 == 0)
+#pragma unroll
+            for (int j = 0; j < 5; ++j) {
+                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src) + j);
+                h[4 * j] = v.x & 0xFFFFu;
+                h[4 * j + 1] = v.x >> 16;
+                h[4 * j + 2] = v.y & 0xFFFFu;
+                h[4 * j + 3] = v.y >> 16;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 20; ++e) h[e] = k0 + e < K ? (uint32_t)__ldg(src + e) : 0u;
+        }
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int t = 0; t < 5; ++t) {
+                const int e = 5 * b + t;
+                const uint32_t u = k0 + e < K ? offset_code(h[e], thr) : 1u;
+                v = v * 3u + u;
+            }
+            word |= v << (8 * b);
+        }
+        wp3[i] = word;
+    }
+}
+
+cudaError_t launch_ternarize_pack_base3(const void *W, int64_t N, int64_t K,
+                                        const double *partials, int P, uint32_t *Wp3,
+                                        float *gamma, cudaStream_t stream) {
+    const int64_t total = N * ((K + 19) / 20);
+    int64_t blocks = (total + kWeightThreads - 1) / kWeightThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    ternarize_pack_base3_kernel<<<(unsigned)blocks, kWeightThreads, 0, stream>>>(
+        reinterpret_cast<const uint16_t *>(W), N, K, (double)N * (double)K, partials, P, Wp3,
+        gamma);
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------------

@@ -227,6 +227,57 @@ int bitnet_bitlinear_forward_act(const void *X_dev, int64_t M, int64_t K, const 
                                  bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* Base-3 weights for decode                                                                */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * Five ternary weights in one byte (BitNet b1.58 2B4T article, section 一.1: 3^5 = 243 <= 256,
+ * 1.6 bits a weight instead of 2), for the weight-streaming product of a few tokens, which is
+ * bound by the bytes of weights it reads.
+ * Layout: row n is ceil(K/20) little-endian 32-bit words; byte i (0..3) of word w holds the
+ * offset codes u = q + 1 of weights k = 20w + 5i .. 20w + 5i + 4 as the base-3 number
+ * u0*81 + u1*27 + u2*9 + u3*3 + u4, the first weight most significant (the article's example:
+ * codes 2,0,1,2,1 -> byte 178).  Weights k >= K (the last word of a row) are stored as u = 1.
+ */
+
+/* Bytes of base-3 weights for an [N, K] matrix: N * 4 * ceil(K / 20). */
+size_t bitnet_base3_weight_bytes(int64_t N, int64_t K);
+
+/*
+ * absmean ternarisation exactly as bitnet_quantize_pack_weights (same gamma, same q for every
+ * weight), stored in the base-3 layout above.  Wp3_dev out: bitnet_base3_weight_bytes(N, K)
+ * bytes; other arguments, shapes and errors as bitnet_quantize_pack_weights.
+ */
+int bitnet_quantize_pack_weights_base3(const void *W_dev, int64_t N, int64_t K, void *Wp3_dev,
+                                       float *gamma_dev, void *ws_dev, size_t ws_bytes,
+                                       bitnet_stream_t stream);
+
+/*
+ * The product of bitnet_ternary_gemm / bitnet_ternary_gemm_act on base-3 weights, for
+ * M <= 8 tokens (else BITNET_ERR_UNSUPPORTED) and INT8 codes (as written by bitnet_act_quant
+ * with act_bits 8).  activation: 0 (none), BITNET_ACT_RELU2 or BITNET_ACT_SWIGLU, with the
+ * outputs of bitnet_ternary_gemm_act; acc_dev (int32 [M, N], exact) only with activation 0.
+ * acc_dev and Y_dev are each optional; at least one must be given.  A byte above 242 in Wp3 is
+ * not a valid store and gives unspecified (but in-bounds) results.
+ */
+int bitnet_ternary_gemv_base3(const void *codes_dev, const float *scales_dev,
+                              const int32_t *rowsum_dev, int64_t M, int64_t K,
+                              const void *Wp3_dev, const float *gamma_dev, int64_t N,
+                              int activation, int32_t *acc_dev, void *Y_dev,
+                              bitnet_stream_t stream);
+
+/*
+ * The whole layer on base-3 weights for M <= 8 tokens: INT8 per-token quantisation (with the
+ * online Hadamard transform when hadamard != 0, as bitnet_hbitlinear_forward), then
+ * bitnet_ternary_gemv_base3 with the given activation (0 for none) into Y_dev (bf16 [M, N], or
+ * [M, N/2] for SwiGLU).  ws_dev: ws_bytes >= bitnet_workspace_bytes(M, K, N, 8).
+ */
+int bitnet_bitlinear_forward_base3(const void *X_dev, int64_t M, int64_t K, const void *Wp3_dev,
+                                   const float *gamma_dev, int64_t N, int hadamard,
+                                   int activation, void *Y_dev, void *ws_dev, size_t ws_bytes,
+                                   bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* Status                                                                                   */
 /* ---------------------------------------------------------------------------------------- */
 

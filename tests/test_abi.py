@@ -125,3 +125,24 @@ def test_activation_entries_reject_bad_arguments_before_the_device(lib):
     assert rc == -1
     rc = lib.bitnet_bitlinear_forward_act(p, 8, 256, p, p, 264, 8, 0, 2, p, p, 1 << 20, None)
     assert rc == -1
+
+
+def test_base3_entries_size_and_rejections_before_the_device(lib):
+    # five weights a byte, rows of ceil(K/20) 32-bit words
+    assert lib.bitnet_base3_weight_bytes(2048, 2048) == 2048 * 4 * 103
+    assert lib.bitnet_base3_weight_bytes(8, 640) == 8 * 4 * 32
+    assert lib.bitnet_base3_weight_bytes(0, 640) == 0
+    p = ctypes.c_void_p(16)
+    # more than 8 tokens: unsupported (the tensor-core product takes the 2-bit layout)
+    assert lib.bitnet_ternary_gemv_base3(p, p, p, 9, 256, p, p, 256, 0, None, p, None) == -2
+    assert lib.bitnet_bitlinear_forward_base3(p, 9, 256, p, p, 256, 0, 0, p, p, 1 << 20,
+                                              None) == -2
+    # unknown activation; an activation together with the int32 product; neither output
+    assert lib.bitnet_ternary_gemv_base3(p, p, p, 4, 256, p, p, 256, 3, None, p, None) == -1
+    assert lib.bitnet_ternary_gemv_base3(p, p, p, 4, 256, p, p, 256, 1, p, p, None) == -1
+    assert lib.bitnet_ternary_gemv_base3(p, p, p, 4, 256, p, p, 256, 0, None, None, None) == -1
+    # K not a multiple of 128; misaligned weights
+    assert lib.bitnet_ternary_gemv_base3(p, p, p, 4, 200, p, p, 256, 0, None, p, None) == -1
+    q = ctypes.c_void_p(20)
+    assert lib.bitnet_quantize_pack_weights_base3(p, 256, 256, q, p, p, 1 << 20, None) == -1
+    assert lib.bitnet_quantize_pack_weights_base3(p, 256, 256, p, p, p, 0, None) == -5

@@ -383,3 +383,105 @@ def test_forward_activation_end_to_end(B, name, act):
     y_ref = oracle.bf16_to_f64(oracle.dequant_act(ref["acc"], ref["d"], ref["gamma"], act))
     y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
     assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
+
+
+# ----------------------------------------------------------------------------------------
+# base-3 weights for decode (2B4T article, section 一.1: five ternary weights a byte)
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(256, 256), (8, 128), (264, 384), (16, 640), (2048, 2048),
+                                 (520, 8192), (8, 32768)])
+def test_base3_weights_bit_exact(B, N, K):
+    W = synth.latent_weights(N, K, seed=N + 2 * K)
+    Wp3, gamma = B.bitnet_quantize_pack_weights_base3(dev_bf16(W))
+    B.bitnet_sync_status()
+    g_ref = oracle.absmean_gamma(W)
+    assert np.float32(gamma.item()) == g_ref
+    words = (K + 19) // 20
+    ref = oracle.pack_ternary_base3(oracle.ternarize(W, g_ref))
+    got = Wp3.cpu().numpy().view(np.uint32).reshape(N, words)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_base3_weights_degenerate(B):
+    # all-zero weights: gamma = 1e-5, every weight q = 0 (u = 1), padding too: byte 121
+    Z = np.zeros((16, 128), np.uint16)
+    Wp3, gamma = B.bitnet_quantize_pack_weights_base3(dev_bf16(Z))
+    B.bitnet_sync_status()
+    assert np.float32(gamma.item()) == np.float32(1e-5)
+    assert np.all(Wp3.cpu().numpy() == 121)
+
+
+@pytest.mark.parametrize("M,K,N", [
+    (1, 128, 8), (1, 2048, 264), (2, 384, 136), (3, 640, 256), (4, 8192, 520),
+    (5, 256, 8), (8, 2048, 1032), (8, 32768, 16),
+])
+def test_base3_product_int32_exact_and_bf16(B, M, K, N):
+    X = synth.sharp_activations(M, K, seed=M * 3 + K)
+    W = synth.latent_weights(N, K, seed=N + 5)
+    Wp3, gamma = B.bitnet_quantize_pack_weights_base3(dev_bf16(W))
+    hadamard = (K & (K - 1)) == 0
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), hadamard, 8)
+    acc, Y = B.bitnet_ternary_gemv_base3(codes, scales, rowsum, K, Wp3, gamma, want_acc=True)
+    B.bitnet_sync_status()
+    c = codes.cpu().numpy().view(np.int8)
+    q, bad = oracle.unpack_ternary_base3(Wp3.cpu().numpy().view(np.uint32), K)
+    assert bad == 0
+    np.testing.assert_array_equal(q, oracle.ternarize(W, oracle.absmean_gamma(W)))
+    acc_ref = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(acc.cpu().numpy().astype(np.int64), acc_ref)
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc_ref, scales.cpu().numpy(),
+                                              np.float32(gamma.item())))
+    y = oracle.bf16_to_f64(to_np_bits(Y))
+    rel = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), 1e-30)
+    assert np.all((rel <= Y_REL) | (y_ref == 0)), rel.max()
+    assert np.all(y[y_ref == 0] == 0)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 2048, 272), (4, 640, 528), (8, 8192, 1040)])
+@pytest.mark.parametrize("act", [1, 2])
+def test_base3_product_activation_matches_oracle(B, M, K, N, act):
+    X = synth.sharp_activations(M, K, seed=M + 2 * K)
+    W = synth.latent_weights(N, K, seed=N + 7)
+    Wp3, gamma = B.bitnet_quantize_pack_weights_base3(dev_bf16(W))
+    hadamard = (K & (K - 1)) == 0
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), hadamard, 8)
+    _, Y = B.bitnet_ternary_gemv_base3(codes, scales, rowsum, K, Wp3, gamma, act)
+    B.bitnet_sync_status()
+    q = oracle.ternarize(W, oracle.absmean_gamma(W))
+    acc_ref = oracle.gemm_i64(codes.cpu().numpy().view(np.int8), q)
+    check_act(Y, oracle.dequant_act(acc_ref, scales.cpu().numpy(), np.float32(gamma.item()), act))
+
+
+@pytest.mark.parametrize("name,act", [("decode_m1_k8192", 0), ("decode_m8_k8192", 0),
+                                      ("decode_m1_k2048", 0), ("decode_m8_k2048", 2),
+                                      ("decode_m1_k8192", 1)])
+def test_base3_forward_end_to_end(B, name, act):
+    wl = synth.WORKLOADS[name]
+    assert wl.act_bits == 8
+    X, W = wl.activations(seed=4), wl.weights(seed=4)
+    Wp3, gamma = B.bitnet_quantize_pack_weights_base3(dev_bf16(W))
+    Y = B.bitnet_bitlinear_forward_base3(dev_bf16(X), Wp3, gamma, wl.hadamard, act)
+    B.bitnet_sync_status()
+    ref = oracle.bitlinear_forward(X, W, wl.hadamard, 8)
+    assert np.float32(gamma.item()) == ref["gamma"]
+    y_ref = ref["y"] if act == 0 else oracle.dequant_act(ref["acc"], ref["d"], ref["gamma"], act)
+    y_ref = oracle.bf16_to_f64(y_ref)
+    y = oracle.bf16_to_f64(to_np_bits(Y))
+    assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
+
+
+def test_base3_product_equals_two_bit_product(B):
+    # the same ternary matrix in both layouts gives the same integers and the same bf16 outputs
+    M, K, N = 8, 4096, 776
+    X = synth.sharp_activations(M, K, seed=11)
+    W = dev_bf16(synth.latent_weights(N, K, seed=12))
+    Wp, g2 = B.bitnet_quantize_pack_weights(W)
+    Wp3, g3 = B.bitnet_quantize_pack_weights_base3(W)
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), True, 8)
+    a2, y2 = B.bitnet_ternary_gemm(codes, scales, rowsum, K, Wp, g2, 8, want_acc=True)
+    a3, y3 = B.bitnet_ternary_gemv_base3(codes, scales, rowsum, K, Wp3, g3, want_acc=True)
+    B.bitnet_sync_status()
+    assert g2.item() == g3.item()
+    assert torch.equal(a2, a3)
+    assert torch.equal(y2.view(torch.int16), y3.view(torch.int16))

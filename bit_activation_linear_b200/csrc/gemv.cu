@@ -1,5 +1,5 @@
 // gemv.cu -- step 4 for a handful of tokens (decode): the ternary x integer product streamed
-// straight from the packed weights, bound by HBM bandwidth on the 2-bit weight stream.
+// straight from the packed weights, bound by HBM bandwidth on the weight stream.
 //
 // 2B4T article, section 一.2: with ternary weights the matrix product is additions and
 // subtractions only.  Here the weights stay as the stored offset codes u = q + 1 in {0,1,2}:
@@ -7,31 +7,41 @@
 // the matching four activation codes accumulates sum_k u * c exactly; the per-token code sum
 // written by the quantiser removes the offset: sum_k q * c = sum_k u * c - sum_k c.
 //
-// A warp owns R consecutive output features (R = 2 from four tokens up, so that each code load
-// serves two rows).  The K axis is walked in steps of 512 weights: in a step lane l takes the
+// A row group of R consecutive output features is owned by KS warps of one CTA (KS = 1, 2 or 4:
+// when a matrix has few row groups, long rows are split so that it still fills the GPU).  The K axis is walked
+// in steps of 512 weights, step s going to warp s mod KS of the group: in a step lane l takes the
 // packed word 32s + l of each row (weights k = 512s + 16l .. +15, one coalesced 128-byte load per
 // warp and row) and the 16 matching codes of each token (one coalesced 16-byte load per lane).
-// The weight words of eight steps are loaded before any is used, so every warp keeps 8R loads
-// in flight and the weight stream is requested at full rate.  Activation codes (at most eight
-// tokens) are read through L1, where every warp of the SM finds them.
+// The weight words of S steps are loaded before any is used, so every warp keeps S*R loads in
+// flight and the weight stream is requested at full rate.  Every code is loaded once per R rows,
+// so R grows with the token count (1 row for 1-2 tokens, 2 for 3-8; 4 for 5-8 tokens when
+// N >= 8192) to keep the L1 traffic of the code loads down.  Activation codes (at most eight tokens) are read
+// through L1, where every warp of the SM finds them.  The lanes' partial sums are reduced with
+// shuffles, then across the group's warps through shared memory, and the group's first warp
+// writes the results.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace bitnet {
 
-constexpr int kGemvSteps = 16;      // 512-weight steps whose weight loads are in flight together
-constexpr int kGemvWarps = 4;       // warps per CTA
+constexpr int kGemvWarps = 4;  // warps per CTA
 
-// Reduce the lanes' partial sums, remove the weight offset with the code sums and write the
-// results: lane r*T + t stores (row n0 + r, token t).  ACT: 0 rescaled output, 1 squared ReLU of
-// it, 2 SwiGLU over the warp's two rows (gate, up = features 2j, 2j+1; output column j; R == 2).
-template <int T, int R, int ACT>
-__device__ __forceinline__ void gemv_epilogue(const int (&acc)[R][T], int lane, int n0, int M,
-                                              int N, const float *__restrict__ scales,
-                                              const int32_t *__restrict__ rowsum, float gamma,
-                                              int32_t *__restrict__ acc_out,
-                                              __nv_bfloat16 *__restrict__ Y) {
-    static_assert(ACT != 2 || R == 2, "SwiGLU needs the gate and up rows in one warp");
+// Reduce the lanes' partial sums (shuffles), then the KS warps' partial sums of the row group
+// (shared memory, one barrier for the whole CTA), remove the weight offset with the code sums and
+// write the results from the group's first warp: lane r*T + t stores (row n0 + r, token t).
+// ACT: 0 rescaled output, 1 squared ReLU of it, 2 SwiGLU over row pairs (gate, up = features
+// 2j, 2j+1 = rows n0 + 2p, n0 + 2p + 1; output column j = n0/2 + p, written by lane p*T + t).
+// Every thread of the CTA must call it (it contains __syncthreads when KS > 1).
+template <int T, int R, int KS, int ACT>
+__device__ __forceinline__ void gemv_finish(const int (&acc)[R][T], int (*red)[R * T],
+                                            bool active, int lane, int n0, int M, int N,
+                                            const float *__restrict__ scales,
+                                            const int32_t *__restrict__ rowsum,
+                                            const float *__restrict__ gamma_ptr,
+                                            int32_t *__restrict__ acc_out,
+                                            __nv_bfloat16 *__restrict__ Y) {
+    static_assert(ACT != 2 || R % 2 == 0, "SwiGLU needs the gate and up rows in one group");
+    const int warp = threadIdx.x >> 5;
     int sums[R][T];  // full sums, the same in every lane
 #pragma unroll
     for (int r = 0; r < R; ++r)
@@ -42,15 +52,39 @@ __device__ __forceinline__ void gemv_epilogue(const int (&acc)[R][T], int lane, 
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
             sums[r][t] = s;
         }
+    if constexpr (KS > 1) {
+        if (lane == 0)
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int t = 0; t < T; ++t) red[warp][r * T + t] = sums[r][t];
+        __syncthreads();
+        if (warp % KS != 0) return;
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+                int s = sums[r][t];
+#pragma unroll
+                for (int w = 1; w < KS; ++w) s += red[warp + w][r * T + t];
+                sums[r][t] = s;
+            }
+    }
+    if (!active) return;
+    const float gamma = *gamma_ptr;
 #pragma unroll
     for (int t = 0; t < T; ++t) {
         if (t >= M) break;
         const float sc = scales[t] * gamma;
         if constexpr (ACT == 2) {
-            if (lane == t && n0 + 1 < N) {
-                const float g = (float)(sums[0][t] - rowsum[t]) * sc;
-                const float u = (float)(sums[1][t] - rowsum[t]) * sc;
-                Y[(int64_t)t * (N / 2) + n0 / 2] = __float2bfloat16_rn(__fdiv_rn(g, 1.f + expf(-g)) * u);
+#pragma unroll
+            for (int p = 0; p < R / 2; ++p) {
+                if (lane == p * T + t && n0 + 2 * p + 1 < N) {
+                    const float g = (float)(sums[2 * p][t] - rowsum[t]) * sc;
+                    const float u = (float)(sums[2 * p + 1][t] - rowsum[t]) * sc;
+                    Y[(int64_t)t * (N / 2) + n0 / 2 + p] =
+                        __float2bfloat16_rn(__fdiv_rn(g, 1.f + expf(-g)) * u);
+                }
             }
         } else {
 #pragma unroll
@@ -70,46 +104,58 @@ __device__ __forceinline__ void gemv_epilogue(const int (&acc)[R][T], int lane, 
     }
 }
 
-// ACT as in gemv_epilogue.
-template <int BITS, int T, int R, int ACT>
+// Warps per row group.  With 1024 or more row groups the GPU has enough warps and a split only
+// adds CTAs and a barrier (measured slower); with fewer, long rows are split so that every warp
+// still walks at least ~4 steps.
+static int gemv_split(int64_t groups, int steps) {
+    if (groups >= 1024) return 1;
+    return steps >= 16 ? 4 : steps >= 8 ? 2 : 1;
+}
+
+// ACT as in gemv_finish; S = steps whose weight loads are in flight together.
+template <int BITS, int T, int R, int S, int KS, int ACT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                         const int32_t *__restrict__ rowsum, int M, int K,
                         const uint32_t *__restrict__ wp, const float *__restrict__ gamma_ptr,
                         int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y,
                         int early_weights) {
+    __shared__ int red[kGemvWarps][R * T];
     if (!early_weights) pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int n0 = (blockIdx.x * kGemvWarps + (threadIdx.x >> 5)) * R;
-    if (n0 >= N) return;  // whole warp leaves together (nothing of its own to wait for)
-    const int words = K / 16;  // packed words per row
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ks = warp % KS;
+    const int n0 = (blockIdx.x * (kGemvWarps / KS) + warp / KS) * R;
+    const bool active = n0 < N;
+    const int words = K / 16;             // packed words per row
     const int steps = (words + 31) / 32;  // the last step may be partial (K % 512 != 0)
+    const int mine = active && steps > ks ? (steps - ks + KS - 1) / KS : 0;  // this warp's steps
     int acc[R][T];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < T; ++t) acc[r][t] = 0;
 
-    for (int s0 = 0; s0 < steps; s0 += kGemvSteps) {
-        uint32_t w[R][kGemvSteps];
+    for (int b0 = 0; b0 < mine; b0 += S) {
+        uint32_t w[R][S];
 #pragma unroll
-        for (int j = 0; j < kGemvSteps; ++j)
+        for (int j = 0; j < S; ++j) {
+            const int wi = 32 * (ks + KS * (b0 + j)) + lane;
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                w[r][j] = (32 * (s0 + j) + lane < words && n0 + r < N)
-                              ? __ldg(wp + (int64_t)(n0 + r) * words + 32 * (s0 + j) + lane)
+                w[r][j] = (b0 + j < mine && wi < words && n0 + r < N)
+                              ? __ldg(wp + (int64_t)(n0 + r) * words + wi)
                               : 0u;
+        }
         // With early_weights the packed weights were complete before the kernel that wrote the
         // codes started, so they are loaded before waiting for that kernel (programmatic
         // dependent launch); the codes, scales and code sums are always read after the wait.
-        if (early_weights && s0 == 0) pdl_wait();
+        if (early_weights && b0 == 0) pdl_wait();
 #pragma unroll
-        for (int j = 0; j < kGemvSteps; ++j) {
-            if (s0 + j >= steps) break;
-            const int k0 = 512 * (s0 + j) + 16 * lane;
+        for (int j = 0; j < S; ++j) {
+            if (b0 + j >= mine) break;
+            const int k0 = 512 * (ks + KS * (b0 + j)) + 16 * lane;
             const bool k_in = k0 < K;  // lanes past the end of a partial step add zero
-            // codes k0 .. k0+15 of every token as four words of four int8 (word p = k0+4p .. +3),
-            // all loaded before the dot products (tokens t >= M read nothing and add zero)
+            // codes k0 .. k0+15 of every token as four words of four int8 (word p = k0+4p .. +3)
             uint32_t xs[T][4];
 #pragma unroll
             for (int t = 0; t < T; ++t) {
@@ -140,16 +186,19 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
                 }
         }
     }
-    gemv_epilogue<T, R, ACT>(acc, lane, n0, M, N, scales, rowsum, *gamma_ptr, acc_out, Y);
+    // the scales and code sums are read below: make sure this warp has waited
+    if (early_weights && mine == 0) pdl_wait();
+    gemv_finish<T, R, KS, ACT>(acc, red, active, lane, n0, M, N, scales, rowsum, gamma_ptr,
+                               acc_out, Y);
 }
 
-template <int BITS, int T, int R, int ACT>
-static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
-    static_assert(R * T <= 32, "one lane per (row, token) result");
-    const int64_t warps = (a.N + R - 1) / R;
-    const unsigned blocks = (unsigned)((warps + kGemvWarps - 1) / kGemvWarps);
+// CTAs of kGemvWarps warps, row groups of R rows owned by KS warps each.
+template <int R, int KS, typename Kern>
+static cudaError_t launch_gemv_kernel(Kern kern, const GemmArgs &a, cudaStream_t stream) {
+    const int64_t groups = (a.N + R - 1) / R;
+    constexpr int per_cta = kGemvWarps / KS;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks, 1, 1);
+    cfg.gridDim = dim3((unsigned)((groups + per_cta - 1) / per_cta), 1, 1);
     cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -157,19 +206,31 @@ static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ternary_gemv_kernel<BITS, T, R, ACT>,
-                              reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum,
-                              (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
+    return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const uint8_t *>(a.codes), a.scales,
+                              a.rowsum, (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
                               reinterpret_cast<__nv_bfloat16 *>(a.Y), a.early_weights ? 1 : 0);
 }
 
+template <int BITS, int T, int R, int S, int ACT>
+static cudaError_t launch_gemv_t(const GemmArgs &a, cudaStream_t stream) {
+    static_assert(R * T <= 32, "one lane per (row, token) result");
+    switch (gemv_split((a.N + R - 1) / R, (int)((a.K / 16 + 31) / 32))) {
+        case 4: return launch_gemv_kernel<R, 4>(ternary_gemv_kernel<BITS, T, R, S, 4, ACT>, a, stream);
+        case 2: return launch_gemv_kernel<R, 2>(ternary_gemv_kernel<BITS, T, R, S, 2, ACT>, a, stream);
+        default: return launch_gemv_kernel<R, 1>(ternary_gemv_kernel<BITS, T, R, S, 1, ACT>, a, stream);
+    }
+}
+
+// Rows per group by token count: the codes of T tokens are loaded once per R rows.  Four rows
+// per group only from N = 8192 up, where the groups still give every SM many warps.
 template <int BITS, int ACT>
 static cudaError_t launch_gemv_a(const GemmArgs &a, cudaStream_t stream) {
-    constexpr int R_SMALL = ACT == 2 ? 2 : 1;  // SwiGLU keeps the row pair in one warp
-    if (a.M <= 1) return launch_gemv_t<BITS, 1, R_SMALL, ACT>(a, stream);
-    if (a.M <= 2) return launch_gemv_t<BITS, 2, R_SMALL, ACT>(a, stream);
-    if (a.M <= 4) return launch_gemv_t<BITS, 4, 2, ACT>(a, stream);
-    return launch_gemv_t<BITS, 8, 2, ACT>(a, stream);
+    constexpr int R_SMALL = ACT == 2 ? 2 : 1;  // SwiGLU keeps each row pair in one group
+    if (a.M <= 1) return launch_gemv_t<BITS, 1, R_SMALL, 16, ACT>(a, stream);
+    if (a.M <= 2) return launch_gemv_t<BITS, 2, R_SMALL, 16, ACT>(a, stream);
+    if (a.M <= 4) return launch_gemv_t<BITS, 4, 2, 16, ACT>(a, stream);
+    if (a.N >= 8192) return launch_gemv_t<BITS, 8, 4, 8, ACT>(a, stream);
+    return launch_gemv_t<BITS, 8, 2, 16, ACT>(a, stream);
 }
 
 template <int BITS>
@@ -190,17 +251,18 @@ cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream) {
 // codes of weights 20w + 5i .. +4, first weight most significant.  A 256-entry table in shared
 // memory turns a byte into its five offset codes, one per byte of a 64-bit entry; the four entries
 // of a word are spliced into five dp4a words of four codes each, matching the 20 activation codes
-// k = 20w .. 20w + 19.  Same K walk as the 2-bit kernel with steps of 640 weights: lane l takes
-// word 32s + l of each row.  INT8 codes only (the 20-code groups do not fall on the 8-code
-// groups of the INT4 nibble layout).
+// k = 20w .. 20w + 19.  Same row groups, K split and finish as the 2-bit kernel, with steps of 640
+// weights: lane l takes word 32s + l of each row.  INT8 codes only (the 20-code groups do not fall
+// on the 8-code groups of the INT4 nibble layout).
 
-template <int T, int R, int ACT>
+template <int T, int R, int S, int KS, int ACT>
 __global__ void __launch_bounds__(kGemvWarps * 32)
     ternary_gemv_base3_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ scales,
                               const int32_t *__restrict__ rowsum, int M, int K,
                               const uint32_t *__restrict__ wp3, const float *__restrict__ gamma_ptr,
                               int N, int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ Y,
                               int early_weights) {
+    __shared__ int red[kGemvWarps][R * T];
     __shared__ unsigned long long digits[256];
     for (int v = threadIdx.x; v < 256; v += kGemvWarps * 32) {
         // byte 4 - j of the entry = base-3 digit j of v (digit 0 least significant); bytes
@@ -216,31 +278,35 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
     }
     __syncthreads();
     if (!early_weights) pdl_wait();
-    const int lane = threadIdx.x & 31;
-    const int n0 = (blockIdx.x * kGemvWarps + (threadIdx.x >> 5)) * R;
-    if (n0 >= N) return;  // whole warp leaves together (after the block's only barrier)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int ks = warp % KS;
+    const int n0 = (blockIdx.x * (kGemvWarps / KS) + warp / KS) * R;
+    const bool active = n0 < N;
     const int words = (K + 19) / 20;
     const int steps = (words + 31) / 32;
+    const int mine = active && steps > ks ? (steps - ks + KS - 1) / KS : 0;
     int acc[R][T];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < T; ++t) acc[r][t] = 0;
 
-    for (int s0 = 0; s0 < steps; s0 += kGemvSteps) {
-        uint32_t w[R][kGemvSteps];
+    for (int b0 = 0; b0 < mine; b0 += S) {
+        uint32_t w[R][S];
 #pragma unroll
-        for (int j = 0; j < kGemvSteps; ++j)
+        for (int j = 0; j < S; ++j) {
+            const int wi = 32 * (ks + KS * (b0 + j)) + lane;
 #pragma unroll
             for (int r = 0; r < R; ++r)
-                w[r][j] = (32 * (s0 + j) + lane < words && n0 + r < N)
-                              ? __ldg(wp3 + (int64_t)(n0 + r) * words + 32 * (s0 + j) + lane)
+                w[r][j] = (b0 + j < mine && wi < words && n0 + r < N)
+                              ? __ldg(wp3 + (int64_t)(n0 + r) * words + wi)
                               : 0u;  // byte 0 decodes to u = 0: adds nothing
-        if (early_weights && s0 == 0) pdl_wait();
+        }
+        if (early_weights && b0 == 0) pdl_wait();
 #pragma unroll
-        for (int j = 0; j < kGemvSteps; ++j) {
-            if (s0 + j >= steps) break;
-            const int k0 = 20 * (32 * (s0 + j) + lane);
+        for (int j = 0; j < S; ++j) {
+            if (b0 + j >= mine) break;
+            const int k0 = 20 * (32 * (ks + KS * (b0 + j)) + lane);
             // codes k0 + 4p .. +3 of every token (K % 4 == 0: a group is wholly in or out)
             uint32_t xs[T][5];
 #pragma unroll
@@ -270,36 +336,29 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
             }
         }
     }
-    gemv_epilogue<T, R, ACT>(acc, lane, n0, M, N, scales, rowsum, *gamma_ptr, acc_out, Y);
+    if (early_weights && mine == 0) pdl_wait();
+    gemv_finish<T, R, KS, ACT>(acc, red, active, lane, n0, M, N, scales, rowsum, gamma_ptr,
+                               acc_out, Y);
 }
 
-template <int T, int R, int ACT>
+template <int T, int R, int S, int ACT>
 static cudaError_t launch_gemv3_t(const GemmArgs &a, cudaStream_t stream) {
     static_assert(R * T <= 32, "one lane per (row, token) result");
-    const int64_t warps = (a.N + R - 1) / R;
-    const unsigned blocks = (unsigned)((warps + kGemvWarps - 1) / kGemvWarps);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks, 1, 1);
-    cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ternary_gemv_base3_kernel<T, R, ACT>,
-                              reinterpret_cast<const uint8_t *>(a.codes), a.scales, a.rowsum,
-                              (int)a.M, (int)a.K, a.Wp, a.gamma, (int)a.N, a.acc,
-                              reinterpret_cast<__nv_bfloat16 *>(a.Y), a.early_weights ? 1 : 0);
+    switch (gemv_split((a.N + R - 1) / R, (int)(((a.K + 19) / 20 + 31) / 32))) {
+        case 4: return launch_gemv_kernel<R, 4>(ternary_gemv_base3_kernel<T, R, S, 4, ACT>, a, stream);
+        case 2: return launch_gemv_kernel<R, 2>(ternary_gemv_base3_kernel<T, R, S, 2, ACT>, a, stream);
+        default: return launch_gemv_kernel<R, 1>(ternary_gemv_base3_kernel<T, R, S, 1, ACT>, a, stream);
+    }
 }
 
 template <int ACT>
 static cudaError_t launch_gemv3_a(const GemmArgs &a, cudaStream_t stream) {
     constexpr int R_SMALL = ACT == 2 ? 2 : 1;
-    if (a.M <= 1) return launch_gemv3_t<1, R_SMALL, ACT>(a, stream);
-    if (a.M <= 2) return launch_gemv3_t<2, R_SMALL, ACT>(a, stream);
-    if (a.M <= 4) return launch_gemv3_t<4, 2, ACT>(a, stream);
-    return launch_gemv3_t<8, 2, ACT>(a, stream);
+    if (a.M <= 1) return launch_gemv3_t<1, R_SMALL, 16, ACT>(a, stream);
+    if (a.M <= 2) return launch_gemv3_t<2, R_SMALL, 16, ACT>(a, stream);
+    if (a.M <= 4) return launch_gemv3_t<4, 2, 16, ACT>(a, stream);
+    if (a.N >= 8192) return launch_gemv3_t<8, 4, 8, ACT>(a, stream);
+    return launch_gemv3_t<8, 2, 16, ACT>(a, stream);
 }
 
 cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream) {

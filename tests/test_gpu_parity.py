@@ -151,6 +151,9 @@ def staged_product(B, M, K, N, bits, seed):
 
 @pytest.mark.parametrize("M,K,N", [
     (1, 256, 256), (3, 384, 136), (8, 2048, 264),          # decode kernel
+    (1, 8320, 136), (2, 4096, 8), (6, 8320, 264),           # decode, rows split over 2 / 4 warps
+    (8, 16384, 520), (4, 32768, 16),                        # (17 steps: uneven split)
+    (7, 4096, 8200),                                        # decode, 4-row groups
     (9, 256, 256), (130, 384, 136), (300, 2048, 264),       # tensor-core kernel, ragged tiles
     (256, 1024, 1024), (513, 128, 8),
     (1000, 640, 520),                                       # several tiles, 2.5 K stages
@@ -346,6 +349,8 @@ def check_act(Y, y_ref_bits):
 
 @pytest.mark.parametrize("M,K,N", [
     (1, 256, 256), (5, 2048, 272), (8, 384, 528),               # decode kernel
+    (8, 8320, 272), (2, 4096, 528),                             # decode, split rows
+    (8, 2048, 8192),                                            # decode, 4-row groups
     (9, 256, 256), (300, 2048, 272), (1000, 640, 528),          # tensor-core kernel
 ])
 @pytest.mark.parametrize("bits", [8, 4])
@@ -414,7 +419,7 @@ def test_base3_weights_degenerate(B):
 
 @pytest.mark.parametrize("M,K,N", [
     (1, 128, 8), (1, 2048, 264), (2, 384, 136), (3, 640, 256), (4, 8192, 520),
-    (5, 256, 8), (8, 2048, 1032), (8, 32768, 16),
+    (5, 256, 8), (8, 2048, 1032), (8, 32768, 16), (1, 10880, 136), (6, 5120, 264),
 ])
 def test_base3_product_int32_exact_and_bf16(B, M, K, N):
     X = synth.sharp_activations(M, K, seed=M * 3 + K)
@@ -438,7 +443,8 @@ def test_base3_product_int32_exact_and_bf16(B, M, K, N):
     assert np.all(y[y_ref == 0] == 0)
 
 
-@pytest.mark.parametrize("M,K,N", [(1, 2048, 272), (4, 640, 528), (8, 8192, 1040)])
+@pytest.mark.parametrize("M,K,N", [(1, 2048, 272), (4, 640, 528), (8, 8192, 1040),
+                                   (8, 1280, 8208)])
 @pytest.mark.parametrize("act", [1, 2])
 def test_base3_product_activation_matches_oracle(B, M, K, N, act):
     X = synth.sharp_activations(M, K, seed=M + 2 * K)

@@ -69,6 +69,7 @@ def lib():
                 "oracle_bitlinear_forward_norm": (i32, [vp, i64, i64, vp, i64, i32, i32, i32,
                                                         vp, f64, vp, vp, vp, vp, vp, vp, vp]),
                 "oracle_quant_act": (None, [vp, i64, i64, i32, vp, vp, vp, vp]),
+                "oracle_quant_act_absmean4": (None, [vp, i64, i64, vp, vp, vp, vp]),
                 "oracle_pack_int4": (None, [vp, i64, i64, vp]),
                 "oracle_unpack_int4": (None, [vp, i64, i64, vp]),
                 "oracle_gemm_i64": (None, [vp, vp, i64, i64, i64, vp]),
@@ -226,6 +227,23 @@ def quant_act(z_f32: np.ndarray, bits: int):
     pre = np.empty((M, K), dtype=np.float64)
     rowsum = np.empty(M, dtype=np.int64)
     lib().oracle_quant_act(_p(z), M, K, int(bits), _p(codes), _p(d), _p(pre), _p(rowsum))
+    return codes, d, pre, rowsum
+
+
+def quant_act_absmean4(z_f32: np.ndarray):
+    """Variant INT4 codes with a per-token absmean scale (the mean |z| maps to code sqrt(7)),
+    decided in fp32 and clipped to [-8, 7].
+
+    Returns (codes int8 [M, K], d float32 [M], pre float64 [M, K], rowsum int64 [M]) where
+    ``pre`` is z * s in double, the value the rounding decides on.
+    """
+    z = np.ascontiguousarray(z_f32, dtype=np.float32)
+    M, K = z.shape
+    codes = np.empty((M, K), dtype=np.int8)
+    d = np.empty(M, dtype=np.float32)
+    pre = np.empty((M, K), dtype=np.float64)
+    rowsum = np.empty(M, dtype=np.int64)
+    lib().oracle_quant_act_absmean4(_p(z), M, K, _p(codes), _p(d), _p(pre), _p(rowsum))
     return codes, d, pre, rowsum
 
 

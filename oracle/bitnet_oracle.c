@@ -32,7 +32,8 @@
  *   with an fp32 IEEE division and round-half-even; Hadamard = Sylvester order, scaled by
  *   1/sqrt(K) (orthonormal), size K; activation quantiser = per-token absmax with Q = 127
  *   (INT8) or Q = 7 (INT4), eps 1e-5, round-half-even, clip to [-Q-1, Q]; output =
- *   bf16_rn(acc * d * gamma) with d = max|z| / Q.
+ *   bf16_rn(acc * d * gamma) with d = max|z| / Q.  Variant INT4 quantiser (not the default):
+ *   absmean scale, the mean |z| of a token mapped to code sqrt(7), clipped to [-8, 7].
  *
  * Parity pins live in tests/test_oracle_pins.py: every exported function is checked there
  * against something independent of it (a page's worked example, a closed form, a library
@@ -313,6 +314,42 @@ void oracle_quant_act(const float *z, int64_t M, int64_t K, int bits, int8_t *co
             codes[m * K + k] = (int8_t)t;
             sum += (int64_t)t;
             if (pre) pre[m * K + k] = (double)row[k] * (double)Q / (double)g;
+        }
+        d[m] = dq;
+        if (rowsum) rowsum[m] = sum;
+    }
+}
+
+/*
+ * Variant INT4 quantiser with an absmean scale [v2: the INT4 activation strategy is named but its
+ * formula is not printed; the weights' absmean function of b1.58 / 2B4T 一.2 gives the form].
+ * Reading: per token row, beta = mean |z| (in double, rounded to fp32 once), g = max(beta,
+ * 1e-5); the mean magnitude is mapped to code sqrt(7): s = fl32(sqrt7 / g) with sqrt7 the fp32
+ * value of sqrt(7); codes = clip(rint(fl32(z * s)), -8, 7), round half to even; d = fl32(g /
+ * sqrt7).  Unlike absmax, values beyond 7/s are clipped.  pre (optional) = z * s in double, the
+ * value the rounding decides on.
+ */
+void oracle_quant_act_absmean4(const float *z, int64_t M, int64_t K, int8_t *codes, float *d,
+                               double *pre, int64_t *rowsum) {
+    const float sqrt7 = (float)sqrt(7.0);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const float *row = z + m * K;
+        double sa = 0.0;
+        for (int64_t k = 0; k < K; ++k) sa += fabs((double)row[k]);
+        double beta = sa / (double)K;
+        float g = (float)(beta < 1e-5 ? 1e-5 : beta);
+        volatile float s = sqrt7 / g;
+        volatile float dq = g / sqrt7;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            volatile float v = row[k] * s;
+            float t = nearbyintf(v);
+            if (t > 7.0f) t = 7.0f;
+            if (t < -8.0f) t = -8.0f;
+            codes[m * K + k] = (int8_t)t;
+            sum += (int64_t)t;
+            if (pre) pre[m * K + k] = (double)row[k] * (double)s;
         }
         d[m] = dq;
         if (rowsum) rowsum[m] = sum;

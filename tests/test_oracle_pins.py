@@ -257,6 +257,77 @@ def test_quant_brute_force_nearest_and_extremes(bits, Q):
     assert np.all(err[live] <= 0.5 * d[live, None] * (1 + 1e-6))
 
 
+# ---- variant INT4 quantiser with an absmean scale (a reading: the pages name the INT4 strategy
+# without its formula; the form is that of the weights' absmean) ----
+
+SQRT7_F32 = np.float32(math.sqrt(7.0))
+
+
+def _nearest_code_brute(v: np.ndarray, lo: int, hi: int) -> np.ndarray:
+    """Nearest integer in [lo, hi] to each value by exhaustive search, ties to the even one."""
+    cand = np.arange(lo, hi + 1, dtype=np.float64)
+    dist = np.abs(v.astype(np.float64)[..., None] - cand)
+    best = dist.min(axis=-1, keepdims=True)
+    tie_ok = np.isclose(dist, best, rtol=0, atol=0)
+    even = (cand % 2 == 0)
+    pick = np.where(tie_ok & even, 0, np.where(tie_ok, 1, 2))  # prefer even among the nearest
+    return cand[np.argmin(pick, axis=-1)].astype(np.int64)
+
+
+def test_absmean4_constant_magnitude_rows():
+    # |z| = a everywhere: beta = a, z * s = +-sqrt(7) -> +-3; d = a / sqrt(7)
+    a = np.float32(0.37)
+    z = np.where(np.arange(64) % 3 == 0, -a, a).astype(np.float32)[None, :].repeat(2, 0)
+    codes, d, _, rowsum = oracle.quant_act_absmean4(z)
+    np.testing.assert_array_equal(codes, np.where(z > 0, 3, -3))
+    assert d[0] == np.float32(a / SQRT7_F32)
+    assert rowsum[0] == codes[0].astype(np.int64).sum()
+
+
+def test_absmean4_brute_force_nearest_with_clipping():
+    rng = np.random.default_rng(11)
+    z = (rng.laplace(size=(12, 128)) * 0.2).astype(np.float32)
+    z[2, 5] = 40.0    # outliers far beyond the clip
+    z[4, 9] = -40.0
+    codes, d, pre, rowsum = oracle.quant_act_absmean4(z)
+    beta = np.abs(z.astype(np.float64)).mean(axis=1)
+    g = np.maximum(beta, 1e-5).astype(np.float32)
+    s = (SQRT7_F32 / g).astype(np.float32)
+    v = (z * s[:, None]).astype(np.float32)          # the fp32 product the decision is taken on
+    np.testing.assert_array_equal(codes, _nearest_code_brute(v, -8, 7))
+    assert codes[2, 5] == 7 and codes[4, 9] == -8
+    assert codes.min() >= -8 and codes.max() <= 7
+    np.testing.assert_array_equal(d, (g / SQRT7_F32).astype(np.float32))
+    np.testing.assert_array_equal(rowsum, codes.astype(np.int64).sum(axis=1))
+    np.testing.assert_allclose(pre, z.astype(np.float64) * s[:, None].astype(np.float64))
+
+
+def test_absmean4_zero_row_and_scale_invariance():
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((6, 256)).astype(np.float32)
+    z[1] = 0.0
+    codes, d, _, _ = oracle.quant_act_absmean4(z)
+    assert not codes[1].any() and d[1] == np.float32(np.float32(1e-5) / SQRT7_F32)
+    # a power-of-two scale leaves the codes unchanged and scales d exactly
+    codes2, d2, _, _ = oracle.quant_act_absmean4((z * np.float32(8.0)).astype(np.float32))
+    np.testing.assert_array_equal(codes2[[0, 2, 3, 4, 5]], codes[[0, 2, 3, 4, 5]])
+    np.testing.assert_array_equal(d2[[0, 2, 3, 4, 5]], d[[0, 2, 3, 4, 5]] * np.float32(8.0))
+
+
+def test_absmean4_gaussian_clip_fraction():
+    # a Gaussian row (what the Hadamard produces): beta ~ sigma*sqrt(2/pi), so code 7 needs
+    # z > 6.5 beta / sqrt(7) and code -8 needs z < -7.5 beta / sqrt(7): the fractions of the
+    # two end codes follow the normal tail at those points
+    from scipy.stats import norm
+    z = np.random.default_rng(9).standard_normal((16, 16384)).astype(np.float32)
+    codes, _, _, _ = oracle.quant_act_absmean4(z)
+    r = math.sqrt(2 / math.pi) / math.sqrt(7.0)
+    p7, p8 = norm.sf(6.5 * r), norm.cdf(-7.5 * r)
+    n = codes.size
+    for frac, p in ((np.mean(codes == 7), p7), (np.mean(codes == -8), p8)):
+        assert abs(frac - p) < 5 * math.sqrt(p * (1 - p) / n), (frac, p)
+
+
 # ----------------------------------------------------------------------------------------
 # Ternary product (2B4T article, 一.2: +1 adds, -1 subtracts, 0 skips)
 # ----------------------------------------------------------------------------------------

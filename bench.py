@@ -314,6 +314,9 @@ def run_gpu(args, wl, rank, world, device):
         gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
 
     def quant(b):
+        if args.absmean4:  # the variant INT4 quantiser (absmean scale)
+            B.bitnet_act_quant_absmean4(b["X"], wl.hadamard, b["codes"], b["scales"], b["rowsum"])
+            return
         if gain is not None:
             B.bitnet_act_quant_norm(b["X"], gain, 1e-5, wl.hadamard, wl.act_bits, b["codes"],
                                     b["scales"], b["rowsum"])
@@ -466,7 +469,8 @@ def run_gpu(args, wl, rank, world, device):
                 "achieved_gbs": w_bytes / (phase_ms[0] * 1e-3) / 1e9,
                 "frac": w_bytes / (phase_ms[0] * 1e-3) / 1e9 / hbm},
             ("fwht_quant" if wl.hadamard else "act_quant_plain")
-            + ("+rmsnorm" if args.rmsnorm else "") + " (alone, outside the timed steps)": {
+            + ("+rmsnorm" if args.rmsnorm else "") + ("+absmean4" if args.absmean4 else "")
+            + " (alone, outside the timed steps)": {
                 "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,
                 "achieved_gbs": q_bytes / (phase_ms[1] * 1e-3) / 1e9,
                 "frac": q_bytes / (phase_ms[1] * 1e-3) / 1e9 / hbm},
@@ -516,6 +520,7 @@ def run_gpu(args, wl, rank, world, device):
                        "act_bits": wl.act_bits, "rmsnorm": bool(args.rmsnorm),
                        "activation": args.activation,
                        "weights": "base3" if args.base3 else "2bit",
+                       "act_scale": "absmean" if args.absmean4 else "absmax",
                        "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {copies} copies "
@@ -563,7 +568,10 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
         gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
 
     def fwd(b):
-        if args.base3:
+        if args.absmean4:
+            B.bitnet_bitlinear_forward_absmean4(b["Xd"], b["Wp"], b["gamma"], wl.hadamard,
+                                                Y=b["Yd"], ws=b["ws"])
+        elif args.base3:
             B.bitnet_bitlinear_forward_base3(b["Xd"], b["Wp"], b["gamma"], wl.hadamard, act,
                                              Y=b["Yd"], ws=b["ws"])
         elif gain is not None:
@@ -641,6 +649,9 @@ def main():
     ap.add_argument("--base3", action="store_true",
                     help="store the weights five to a byte (base 3) for the decode product "
                          "(at most 8 tokens, INT8 activations)")
+    ap.add_argument("--absmean4", action="store_true",
+                    help="variant INT4 activation quantiser with a per-token absmean scale "
+                         "(INT4 workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -651,6 +662,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = synth.WORKLOADS[args.workload]
+    if args.absmean4 and (wl.act_bits != 4 or args.rmsnorm or args.base3 or
+                          args.activation != "none"):
+        ap.error("--absmean4 serves INT4 workloads, without --rmsnorm, --base3 or --activation")
     if args.base3 and (wl.M > 8 or wl.act_bits != 8 or args.rmsnorm):
         ap.error("--base3 serves workloads of at most 8 tokens with INT8 activations, "
                  "without --rmsnorm")

@@ -90,6 +90,15 @@ _SIGS = {
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                                     ctypes.c_void_p, ctypes.c_size_t,
                                                     ctypes.c_void_p]),
+    "bitnet_act_quant_absmean4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p]),
+    "bitnet_bitlinear_forward_absmean4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                         ctypes.c_int64, ctypes.c_void_p,
+                                                         ctypes.c_void_p, ctypes.c_int64,
+                                                         ctypes.c_int, ctypes.c_void_p,
+                                                         ctypes.c_void_p, ctypes.c_size_t,
+                                                         ctypes.c_void_p]),
     "bitnet_base3_weight_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
     "bitnet_quantize_pack_weights_base3": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
                                                           ctypes.c_int64, ctypes.c_void_p,
@@ -427,6 +436,50 @@ def bitnet_norm_bitlinear_forward(X, norm_gain, eps, hadamard, Wp, gamma, act_bi
                                         int(act_bits), Y.data_ptr(), ws.data_ptr(),
                                         ws.numel() * ws.element_size(), _stream(stream)),
         "bitnet_norm_bitlinear_forward")
+    return Y
+
+
+def bitnet_act_quant_absmean4(X: torch.Tensor, hadamard: bool, codes=None, scales=None,
+                              rowsum=None, stream=None):
+    """Variant INT4 quantiser with a per-token absmean scale.  Returns (codes uint8 [M, K/2]
+    nibbles, scales, rowsum), consumed by the product with act_bits 4."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, K = X.shape
+    if codes is None:
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(M, dtype=torch.float32, device=X.device)
+    if rowsum is None:
+        rowsum = torch.empty(M, dtype=torch.int32, device=X.device)
+    _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, 4)), "codes")
+    _nbytes_at_least(scales, 4 * M, "scales")
+    _nbytes_at_least(rowsum, 4 * M, "rowsum")
+    _rc(L.bitnet_act_quant_absmean4(X.data_ptr(), M, K, int(bool(hadamard)), codes.data_ptr(),
+                                    scales.data_ptr(), rowsum.data_ptr(), _stream(stream)),
+        "bitnet_act_quant_absmean4")
+    return codes, scales, rowsum
+
+
+def bitnet_bitlinear_forward_absmean4(X, Wp, gamma, hadamard: bool, Y=None, ws=None, stream=None):
+    """Y = (H-)BitLinear(X) with the absmean INT4 activation quantiser."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    _check(Wp, "Wp")
+    _check(gamma, "gamma", torch.float32)
+    M, K = X.shape
+    N = Wp.shape[0]
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    _nbytes_at_least(Y, 2 * M * N, "Y")
+    need = int(L.bitnet_workspace_bytes(M, K, N, 4))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _rc(L.bitnet_bitlinear_forward_absmean4(X.data_ptr(), M, K, Wp.data_ptr(), gamma.data_ptr(),
+                                            N, int(bool(hadamard)), Y.data_ptr(), ws.data_ptr(),
+                                            ws.numel() * ws.element_size(), _stream(stream)),
+        "bitnet_bitlinear_forward_absmean4")
     return Y
 
 

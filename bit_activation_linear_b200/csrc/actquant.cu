@@ -53,8 +53,8 @@ struct FwhtPlan {
     // resident CTAs per SM the register allocation is sized for: 16 warps per SM
     static constexpr int MIN_BLOCKS = THREADS >= 512 ? 1 : 512 / THREADS;
     static constexpr int WARPS_PER_TEAM = TEAM >= 32 ? TEAM / 32 : 1;
-    static constexpr int RED = TEAMS * WARPS_PER_TEAM;         // reduction slots (max, then sum)
-    static constexpr int RED_BYTES = (2 * RED * 4 + 15) / 16 * 16;
+    static constexpr int RED = TEAMS * WARPS_PER_TEAM;  // reduction slots: max, code sum, |z| sum
+    static constexpr int RED_BYTES = (2 * RED * 4 + RED * 8 + 15) / 16 * 16;
     static constexpr int CHUNKS = L / 4;                       // 16-byte chunks per run
     static constexpr int SWZ = (CHUNKS < 8 ? CHUNKS : 8) - 1;  // chunk XOR mask
     static constexpr size_t SMEM =
@@ -96,7 +96,13 @@ __device__ __forceinline__ void team_sync(int team) {
     }
 }
 
-template <class P, int BITS, bool ZOUT, bool NORM>
+// sqrt(7) rounded to fp32: the code the mean |z| of a token maps to in the absmean INT4 variant
+constexpr float kSqrt7 = 2.6457513110645906f;
+
+// ABSMEAN: the variant INT4 quantiser (BITS == 4 only): the scale comes from the mean |z| of
+// the token (summed in double) instead of max |z|, s = sqrt7 / max(mean, 1e-5), and codes are
+// clipped to [-8, 7].
+template <class P, int BITS, bool ZOUT, bool NORM, bool ABSMEAN = false>
 __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     fwht_quant_kernel(const uint8_t *__restrict__ X, int M, float rsqrt_k,
                       const uint32_t *__restrict__ gain2, float eps,
@@ -259,15 +265,19 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
         }
     }
 
-    // ---- normalise and reduce max|z| over the team ----
+    // ---- normalise and reduce max|z| (or, ABSMEAN, sum |z|) over the team ----
     const float2 rk2 = make_float2(rsqrt_k, rsqrt_k);
     float mx = 0.f;
+    double sa = 0.0;
 #pragma unroll
     for (int col = 0; col < P::COLS; ++col)
 #pragma unroll
         for (int p = 0; p < L / 2; ++p) {
             b[col][p] = mul2_rn(b[col][p], rk2);
-            mx = fmaxf(mx, fmaxf(fabsf(b[col][p].x), fabsf(b[col][p].y)));
+            if constexpr (ABSMEAN)
+                sa += fabs((double)b[col][p].x) + fabs((double)b[col][p].y);
+            else
+                mx = fmaxf(mx, fmaxf(fabsf(b[col][p].x), fabsf(b[col][p].y)));
         }
 
     if constexpr (ZOUT) {
@@ -285,19 +295,37 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
         }
     } else {
         constexpr int W = TEAM < 32 ? TEAM : 32;
+        static_assert(!ABSMEAN || BITS == 4, "the absmean variant is an INT4 quantiser");
+        float g;
+        if constexpr (ABSMEAN) {
 #pragma unroll
-        for (int o = W / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        if constexpr (TEAM > 32) {
-            // all warps of this team finished their phase-B reads of tbuf before this barrier
-            constexpr int WPT = P::WARPS_PER_TEAM;
-            if (lane == 0) red[team * WPT + (r >> 5)] = mx;
-            team_sync<TEAM>(team);
-            mx = red[team * WPT];
+            for (int o = W / 2; o > 0; o >>= 1) sa += __shfl_xor_sync(0xFFFFFFFFu, sa, o);
+            if constexpr (TEAM > 32) {
+                constexpr int WPT = P::WARPS_PER_TEAM;
+                double *redd = reinterpret_cast<double *>(reinterpret_cast<uint8_t *>(red) +
+                                                          2 * P::RED * 4);
+                if (lane == 0) redd[team * WPT + (r >> 5)] = sa;
+                team_sync<TEAM>(team);
+                sa = redd[team * WPT];
 #pragma unroll
-            for (int i = 1; i < WPT; ++i) mx = fmaxf(mx, red[team * WPT + i]);
+                for (int i = 1; i < WPT; ++i) sa += redd[team * WPT + i];
+            }
+            g = (float)fmax(sa / (double)K, 1e-5);
+        } else {
+#pragma unroll
+            for (int o = W / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+            if constexpr (TEAM > 32) {
+                // all warps of this team finished their phase-B reads of tbuf before this barrier
+                constexpr int WPT = P::WARPS_PER_TEAM;
+                if (lane == 0) red[team * WPT + (r >> 5)] = mx;
+                team_sync<TEAM>(team);
+                mx = red[team * WPT];
+#pragma unroll
+                for (int i = 1; i < WPT; ++i) mx = fmaxf(mx, red[team * WPT + i]);
+            }
+            g = fmaxf(mx, 1e-5f);
         }
-        constexpr float Q = BITS == 4 ? 7.f : 127.f;
-        const float g = fmaxf(mx, 1e-5f);
+        constexpr float Q = ABSMEAN ? kSqrt7 : BITS == 4 ? 7.f : 127.f;
         const float s = __fdiv_rn(Q, g);
         const float dq = __fdiv_rn(g, Q);
         const float2 magic2 = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
@@ -317,6 +345,8 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
                     // round(fl(z * s)), the same two roundings the reference takes
                     float2 t = make_float2(__fmul_rn(b[col][g16 * 8 + i].x, s),
                                            __fmul_rn(b[col][g16 * 8 + i].y, s));
+                    if constexpr (ABSMEAN)  // clip before rounding: the same as after it
+                        t = make_float2(fminf(fmaxf(t.x, -8.f), 7.f), fminf(fmaxf(t.y, -8.f), 7.f));
                     float2 u = __fadd2_rn(t, magic2);
                     f[2 * i] = __float_as_uint(u.x);
                     f[2 * i + 1] = __float_as_uint(u.y);
@@ -375,7 +405,7 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
 // One warp per token row, two passes over the row (the second one hits L1/L2).
 // With NORM each value is first RMS-normalised, y = (x * rinv) * g as in fwht_quant_kernel (an
 // extra pass over the row for sum(x^2)); with ZOUT the kernel writes y in fp32 instead of codes.
-template <int BITS, bool NORM, bool ZOUT>
+template <int BITS, bool NORM, bool ZOUT, bool ABSMEAN = false>
 __global__ void __launch_bounds__(256)
     act_quant_plain_kernel(const uint4 *__restrict__ X, int64_t M, int64_t K,
                            const uint4 *__restrict__ gain8, float eps,
@@ -432,17 +462,31 @@ __global__ void __launch_bounds__(256)
         }
         return;
     }
+    static_assert(!ABSMEAN || BITS == 4, "the absmean variant is an INT4 quantiser");
     float mx = 0.f;
+    double sa = 0.0;  // ABSMEAN: sum |y| in double (see fwht_quant_kernel)
     for (int64_t c = lane; c < nchunk; c += 32) {
         float2 y[4];
         load8(c, y);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fmaxf(fabsf(y[i].x), fabsf(y[i].y)));
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (ABSMEAN)
+                sa += fabs((double)y[i].x) + fabs((double)y[i].y);
+            else
+                mx = fmaxf(mx, fmaxf(fabsf(y[i].x), fabsf(y[i].y)));
+        }
     }
+    float g;
+    if constexpr (ABSMEAN) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    constexpr float Q = BITS == 4 ? 7.f : 127.f;
-    const float g = fmaxf(mx, 1e-5f);
+        for (int o = 16; o > 0; o >>= 1) sa += __shfl_xor_sync(0xFFFFFFFFu, sa, o);
+        g = (float)fmax(sa / (double)K, 1e-5);
+    } else {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        g = fmaxf(mx, 1e-5f);
+    }
+    constexpr float Q = ABSMEAN ? kSqrt7 : BITS == 4 ? 7.f : 127.f;
     const float s = __fdiv_rn(Q, g);
     const float dq = __fdiv_rn(g, Q);
     const float2 magic2 = make_float2(12582912.f, 12582912.f);
@@ -454,7 +498,10 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             // __fmul_rn is never contracted with the following add (see fwht_quant_kernel)
-            float2 u = __fadd2_rn(make_float2(__fmul_rn(y[i].x, s), __fmul_rn(y[i].y, s)), magic2);
+            float2 t = make_float2(__fmul_rn(y[i].x, s), __fmul_rn(y[i].y, s));
+            if constexpr (ABSMEAN)
+                t = make_float2(fminf(fmaxf(t.x, -8.f), 7.f), fminf(fmaxf(t.y, -8.f), 7.f));
+            float2 u = __fadd2_rn(t, magic2);
             f[2 * i] = __float_as_uint(u.x);
             f[2 * i + 1] = __float_as_uint(u.y);
         }
@@ -477,11 +524,11 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <class P, int BITS, bool ZOUT, bool NORM>
+template <class P, int BITS, bool ZOUT, bool NORM, bool ABSMEAN = false>
 static cudaError_t launch_fwht_t(const void *X, int64_t M, const NormArgs &nrm, void *codes,
                                  float *scales, int32_t *rowsum, float *zout, int *status,
                                  cudaStream_t stream) {
-    auto kern = fwht_quant_kernel<P, BITS, ZOUT, NORM>;
+    auto kern = fwht_quant_kernel<P, BITS, ZOUT, NORM, ABSMEAN>;
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -514,6 +561,12 @@ static cudaError_t launch_fwht_n(const void *X, int64_t M, int act_bits, const N
                                  void *codes, float *scales, int32_t *rowsum, float *zout,
                                  int *status, cudaStream_t stream) {
     using P = typename FwhtConfig<LOGK>::P;
+    if (act_bits == kActInt4Absmean) {
+        if constexpr (NORM) return cudaErrorInvalidValue;  // not offered with the norm
+        else
+            return launch_fwht_t<P, 4, false, false, true>(X, M, nrm, codes, scales, rowsum,
+                                                            nullptr, status, stream);
+    }
     if (zout)
         return launch_fwht_t<P, 8, true, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
                                                stream);
@@ -568,6 +621,14 @@ static cudaError_t launch_plain_t(const void *X, int64_t M, int64_t K, const Nor
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
                                    const NormArgs &nrm, void *codes, float *scales,
                                    int32_t *rowsum, float *zout, cudaStream_t stream) {
+    if (act_bits == kActInt4Absmean) {
+        if (nrm.on || zout) return cudaErrorInvalidValue;
+        const int64_t blocks = (M + 7) / 8;
+        act_quant_plain_kernel<4, false, false, true><<<(unsigned)blocks, 256, 0, stream>>>(
+            reinterpret_cast<const uint4 *>(X), M, K, nullptr, 0.f,
+            reinterpret_cast<uint8_t *>(codes), scales, rowsum, nullptr);
+        return cudaGetLastError();
+    }
     if (zout)  // the normalised rows themselves (the parity entry); only with a norm
         return launch_plain_t<8, true, true>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
     if (nrm.on)

@@ -151,7 +151,8 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
 
 int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const float *gamma,
                  int64_t N, int act_bits, void *Y, void *ws, size_t ws_bytes, int hadamard,
-                 cudaStream_t stream, const NormArgs &nrm = NormArgs(), int activation = 0) {
+                 cudaStream_t stream, const NormArgs &nrm = NormArgs(), int activation = 0,
+                 bool absmean4 = false) {
     int rc = check_shape(M, K, N, true, true);
     if (rc) return rc;
     if (act_bits != 8 && act_bits != 4)
@@ -170,8 +171,8 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
     float *scales = reinterpret_cast<float *>(w + round256(bitnet_act_codes_bytes(M, K, act_bits)));
     int32_t *rowsum = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(scales) +
                                                   round256((size_t)M * sizeof(float)));
-    if ((rc = act_quant_impl(st, X, M, K, hadamard, act_bits, codes, scales, rowsum, nullptr,
-                             stream, nrm)))
+    if ((rc = act_quant_impl(st, X, M, K, hadamard, absmean4 ? kActInt4Absmean : act_bits, codes,
+                             scales, rowsum, nullptr, stream, nrm)))
         return rc;
     // the quantiser above was launched in stream order after whatever wrote Wp
     return gemm_impl(st, codes, scales, rowsum, M, K, Wp, gamma, N, act_bits, nullptr, Y, stream,
@@ -443,6 +444,29 @@ int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const voi
                               void *ws_dev, size_t ws_bytes, bitnet_stream_t stream) {
     return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, act_bits, Y_dev, ws_dev, ws_bytes, 1,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadamard,
+                              void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
+                              bitnet_stream_t stream) {
+    int rc = check_shape(M, K, 8, true, false);
+    if (rc) return rc;
+    if (!X_dev || !codes_dev || !scales_dev || !rowsum_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(X_dev) || !aligned16(codes_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    return act_quant_impl(st, X_dev, M, K, hadamard ? 1 : 0, kActInt4Absmean, codes_dev,
+                          scales_dev, rowsum_dev, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_bitlinear_forward_absmean4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                                      const float *gamma_dev, int64_t N, int hadamard, void *Y_dev,
+                                      void *ws_dev, size_t ws_bytes, bitnet_stream_t stream) {
+    return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, 4, Y_dev, ws_dev, ws_bytes,
+                        hadamard ? 1 : 0, reinterpret_cast<cudaStream_t>(stream), NormArgs(), 0,
+                        true);
 }
 
 size_t bitnet_base3_weight_bytes(int64_t N, int64_t K) {

@@ -33,6 +33,10 @@ struct NormArgs {
 cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
                               const NormArgs &nrm, void *codes, float *scales, int32_t *rowsum,
                               float *zout, int *status, cudaStream_t stream);
+// act_bits value that selects the variant INT4 quantiser with an absmean scale (INT4 codes,
+// layout as act_bits 4); the launchers reject it together with a norm or a z output.
+constexpr int kActInt4Absmean = 0x104;
+
 // Quantise without a transform; K % 128 == 0.  zout != nullptr (with nrm.on) writes the
 // normalised rows in fp32 instead of codes.
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,

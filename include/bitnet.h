@@ -227,6 +227,34 @@ int bitnet_bitlinear_forward_act(const void *X_dev, int64_t M, int64_t K, const 
                                  bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* Variant INT4 quantiser with an absmean scale                                              */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * The BitNet v2 write-up names a 4-bit activation strategy but its formula is not printed; the
+ * default INT4 path (act_bits 4) uses absmax like INT8.  This variant takes the form of the
+ * weights' absmean function ("The Era of 1-bit LLMs" summary, 方法论; 2B4T article, 一.2) for the
+ * activations instead.  Per token row, with z = (1/sqrt(K)) H_K x (hadamard != 0) or z = x:
+ *   beta = mean_k |z_k| (summed in double), g = fp32(max(beta, 1e-5)),
+ *   s = sqrt7 / g (sqrt7 = fp32 value of sqrt(7), IEEE fp32 division): the mean magnitude maps to
+ *   code sqrt(7), so a Gaussian row spans the 4-bit range to about 2.3 standard deviations;
+ *   codes = clip(round_half_even(z * s), -8, 7)  (values beyond the range are clipped);
+ *   scales[m] = g / sqrt7;  rowsum[m] = sum_k codes.
+ * Outputs in the INT4 layout of bitnet_act_quant (act_bits 4), so bitnet_ternary_gemm with
+ * act_bits 4 consumes them.  Shapes, alignment and errors as bitnet_act_quant.
+ */
+int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadamard,
+                              void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
+                              bitnet_stream_t stream);
+
+/* The whole layer with this quantiser: bitnet_act_quant_absmean4, then the product with act_bits
+ * 4.  ws_bytes >= bitnet_workspace_bytes(M, K, N, 4); other arguments as
+ * bitnet_bitlinear_forward. */
+int bitnet_bitlinear_forward_absmean4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                                      const float *gamma_dev, int64_t N, int hadamard, void *Y_dev,
+                                      void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* Base-3 weights for decode                                                                */
 /* ---------------------------------------------------------------------------------------- */
 

@@ -491,3 +491,60 @@ def test_base3_product_equals_two_bit_product(B):
     assert g2.item() == g3.item()
     assert torch.equal(a2, a3)
     assert torch.equal(y2.view(torch.int16), y3.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------------------
+# variant INT4 quantiser with a per-token absmean scale
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("K", [128, 256, 2048, 4096, 8192, 16384, 32768])
+def test_absmean4_hadamard_codes(B, K):
+    M = 37 if K <= 8192 else 9
+    X = synth.sharp_activations(M, K, seed=5 * K + 1)
+    Xd = dev_bf16(X)
+    z = B.bitnet_fwht_f32(Xd).cpu().numpy()
+    codes, scales, rowsum = B.bitnet_act_quant_absmean4(Xd, True)
+    B.bitnet_sync_status()
+    c_ref, d_ref, pre, _ = oracle.quant_act_absmean4(z)
+    c = oracle.unpack_int4(codes.cpu().numpy().view(np.uint8), K)
+    n_diff = check_codes(c, c_ref, pre)
+    assert n_diff == 0, f"{n_diff} codes differ (within the boundary tolerance)"
+    np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), c.astype(np.int64).sum(axis=1))
+    assert (c == 7).any() or (c == -8).any()  # the clip is exercised
+
+
+@pytest.mark.parametrize("K", [128, 640, 4096])
+def test_absmean4_plain_codes(B, K):
+    M = 19
+    X = synth.gaussian_activations(M, K, seed=K + 17)
+    X[3] = 0  # a zero row: zero codes, guarded scale
+    codes, scales, rowsum = B.bitnet_act_quant_absmean4(dev_bf16(X), False)
+    B.bitnet_sync_status()
+    z = oracle.bf16_to_f64(X).astype(np.float32)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act_absmean4(z)
+    c = oracle.unpack_int4(codes.cpu().numpy().view(np.uint8), K)
+    assert check_codes(c, c_ref, pre) == 0
+    np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
+    assert not c[3].any()
+
+
+@pytest.mark.parametrize("name,rows", [("wdown_8192", 16), ("tiny", None)])
+def test_absmean4_forward_end_to_end(B, name, rows):
+    wl = synth.WORKLOADS[name]
+    X, W = wl.activations(seed=6), wl.weights(seed=6)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    Y = B.bitnet_bitlinear_forward_absmean4(dev_bf16(X), Wp, gamma, wl.hadamard)
+    B.bitnet_sync_status()
+    sel = np.arange(wl.M) if rows is None else np.sort(
+        np.random.default_rng(6).choice(wl.M, size=rows, replace=False))
+    x = oracle.bf16_to_f64(X[sel])
+    z = (oracle.fwht(x) if wl.hadamard else x).astype(np.float32)
+    codes, d, _, _ = oracle.quant_act_absmean4(z)
+    g = oracle.absmean_gamma(W)
+    assert np.float32(gamma.item()) == g
+    acc = oracle.gemm_i64(codes, oracle.ternarize(W, g))
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc, d, g))
+    y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
+    assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL

@@ -58,6 +58,8 @@ def lib():
                 "oracle_abs_sum_bf16": (f64, [vp, i64]),
                 "oracle_absmean_gamma": (f32, [vp, i64]),
                 "oracle_ternarize": (None, [vp, i64, f32, vp]),
+                "oracle_absmean_gamma_f32": (f32, [vp, i64]),
+                "oracle_ternarize_f32": (None, [vp, i64, f32, vp]),
                 "oracle_pack_ternary": (None, [vp, i64, i64, vp]),
                 "oracle_unpack_ternary": (i64, [vp, i64, i64, vp]),
                 "oracle_pack_base3": (None, [vp, i64, vp]),
@@ -127,6 +129,27 @@ def ternarize(w_bf16: np.ndarray, gamma) -> np.ndarray:
     q = np.empty(w.shape, dtype=np.int8)
     lib().oracle_ternarize(_p(w), w.size, ctypes.c_float(float(gamma)), _p(q))
     return q
+
+
+def absmean_gamma_f32(w_f32: np.ndarray) -> np.float32:
+    """absmean scale of fp32 weights (the Hadamard-rotated rows): fp32(max(mean|w|, 1e-5)),
+    the sum in double."""
+    w = np.ascontiguousarray(w_f32, dtype=np.float32)
+    return np.float32(lib().oracle_absmean_gamma_f32(_p(w), w.size))
+
+
+def ternarize_f32(w_f32: np.ndarray, gamma) -> np.ndarray:
+    """RoundClip(w / gamma, -1, 1) on fp32 weights, decided in fp32.  int8, same shape."""
+    w = np.ascontiguousarray(w_f32, dtype=np.float32)
+    q = np.empty(w.shape, dtype=np.int8)
+    lib().oracle_ternarize_f32(_p(w), w.size, float(gamma), _p(q))
+    return q
+
+
+def rotate_weights(w_bf16: np.ndarray) -> np.ndarray:
+    """Weight half of the weight + activation rotation: W' = W H / sqrt(K) row by row (H is
+    symmetric, so W' x' = W x for x' = H x / sqrt(K)), in double, rounded to fp32 once."""
+    return fwht(bf16_to_f64(w_bf16)).astype(np.float32)
 
 
 def pack_ternary(q: np.ndarray) -> np.ndarray:

@@ -34,6 +34,9 @@
  *   (INT8) or Q = 7 (INT4), eps 1e-5, round-half-even, clip to [-Q-1, Q]; output =
  *   bf16_rn(acc * d * gamma) with d = max|z| / Q.  Variant INT4 quantiser (not the default):
  *   absmean scale, the mean |z| of a token mapped to code sqrt(7), clipped to [-8, 7].
+ *   Variant weight + activation rotation (not the default): the rows of W are transformed by
+ *   the same orthonormal Hadamard before the absmean ternarisation, W' = W H / sqrt(K), so that
+ *   W' (H x / sqrt(K)) = W x; the rotated rows are rounded to fp32 once, then ternarised.
  *
  * Parity pins live in tests/test_oracle_pins.py: every exported function is checked there
  * against something independent of it (a page's worked example, a closed form, a library
@@ -118,6 +121,28 @@ void oracle_ternarize(const uint16_t *w, int64_t n, float gamma, int8_t *q) {
     for (int64_t i = 0; i < n; ++i) {
         float wf = (float)bf16_to_double(w[i]);
         volatile float r = wf / gamma;          /* volatile: keep it one fp32 division */
+        float t = nearbyintf(r);
+        if (t > 1.0f) t = 1.0f;
+        if (t < -1.0f) t = -1.0f;
+        q[i] = (int8_t)t;
+    }
+}
+
+/* The same absmean ternarisation on fp32 weights: the Hadamard-rotated rows W' = W H / sqrt(K)
+ * of the weight + activation rotation [v2: Hadamard rotation of the weights and the activations,
+ * or of the activations only].  gamma = fp32(max(mean |w'|, 1e-5)), the sum in double; then
+ * q = RoundClip(w' / gamma, -1, 1) with one IEEE fp32 division and round-half-to-even. */
+float oracle_absmean_gamma_f32(const float *w, int64_t n) {
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i) s += fabs((double)w[i]);
+    double mean = s / (double)n;
+    if (mean < 1e-5) mean = 1e-5;
+    return (float)mean;
+}
+
+void oracle_ternarize_f32(const float *w, int64_t n, float gamma, int8_t *q) {
+    for (int64_t i = 0; i < n; ++i) {
+        volatile float r = w[i] / gamma;
         float t = nearbyintf(r);
         if (t > 1.0f) t = 1.0f;
         if (t < -1.0f) t = -1.0f;

@@ -170,6 +170,50 @@ def test_ternarize_constant_and_zero_weights():
     np.testing.assert_array_equal(oracle.ternarize(Z, oracle.absmean_gamma(Z)), 0)
 
 
+# ---- weight + activation rotation: absmean ternarisation of the rotated fp32 rows ----
+
+def test_ternarize_f32_equals_bf16_path_on_bf16_values():
+    # fp32 weights that are exactly bf16 values give the bf16 path's gamma and codes
+    W = synth.latent_weights(64, 256, seed=21)
+    wf = oracle.bf16_to_f64(W).astype(np.float32)
+    g = oracle.absmean_gamma(W)
+    assert oracle.absmean_gamma_f32(wf) == g
+    np.testing.assert_array_equal(oracle.ternarize_f32(wf, g), oracle.ternarize(W, g))
+
+
+def test_ternarize_f32_brute_force_and_library_mean():
+    rng = np.random.default_rng(22)
+    w = (rng.standard_normal((32, 128)) * 0.02).astype(np.float32)
+    w[0, :4] = [0.0, -0.0, 1e-9, -1e-9]
+    g = oracle.absmean_gamma_f32(w)
+    assert g == np.float32(np.abs(w.astype(np.float64)).mean())
+    r = (w / g).astype(np.float32)                    # one fp32 division, as the decision takes it
+    cand = np.array([-1.0, 0.0, 1.0])
+    dist = np.abs(r.astype(np.float64)[..., None] - cand)
+    best = dist.min(axis=-1, keepdims=True)
+    # nearest of {-1, 0, 1}; a tie at +-0.5 goes to 0 (even)
+    pick = np.where(dist == best, np.where(cand == 0, 0, 1), 2)
+    q_ref = cand[np.argmin(pick, axis=-1)].astype(np.int8)
+    np.testing.assert_array_equal(oracle.ternarize_f32(w, g), q_ref)
+    # ties exactly at half of gamma
+    half = np.array([[g * np.float32(0.5), -g * np.float32(0.5)]], dtype=np.float32)
+    np.testing.assert_array_equal(oracle.ternarize_f32(half, g), [[0, 0]])
+
+
+@pytest.mark.parametrize("K", [128, 1024])
+def test_rotate_weights_is_the_explicit_product_and_preserves_wx(K):
+    W = synth.latent_weights(24, K, seed=K)
+    Wr = oracle.rotate_weights(W)
+    H = scipy.linalg.hadamard(K).astype(np.float64)
+    ref = (oracle.bf16_to_f64(W) @ H / math.sqrt(K)).astype(np.float32)
+    np.testing.assert_array_equal(Wr, ref)
+    # W' (H x / sqrt(K)) = W x: the rotation cancels in the product
+    x = np.random.default_rng(K).standard_normal((5, K))
+    lhs = Wr.astype(np.float64) @ oracle.fwht(x).T
+    rhs = oracle.bf16_to_f64(W) @ x.T
+    np.testing.assert_allclose(lhs, rhs, rtol=0, atol=1e-6 * np.abs(rhs).max())
+
+
 def test_ternarize_ties_round_half_to_even():
     """|w / gamma| = 0.5 exactly rounds to 0, 1.5 rounds to 2 and clips to 1."""
     gamma = np.float32(0.25)

@@ -65,15 +65,16 @@ def weight_bytes(N: int, K: int, base3: bool) -> int:
     return N * 4 * ((K + 19) // 20) if base3 else N * K // 4
 
 
-def kernel_work(wl, base3: bool = False):
+def kernel_work(wl, base3: bool = False, rotate: bool = False):
     M, K, N = wl.M, wl.K, wl.N
     code_bytes = M * K if wl.act_bits == 8 else M * K // 2
     wb = weight_bytes(N, K, base3)
     return {
-        # read W (bf16) once
-        "absmean_partials": {"bytes": 2 * N * K},
+        # read W (bf16) once; with the weight rotation: the transform (bf16 in, fp32 out), then
+        # the sum over the fp32 rows
+        "absmean_partials": {"bytes": (2 + 4 + 4) * N * K if rotate else 2 * N * K},
         # read W (bf16) once, write the stored weights
-        "ternarize_pack": {"bytes": 2 * N * K + wb},
+        "ternarize_pack": {"bytes": (4 if rotate else 2) * N * K + wb},
         # read X (bf16), write codes + scale + code sum per token
         "fwht_quant": {"bytes": 2 * M * K + code_bytes + 8 * M},
         # product: 2 M N K integer ops; bytes = codes + 2-bit weights + bf16 Y
@@ -269,6 +270,12 @@ def barrier():
         dist.barrier()
 
 
+def weight_ws_bytes(B, args, N: int, K: int) -> int:
+    if args.rotate_weights:
+        return B.bitnet_weight_workspace_bytes_rotated(N, K)
+    return B.bitnet_weight_workspace_bytes(N, K)
+
+
 def run_gpu(args, wl, rank, world, device):
     from bit_activation_linear_b200 import binding as B
     B.load_library()
@@ -290,7 +297,7 @@ def run_gpu(args, wl, rank, world, device):
         Wp = torch.empty((N, weight_bytes(N, K, args.base3) // N), dtype=torch.uint8,
                          device=device)
         gamma = torch.empty(1, dtype=torch.float32, device=device)
-        wws = torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
+        wws = torch.empty(max(weight_ws_bytes(B, args, N, K), 256), dtype=torch.uint8,
                           device=device)
         codes = torch.empty((M, K if wl.act_bits == 8 else K // 2), dtype=torch.uint8,
                             device=device)
@@ -301,6 +308,9 @@ def run_gpu(args, wl, rank, world, device):
                          rowsum=rowsum, Y=Y))
 
     def weights(b):
+        if args.rotate_weights:  # the weight half of the weight + activation rotation
+            B.bitnet_quantize_pack_weights_rotated(b["W"], b["Wp"], b["gamma"], b["wws"])
+            return
         if args.base3:
             B.bitnet_quantize_pack_weights_base3(b["W"], b["Wp"], b["gamma"], b["wws"])
             return
@@ -457,7 +467,7 @@ def run_gpu(args, wl, rank, world, device):
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
-        work = kernel_work(wl, args.base3)
+        work = kernel_work(wl, args.base3, args.rotate_weights)
         int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
         achieved = work["ternary_gemm_tc"]["ops"] / (gemm_ms * 1e-3) / 1e12
         hbm = peaks["hbm_gbs"]
@@ -521,6 +531,7 @@ def run_gpu(args, wl, rank, world, device):
                        "activation": args.activation,
                        "weights": "base3" if args.base3 else "2bit",
                        "act_scale": "absmean" if args.absmean4 else "absmax",
+                       "weight_rotation": bool(args.rotate_weights),
                        "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
                        "l2": f"inputs rotated over {copies} copies "
@@ -558,7 +569,7 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
             Wp=torch.empty((N, weight_bytes(N, K, args.base3) // N), dtype=torch.uint8,
                            device=device),
             gamma=torch.empty(1, dtype=torch.float32, device=device),
-            wws=torch.empty(max(B.bitnet_weight_workspace_bytes(N, K), 256), dtype=torch.uint8,
+            wws=torch.empty(max(weight_ws_bytes(B, args, N, K), 256), dtype=torch.uint8,
                             device=device),
             ws=torch.empty(max(B.bitnet_workspace_bytes(M, K, N, wl.act_bits), 256),
                            dtype=torch.uint8, device=device)))
@@ -605,6 +616,7 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
         with torch.cuda.stream(s_c):
             s_c.wait_event(ev_in[k])
             pack = (B.bitnet_quantize_pack_weights_base3 if args.base3
+                    else B.bitnet_quantize_pack_weights_rotated if args.rotate_weights
                     else B.bitnet_quantize_pack_weights)
             pack(b["Wd"], b["Wp"], b["gamma"], b["wws"])
             fwd(b)
@@ -652,6 +664,9 @@ def main():
     ap.add_argument("--absmean4", action="store_true",
                     help="variant INT4 activation quantiser with a per-token absmean scale "
                          "(INT4 workloads)")
+    ap.add_argument("--rotate-weights", action="store_true",
+                    help="weight + activation Hadamard rotation: ternarise the rotated weight "
+                         "rows (H-BitLinear workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -665,6 +680,8 @@ def main():
     if args.absmean4 and (wl.act_bits != 4 or args.rmsnorm or args.base3 or
                           args.activation != "none"):
         ap.error("--absmean4 serves INT4 workloads, without --rmsnorm, --base3 or --activation")
+    if args.rotate_weights and (not wl.hadamard or args.base3):
+        ap.error("--rotate-weights serves H-BitLinear workloads with the 2-bit weights")
     if args.base3 and (wl.M > 8 or wl.act_bits != 8 or args.rmsnorm):
         ap.error("--base3 serves workloads of at most 8 tokens with INT8 activations, "
                  "without --rmsnorm")

@@ -90,6 +90,11 @@ _SIGS = {
                                                     ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                                     ctypes.c_void_p, ctypes.c_size_t,
                                                     ctypes.c_void_p]),
+    "bitnet_weight_workspace_bytes_rotated": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "bitnet_quantize_pack_weights_rotated": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+                                                            ctypes.c_int64, ctypes.c_void_p,
+                                                            ctypes.c_void_p, ctypes.c_void_p,
+                                                            ctypes.c_size_t, ctypes.c_void_p]),
     "bitnet_act_quant_absmean4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p]),
@@ -437,6 +442,33 @@ def bitnet_norm_bitlinear_forward(X, norm_gain, eps, hadamard, Wp, gamma, act_bi
                                         ws.numel() * ws.element_size(), _stream(stream)),
         "bitnet_norm_bitlinear_forward")
     return Y
+
+
+def bitnet_weight_workspace_bytes_rotated(N: int, K: int) -> int:
+    return int(load_library().bitnet_weight_workspace_bytes_rotated(N, K))
+
+
+def bitnet_quantize_pack_weights_rotated(W: torch.Tensor, Wp: torch.Tensor | None = None,
+                                         gamma: torch.Tensor | None = None,
+                                         ws: torch.Tensor | None = None, stream=None):
+    """Weight half of the weight + activation Hadamard rotation: ternarise and pack the rows of
+    W H / sqrt(K).  Returns (Wp uint8 [N, K/4], gamma float [1]) for bitnet_hbitlinear_forward."""
+    L = load_library()
+    _check(W, "W", torch.bfloat16, 2)
+    N, K = W.shape
+    if Wp is None:
+        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    _nbytes_at_least(Wp, int(L.bitnet_packed_weight_bytes(N, K)), "Wp")
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    need = int(L.bitnet_weight_workspace_bytes_rotated(N, K))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    _rc(L.bitnet_quantize_pack_weights_rotated(W.data_ptr(), N, K, Wp.data_ptr(),
+                                               gamma.data_ptr(), ws.data_ptr(),
+                                               ws.numel() * ws.element_size(), _stream(stream)),
+        "bitnet_quantize_pack_weights_rotated")
+    return Wp, gamma
 
 
 def bitnet_act_quant_absmean4(X: torch.Tensor, hadamard: bool, codes=None, scales=None,

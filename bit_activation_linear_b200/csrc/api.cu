@@ -446,6 +446,40 @@ int bitnet_hbitlinear_forward(const void *X_dev, int64_t M, int64_t K, const voi
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t bitnet_weight_workspace_bytes_rotated(int64_t N, int64_t K) {
+    if (N <= 0 || K <= 0) return 0;
+    return round256((size_t)N * (size_t)K * sizeof(float)) + bitnet_weight_workspace_bytes(N, K);
+}
+
+int bitnet_quantize_pack_weights_rotated(const void *W_dev, int64_t N, int64_t K, void *Wp_dev,
+                                         float *gamma_dev, void *ws_dev, size_t ws_bytes,
+                                         bitnet_stream_t stream) {
+    int rc = check_shape(N, K, 8, true, false);  // N rows are transformed like M token rows
+    if (rc) return rc;
+    if (N % 8 != 0)
+        return fail(BITNET_ERR_INVALID, "N = %lld must be a positive multiple of 8", (long long)N);
+    if (!W_dev || !Wp_dev || !gamma_dev || !ws_dev)
+        return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(W_dev) || !aligned16(Wp_dev) || !aligned16(ws_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    const size_t need = bitnet_weight_workspace_bytes_rotated(N, K);
+    if (ws_bytes < need)
+        return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *rot = static_cast<float *>(ws_dev);
+    double *partials = reinterpret_cast<double *>(static_cast<uint8_t *>(ws_dev) +
+                                                  round256((size_t)N * (size_t)K * sizeof(float)));
+    // the rotated rows W' = W H / sqrt(K): the transform of the activation path, on weight rows
+    if ((rc = act_quant_impl(st, W_dev, N, K, 1, 8, nullptr, nullptr, nullptr, rot, s)))
+        return rc;
+    const int P = absmean_num_partials(N * K);
+    return launched(launch_ternarize_pack_f32(rot, N * K, partials, P,
+                                              static_cast<uint32_t *>(Wp_dev), gamma_dev, s),
+                    2, "ternarize_pack_f32");
+}
+
 int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadamard,
                               void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
                               bitnet_stream_t stream) {

@@ -14,6 +14,11 @@ cudaError_t launch_absmean_partials(const void *W, int64_t n, double *partials, 
                                     cudaStream_t stream);
 cudaError_t launch_ternarize_pack(const void *W, int64_t n, const double *partials, int P,
                                   uint32_t *Wp, float *gamma, cudaStream_t stream);
+// absmean ternarisation and 2-bit pack of fp32 weights (the Hadamard-rotated rows): two
+// launches, the partial sums into partials[P].
+cudaError_t launch_ternarize_pack_f32(const float *W, int64_t n, double *partials, int P,
+                                      uint32_t *Wp, float *gamma, cudaStream_t stream);
+
 // Base-3 rows (five weights per byte, ceil(K/20) 32-bit words per row) for the decode product.
 cudaError_t launch_ternarize_pack_base3(const void *W, int64_t N, int64_t K,
                                         const double *partials, int P, uint32_t *Wp3,

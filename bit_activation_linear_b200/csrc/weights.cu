@@ -93,13 +93,13 @@ __device__ __forceinline__ uint32_t ternary_threshold_bits(float gamma) {
     return h;
 }
 
-// gamma from the P partial sums, then its decision threshold; every block computes it the same
-// way (a fixed assignment of partials to threads and a fixed reduction tree), so gamma does not
-// depend on the launch.  Block 0 writes gamma.  Contains __syncthreads.
-__device__ __forceinline__ uint32_t block_threshold(const double *__restrict__ partials, int P,
-                                                    double n_weights, float *__restrict__ gamma_out) {
+// gamma from the P partial sums; every block computes it the same way (a fixed assignment of
+// partials to threads and a fixed reduction tree), so gamma does not depend on the launch.
+// Block 0 writes gamma.  Contains __syncthreads.
+__device__ __forceinline__ float block_gamma(const double *__restrict__ partials, int P,
+                                             double n_weights, float *__restrict__ gamma_out) {
     __shared__ double warp_sums[kWeightThreads / 32];
-    __shared__ uint32_t s_thr;
+    __shared__ float s_gamma;
     double s = 0.0;
     for (int j = threadIdx.x; j < P; j += kWeightThreads) s += partials[j];
 #pragma unroll
@@ -110,11 +110,17 @@ __device__ __forceinline__ uint32_t block_threshold(const double *__restrict__ p
         double t = 0.0;
         for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
         const float g = (float)fmax(t / n_weights, 1e-5);
-        s_thr = ternary_threshold_bits(g);
+        s_gamma = g;
         if (blockIdx.x == 0) *gamma_out = g;
     }
     __syncthreads();
-    return s_thr;
+    return s_gamma;
+}
+
+// gamma (block_gamma) and its decision threshold for bf16 weights.
+__device__ __forceinline__ uint32_t block_threshold(const double *__restrict__ partials, int P,
+                                                    double n_weights, float *__restrict__ gamma_out) {
+    return ternary_threshold_bits(block_gamma(partials, P, n_weights, gamma_out));
 }
 
 // Offset code u = q + 1 of one bf16 weight against the threshold (see ternary_threshold_bits).
@@ -212,6 +218,85 @@ cudaError_t launch_ternarize_pack_base3(const void *W, int64_t N, int64_t K,
     ternarize_pack_base3_kernel<<<(unsigned)blocks, kWeightThreads, 0, stream>>>(
         reinterpret_cast<const uint16_t *>(W), N, K, (double)N * (double)K, partials, P, Wp3,
         gamma);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// fp32 weights: the rows W' = W H / sqrt(K) of the weight + activation rotation (BitNet v2
+// write-up: Hadamard rotation of the weights and the activations, or of the activations only).
+// The same absmean ternarisation on fp32 values: partial sums of |w'| in fp64 (a fixed grid of P
+// blocks, as for bf16), then q = RoundClip(w' / gamma, -1, 1) with one IEEE fp32 division.
+
+__global__ void __launch_bounds__(kWeightThreads)
+    absmean_partials_f32_kernel(const float4 *__restrict__ w, int64_t nvec,
+                                double *__restrict__ partials) {
+    double acc0 = 0.0, acc1 = 0.0;
+    const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
+    int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {  // four 16-byte loads in flight
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(w + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            acc0 += fabs((double)v[u].x) + fabs((double)v[u].y);
+            acc1 += fabs((double)v[u].z) + fabs((double)v[u].w);
+        }
+    }
+    for (; i < nvec; i += stride) {
+        const float4 v = __ldg(w + i);
+        acc0 += fabs((double)v.x) + fabs((double)v.y);
+        acc1 += fabs((double)v.z) + fabs((double)v.w);
+    }
+    double s = acc0 + acc1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    __shared__ double warp_sums[kWeightThreads / 32];
+    if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int k = 0; k < kWeightThreads / 32; ++k) t += warp_sums[k];
+        partials[blockIdx.x] = t;
+    }
+}
+
+__global__ void __launch_bounds__(kWeightThreads)
+    ternarize_pack_f32_kernel(const float4 *__restrict__ w, int64_t nwords, double n_weights,
+                              const double *__restrict__ partials, int P,
+                              uint32_t *__restrict__ wp, float *__restrict__ gamma_out) {
+    const float g = block_gamma(partials, P, n_weights, gamma_out);
+    const int64_t stride = (int64_t)gridDim.x * kWeightThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kWeightThreads + threadIdx.x; i < nwords; i += stride) {
+        float4 v[4];  // weights 16i .. 16i+15
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = __ldg(w + 4 * i + c);
+        const float f[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                             v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            // rint(r) with ties to even is 0 for |r| <= 0.5 and +-1 (after the clip) above
+            const float r = __fdiv_rn(f[e], g);
+            const uint32_t u = fabsf(r) > 0.5f ? (r > 0.f ? 2u : 0u) : 1u;
+            word |= u << (8 * (e & 3) + 2 * (e >> 2));
+        }
+        wp[i] = word;
+    }
+}
+
+cudaError_t launch_ternarize_pack_f32(const float *W, int64_t n, double *partials, int P,
+                                      uint32_t *Wp, float *gamma, cudaStream_t stream) {
+    absmean_partials_f32_kernel<<<P, kWeightThreads, 0, stream>>>(
+        reinterpret_cast<const float4 *>(W), n / 4, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t nwords = n / 16;
+    int64_t blocks = (nwords + kWeightThreads - 1) / kWeightThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    ternarize_pack_f32_kernel<<<(unsigned)blocks, kWeightThreads, 0, stream>>>(
+        reinterpret_cast<const float4 *>(W), nwords, (double)n, partials, P, Wp, gamma);
     return cudaGetLastError();
 }
 

@@ -227,6 +227,29 @@ int bitnet_bitlinear_forward_act(const void *X_dev, int64_t M, int64_t K, const 
                                  bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* Variant: weight + activation Hadamard rotation                                            */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * The BitNet v2 write-up's ablation rotates the weights as well as the activations (Hadamard
+ * rotation of weights + activations, or of activations only).  With the orthonormal, symmetric
+ * H' = H_K / sqrt(K) (Sylvester order), W x = (W H')(H' x): the activation half is
+ * bitnet_hbitlinear_forward unchanged, and this call prepares the weight half.  Per weight row:
+ *   w' = H' w computed in fp32 by the transform of bitnet_fwht_f32 (the same kernel), then
+ *   gamma = fp32(max(mean |w'|, 1e-5)) (sum in double), q = RoundClip(w' / gamma, -1, 1) with an
+ *   IEEE fp32 division and round-half-to-even, packed as bitnet_quantize_pack_weights.
+ * K must be a power of two in [128, 32768] (else BITNET_ERR_UNSUPPORTED) and N a multiple of 8.
+ * ws_dev: ws_bytes >= bitnet_weight_workspace_bytes_rotated(N, K) (the fp32 rotated rows, 4NK
+ * bytes, then the partial sums); contents undefined afterwards.  Use the result with
+ * bitnet_hbitlinear_forward.
+ */
+size_t bitnet_weight_workspace_bytes_rotated(int64_t N, int64_t K);
+
+int bitnet_quantize_pack_weights_rotated(const void *W_dev, int64_t N, int64_t K, void *Wp_dev,
+                                         float *gamma_dev, void *ws_dev, size_t ws_bytes,
+                                         bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* Variant INT4 quantiser with an absmean scale                                              */
 /* ---------------------------------------------------------------------------------------- */
 

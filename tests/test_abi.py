@@ -156,3 +156,15 @@ def test_absmean4_entries_reject_bad_arguments_before_the_device(lib):
     q = ctypes.c_void_p(24)
     assert lib.bitnet_act_quant_absmean4(q, 4, 256, 1, p, p, p, None) == -1      # misaligned
     assert lib.bitnet_bitlinear_forward_absmean4(p, 4, 256, p, p, 256, 1, p, p, 0, None) == -5
+
+
+def test_rotated_weight_entries_size_and_rejections_before_the_device(lib):
+    ws = lib.bitnet_weight_workspace_bytes_rotated(2048, 2048)
+    assert ws >= 4 * 2048 * 2048 + lib.bitnet_weight_workspace_bytes(2048, 2048)
+    assert ws % 256 == 0 and lib.bitnet_weight_workspace_bytes_rotated(0, 128) == 0
+    p = ctypes.c_void_p(16)
+    assert lib.bitnet_quantize_pack_weights_rotated(p, 256, 200, p, p, p, 1 << 30, None) == -1
+    assert lib.bitnet_quantize_pack_weights_rotated(p, 12, 256, p, p, p, 1 << 30, None) == -1
+    assert lib.bitnet_quantize_pack_weights_rotated(p, 256, 256, p, p, p, 1024, None) == -5
+    q = ctypes.c_void_p(24)
+    assert lib.bitnet_quantize_pack_weights_rotated(p, 256, 256, q, p, p, 1 << 30, None) == -1

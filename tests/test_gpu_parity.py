@@ -548,3 +548,52 @@ def test_absmean4_forward_end_to_end(B, name, rows):
     y_ref = oracle.bf16_to_f64(oracle.dequant(acc, d, g))
     y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
     assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
+
+
+# ----------------------------------------------------------------------------------------
+# variant: weight + activation Hadamard rotation (the weight half)
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K", [(256, 256), (8, 128), (264, 2048), (1032, 8192), (16, 32768)])
+def test_rotated_weights_bit_exact_on_the_gpu_rotation(B, N, K):
+    W = synth.latent_weights(N, K, seed=N + 3 * K)
+    Wd = dev_bf16(W)
+    Wp, gamma = B.bitnet_quantize_pack_weights_rotated(Wd)
+    Wr = B.bitnet_fwht_f32(Wd).cpu().numpy()  # the same transform, as fp32 rows
+    B.bitnet_sync_status()
+    g_ref = oracle.absmean_gamma_f32(Wr)
+    assert np.float32(gamma.item()) == g_ref
+    ref = oracle.pack_ternary(oracle.ternarize_f32(Wr, g_ref))
+    np.testing.assert_array_equal(Wp.cpu().numpy().view(np.uint32).reshape(N, K // 16), ref)
+    # the GPU rotation against the oracle's double transform
+    Wr_ref = oracle.rotate_weights(W)
+    err = np.abs(Wr - Wr_ref).max(axis=1) / np.abs(Wr_ref).max(axis=1)
+    assert err.max() <= FWHT_REL
+
+
+def test_rotated_weights_degenerate(B):
+    Wp, gamma = B.bitnet_quantize_pack_weights_rotated(dev_bf16(np.zeros((16, 256), np.uint16)))
+    B.bitnet_sync_status()
+    assert np.float32(gamma.item()) == np.float32(1e-5)
+    q, bad = oracle.unpack_ternary(Wp.cpu().numpy().view(np.uint32), 256)
+    assert bad == 0 and not q.any()
+
+
+@pytest.mark.parametrize("name,rows", [("tiny", None), ("wo_2048", 32), ("wdown_8192", 8)])
+def test_rotated_forward_end_to_end(B, name, rows):
+    wl = synth.WORKLOADS[name]
+    X, W = wl.activations(seed=8), wl.weights(seed=8)
+    Wp, gamma = B.bitnet_quantize_pack_weights_rotated(dev_bf16(W))
+    Y = B.bitnet_hbitlinear_forward(dev_bf16(X), Wp, gamma, wl.act_bits)
+    B.bitnet_sync_status()
+    sel = np.arange(wl.M) if rows is None else np.sort(
+        np.random.default_rng(8).choice(wl.M, size=rows, replace=False))
+    z = oracle.fwht(oracle.bf16_to_f64(X[sel])).astype(np.float32)
+    codes, d, _, _ = oracle.quant_act(z, wl.act_bits)
+    Wr = oracle.rotate_weights(W)
+    g = oracle.absmean_gamma_f32(Wr)
+    assert abs(np.float32(gamma.item()) / g - 1) <= 1e-6
+    acc = oracle.gemm_i64(codes, oracle.ternarize_f32(Wr, g))
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc, d, g))
+    y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
+    assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL

@@ -7,18 +7,18 @@
 // the matching four activation codes accumulates sum_k u * c exactly; the per-token code sum
 // written by the quantiser removes the offset: sum_k q * c = sum_k u * c - sum_k c.
 //
-// A row group of R consecutive output features is owned by KS warps of one CTA (KS = 1, 2 or 4:
-// when a matrix has few row groups, long rows are split so that it still fills the GPU).  The K axis is walked
-// in steps of 512 weights, step s going to warp s mod KS of the group: in a step lane l takes the
-// packed word 32s + l of each row (weights k = 512s + 16l .. +15, one coalesced 128-byte load per
-// warp and row) and the 16 matching codes of each token (one coalesced 16-byte load per lane).
-// The weight words of S steps are loaded before any is used, so every warp keeps S*R loads in
-// flight and the weight stream is requested at full rate.  Every code is loaded once per R rows,
-// so R grows with the token count (1 row for 1-2 tokens, 2 for 3-8; 4 for 5-8 tokens when
-// N >= 8192) to keep the L1 traffic of the code loads down.  Activation codes (at most eight tokens) are read
-// through L1, where every warp of the SM finds them.  The lanes' partial sums are reduced with
-// shuffles, then across the group's warps through shared memory, and the group's first warp
-// writes the results.
+// A row group of R consecutive output features is owned by KS warps of one CTA (KS = 1, 2 or
+// 4: when a matrix has few row groups, long rows are split so that it still fills the GPU).  The
+// K axis is walked in steps of 512 weights, step s going to warp s mod KS of the group: in a step
+// lane l takes the packed word 32s + l of each row (weights k = 512s + 16l .. +15, one coalesced
+// 128-byte load per warp and row) and the 16 matching codes of each token (one coalesced 16-byte
+// load per lane).  The weight words of S steps are loaded before any is used, so every warp keeps
+// S*R loads in flight and the weight stream is requested at full rate.  Every code is loaded once
+// per R rows, so R grows with the token count (1 row for 1-2 tokens, 2 for 3-8, and 4 for 5-8
+// tokens when N >= 8192) to keep the L1 traffic of the code loads down.  Activation codes (at
+// most eight tokens) are read through L1, where every warp of the SM finds them.  The lanes'
+// partial sums are reduced with shuffles, then across the group's warps through shared memory,
+// and the group's first warp writes the results.
 #include "common.cuh"
 #include "kernels.h"
 

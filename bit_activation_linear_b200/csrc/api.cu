@@ -144,9 +144,9 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
     a.early_weights = early_weights;
     a.activation = activation;
     if (M <= kGemvMaxTokens) return launched(launch_ternary_gemv(a, stream), 1, "ternary_gemv");
-    const int n = (acc ? 1 : 0) + (Y ? 1 : 0);
-    return launched(launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream), n,
-                    "ternary_gemm_tc");
+    int n = 0;
+    const cudaError_t e = launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream, &n);
+    return launched(e, n, "ternary_gemm_tc");
 }
 
 int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const float *gamma,

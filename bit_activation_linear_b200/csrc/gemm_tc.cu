@@ -78,7 +78,9 @@ constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_EPI = 16;
 // What the epilogue writes: the int32 accumulators (parity entry), the rescaled bf16 output, or
 // the rescaled output through an activation (squared ReLU; SwiGLU over interleaved gate/up
 // features, half as many columns).
-enum OutMode { OUT_ACC = 0, OUT_BF16 = 1, OUT_RELU2 = 2, OUT_SWIGLU = 3 };
+// OUT_PARTIAL: the raw int32 sums of a unit's K chunk are added atomically into an int32 [M, N]
+// scratch; splitk_finish_kernel then writes the outputs (see launch_ternary_gemm_tc).
+enum OutMode { OUT_ACC = 0, OUT_BF16 = 1, OUT_RELU2 = 2, OUT_SWIGLU = 3, OUT_PARTIAL = 4 };
 constexpr int NUM_THREADS = 24 * 32;
 
 // Unpack / code warps: eight warps outside the MMA warp's scheduler partition (warp % 4 == 1).
@@ -139,7 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                            const __grid_constant__ CUtensorMap tmap_y,
                            void *__restrict__ Yout, const float *__restrict__ scales,
                            const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
-                           int M, int N, int K, int *status) {
+                           int M, int N, int K, int split, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,8 +163,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int num_tiles = n_ftiles * n_ttiles;
     const int KS = (K + BK - 1) / BK;  // stages per tile (the last one may be half: K % 256 = 128)
     constexpr int B_GROUPS = BITS == 8 ? 2 : 1;
-    const int my_tiles = pair < num_tiles ? (num_tiles - 1 - pair) / npairs + 1 : 0;
-    const int total = my_tiles * KS;  // (tile, stage) iterations of this pair
+    // Work units: tile x K chunk (split chunks per tile, split <= KS; split = 1 unless
+    // MODE == OUT_PARTIAL).  Pair p takes units p, p + npairs, ...; unit u is tile u / split,
+    // stages [c*KS/split, (c+1)*KS/split) of it with c = u % split.
+    if constexpr (MODE != OUT_PARTIAL) split = 1;  // a constant: the one-pass loops as written
+    const int num_units = num_tiles * split;
+    const int my_units = pair < num_units ? (num_units - 1 - pair) / npairs + 1 : 0;
+    auto unit = [&](int t, int &tile, int &kb, int &ke) {
+        const int u = pair + t * npairs;
+        tile = u / split;
+        const int c = u - tile * split;
+        kb = c * KS / split;
+        ke = (c + 1) * KS / split;
+    };
+    int total = 0;  // (unit, stage) iterations of this pair
+    for (int t = 0; t < my_units; ++t) {
+        int tile, kb, ke;
+        unit(t, tile, kb, ke);
+        total += ke - kb;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -186,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (warp == WARP_TMA && lane == 0) {
         prefetch_tensormap(&tmap_codes);
         prefetch_tensormap(&tmap_w);
-        if (MODE != OUT_ACC) prefetch_tensormap(&tmap_y);
+        if (MODE != OUT_ACC && MODE != OUT_PARTIAL) prefetch_tensormap(&tmap_y);
     }
     if (warp == WARP_MMA) {
         tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
@@ -204,10 +223,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------------------ code TMA
         if (lane == 0) {
             uint32_t issued = 0, ph = 0;  // for the final drain
-            int t = 0, ks = 0, s = 0;
+            int t = 0, s = 0, tile = 0, kb = 0, ke = 0;
+            if (my_units > 0) unit(0, tile, kb, ke);
+            int ks = kb;
             uint32_t p = 0;
             for (int it = 0; it < total; ++it) {
-                const int tile = pair + t * npairs;
                 const int m0 = (tile / n_ftiles) * BM + (int)rank * HM;
                 if (!mbar_wait(&bar->empty[s], p ^ 1, status)) break;
                 uint8_t *dst = sa + (size_t)s * A_STAGE_BYTES;
@@ -224,7 +244,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 issued |= 1u << s;
                 ph = (ph & ~(1u << s)) | (p << s);
-                if (++ks == KS) { ks = 0; ++t; }
+                if (++ks == ke && ++t < my_units) {
+                    unit(t, tile, kb, ke);
+                    ks = kb;
+                }
                 if (++s == STAGES) { s = 0; p ^= 1; }
             }
             // no copy may still be writing shared memory when the CTA exits: each CTA waits
@@ -237,17 +260,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // ------------------------------------------------------------------ weight-tile TMA
         if (lane == 0) {
             uint32_t issued = 0, ph = 0;
-            int t = 0, ks = 0, s_w = 0;
+            int t = 0, s_w = 0, tile = 0, kb = 0, ke = 0;
+            if (my_units > 0) unit(0, tile, kb, ke);
+            int ks = kb;
             uint32_t p_w = 0;
             for (int it = 0; it < total; ++it) {
-                const int tile = pair + t * npairs;
                 if (!mbar_wait(&bar->empty_w[s_w], p_w ^ 1, status)) break;
                 mbar_arrive_expect_tx(&bar->full_w[s_w], W_STAGE_BYTES);
                 tma_load_2d(sw + (size_t)s_w * W_STAGE_BYTES, &tmap_w, ks * (BK / 4),
                             (tile % n_ftiles) * BN + (int)rank * HN, &bar->full_w[s_w]);
                 issued |= 1u << s_w;
                 ph = (ph & ~(1u << s_w)) | (p_w << s_w);
-                if (++ks == KS) { ks = 0; ++t; }
+                if (++ks == ke && ++t < my_units) {
+                    unit(t, tile, kb, ke);
+                    ks = kb;
+                }
                 if (++s_w == W_STAGES) { s_w = 0; p_w ^= 1; }
             }
             for (int i = 0; i < W_STAGES; ++i)
@@ -260,11 +287,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const uint32_t sa_addr = smem_addr(sa);
             const uint32_t sb_addr = smem_addr(sb);
             bool next = total > 0 && mbar_test_wait(&bar->full[0], 0);
-            int t = 0, ks = 0, s = 0;
+            int t = 0, s = 0, tile = 0, kb = 0, ke = 0;
+            if (my_units > 0) unit(0, tile, kb, ke);
+            int ks = kb;
             uint32_t p = 0;
             for (int it = 0; it < total; ++it) {
                 const int ab = t & 1;
-                if (ks == 0 &&
+                if (ks == kb &&
                     !mbar_wait(&bar->acc_empty[ab], ((uint32_t)(t >> 1) & 1) ^ 1, status))
                     break;
                 if (!next && !mbar_wait(&bar->full[s], p, status)) break;
@@ -284,11 +313,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     for (int kk = 0; kk < SUBK / UMMA_K; ++kk)
                         mma_i8_ss_pair(d_tmem, adesc + (uint64_t)(kk * UMMA_K / 16),
                                        bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
-                                       (ks | sub | kk) != 0 ? 1u : 0u);
+                                       (ks != kb || sub != 0 || kk != 0) ? 1u : 0u);
                 }
                 mma_commit_pair(&bar->empty[s], 3);
-                if (ks == KS - 1) mma_commit_pair(&bar->acc_full[ab], 3);
-                if (++ks == KS) { ks = 0; ++t; }
+                if (ks == ke - 1) mma_commit_pair(&bar->acc_full[ab], 3);
+                if (++ks == ke && ++t < my_units) {
+                    unit(t, tile, kb, ke);
+                    ks = kb;
+                }
                 s = s1;
                 if (s == 0) p ^= 1;
             }
@@ -347,8 +379,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         const uint32_t t_lane = tmem + ((uint32_t)(wq * 32) << 16);
         uint8_t *ybox = sy + (size_t)(warp - WARP_EPI) * Y_BOX_BYTES;
         const float gamma = *gamma_ptr;
-        for (int t = 0; t < my_tiles; ++t) {
-            const int tile = pair + t * npairs;
+        for (int t = 0; t < my_units; ++t) {
+            int tile, kb, ke;
+            unit(t, tile, kb, ke);
             const int nf = tile % n_ftiles;
             const int mt = tile / n_ftiles;
             const int ab = t & 1;
@@ -365,7 +398,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_32x32b_x32(t_lane + ab * BN + col, v);
                 tmem_wait_ld();
                 const int n0 = nf * BN + col;
-                if constexpr (MODE == OUT_ACC) {
+                if constexpr (MODE == OUT_PARTIAL) {
+                    // this unit's K chunk of the raw sums (the code-sum offset is removed once,
+                    // by splitk_finish_kernel); integer additions in any order are exact
+                    int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (m_ok && n0 + j < N) atomicAdd(row + n0 + j, (int)v[j]);
+                } else if constexpr (MODE == OUT_ACC) {
                     int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -514,7 +554,7 @@ static int max_pairs(int num_sms) {
 template <int BITS, int MODE>
 static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
                                const CUtensorMap &my, void *out, int64_t tiles, int num_sms,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, int split = 1) {
     auto kern = ternary_gemm_tc_kernel<BITS, MODE>;
     static bool configured[64] = {};
     int dev = 0;
@@ -526,7 +566,8 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
         configured[dev] = true;
     }
     const int pairs_max = max_pairs<BITS, MODE>(num_sms);
-    const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
+    const int64_t units = tiles * split;
+    const int pairs = (int)(units < pairs_max ? units : pairs_max);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -538,7 +579,115 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mc, mw, my, out, a.scales, a.rowsum, a.gamma, (int)a.M,
-                              (int)a.N, (int)a.K, a.status);
+                              (int)a.N, (int)a.K, split, a.status);
+}
+
+// ------------------------------------------------------------------------------------------
+// K split for small tile counts.  With few tiles (decode-sized token counts) most pairs would
+// idle while a few walk the whole K axis; instead each tile's K axis is cut into `split` chunks,
+// every (tile, chunk) unit goes to its own pair, and the units' int32 sums are added atomically
+// into a library-owned scratch (exact: integer addition in any order).  splitk_finish_kernel then
+// applies the epilogue arithmetic of the one-pass kernel (same fp32 operations, so the same bf16
+// results) and returns the scratch to zero for the next call.  One scratch per device: calls
+// that take this path must not overlap on the GPU (they are serialised on one stream).
+
+constexpr int64_t kSplitAccElems = int64_t(1) << 21;  // 8 MB of int32: M * N <= 2^21
+__device__ __align__(16) int32_t g_splitk_acc[kSplitAccElems];  // read as int4 vectors
+
+// thread = 8 consecutive features of one token (N % 8 == 0)
+template <int ACT>
+__global__ void __launch_bounds__(256)
+    splitk_finish_kernel(int32_t *__restrict__ acc, const float *__restrict__ scales,
+                         const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
+                         int M, int N, int32_t *__restrict__ acc_out,
+                         __nv_bfloat16 *__restrict__ Y) {
+    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;  // group of 8 features
+    const int64_t groups = (int64_t)M * (N / 8);
+    if (i >= groups) return;
+    const int64_t m = i / (N / 8);
+    const int n0 = (int)(i - m * (N / 8)) * 8;
+    int4 *src = reinterpret_cast<int4 *>(acc + m * N + n0);
+    const int4 a0 = src[0], a1 = src[1];
+    src[0] = make_int4(0, 0, 0, 0);  // the scratch is zero again for the next call
+    src[1] = make_int4(0, 0, 0, 0);
+    const int rs = rowsum[m];
+    const int v[8] = {a0.x - rs, a0.y - rs, a0.z - rs, a0.w - rs,
+                      a1.x - rs, a1.y - rs, a1.z - rs, a1.w - rs};
+    if (acc_out) {
+        int4 *dst = reinterpret_cast<int4 *>(acc_out + m * N + n0);
+        dst[0] = make_int4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_int4(v[4], v[5], v[6], v[7]);
+    }
+    if (!Y) return;
+    const float sc = scales[m] * *gamma_ptr;
+    if constexpr (ACT == OUT_SWIGLU) {
+        uint32_t pk[2];
+#pragma unroll
+        for (int i2 = 0; i2 < 2; ++i2) {
+            float o[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float g = (float)v[4 * i2 + 2 * e] * sc;
+                const float u = (float)v[4 * i2 + 2 * e + 1] * sc;
+                o[e] = __fdiv_rn(g, 1.f + expf(-g)) * u;
+            }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
+            pk[i2] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint2 *>(Y + m * (N / 2) + n0 / 2) = make_uint2(pk[0], pk[1]);
+    } else {
+        uint32_t pk[4];
+#pragma unroll
+        for (int i2 = 0; i2 < 4; ++i2) {
+            float y0 = (float)v[2 * i2] * sc, y1 = (float)v[2 * i2 + 1] * sc;
+            if constexpr (ACT == OUT_RELU2) {
+                y0 = y0 > 0.f ? y0 * y0 : 0.f;
+                y1 = y1 > 0.f ? y1 * y1 : 0.f;
+            }
+            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+            pk[i2] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(Y + m * N + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
+// Chunks per tile for the K split, or 1 for the one-pass kernel: only when fewer than half of the
+// pairs would get a tile, the K axis has at least two stages and the output fits the scratch.
+static int choose_split(int64_t tiles, int64_t M, int64_t N, int64_t K, int pairs_max) {
+    const int64_t KS = (K + BK - 1) / BK;
+    if (tiles * 2 > pairs_max || KS < 2 || M * N > kSplitAccElems) return 1;
+    int64_t split = pairs_max / tiles;
+    if (split > KS) split = KS;
+    return split < 2 ? 1 : (int)split;
+}
+
+template <int BITS>
+static cudaError_t launch_split(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
+                                int64_t tiles, int split, int num_sms, cudaStream_t stream) {
+    int32_t *acc = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&acc), g_splitk_acc);
+    if (e != cudaSuccess) return e;
+    CUtensorMap unused;
+    memset(&unused, 0, sizeof unused);
+    e = launch_tc_t<BITS, OUT_PARTIAL>(a, mc, mw, unused, acc, tiles, num_sms, stream, split);
+    if (e != cudaSuccess) return e;
+    const int64_t groups = a.M * (a.N / 8);
+    const unsigned blocks = (unsigned)((groups + 255) / 256);
+    auto *Y = reinterpret_cast<__nv_bfloat16 *>(a.Y);
+    switch (a.Y ? a.activation : 0) {
+        case 1:
+            splitk_finish_kernel<OUT_RELU2><<<blocks, 256, 0, stream>>>(
+                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
+            break;
+        case 2:
+            splitk_finish_kernel<OUT_SWIGLU><<<blocks, 256, 0, stream>>>(
+                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
+            break;
+        default:
+            splitk_finish_kernel<OUT_BF16><<<blocks, 256, 0, stream>>>(
+                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace tc
@@ -557,7 +706,7 @@ static CUresult encode_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType
 }
 
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, int *launches) {
     using namespace tc;
     const int64_t tiles = ((a.N + BN - 1) / BN) * ((a.M + BM - 1) / BM);
     CUtensorMap mc, mw, my;
@@ -578,6 +727,15 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
                   CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
+    const int split = choose_split(tiles, a.M, a.N, a.K,
+                                   a.act_bits == 8 ? max_pairs<8, OUT_PARTIAL>(num_sms)
+                                                   : max_pairs<4, OUT_PARTIAL>(num_sms));
+    if (split > 1) {
+        if (launches) *launches = 2;
+        return a.act_bits == 8 ? launch_split<8>(a, mc, mw, tiles, split, num_sms, stream)
+                               : launch_split<4>(a, mc, mw, tiles, split, num_sms, stream);
+    }
+    if (launches) *launches = (a.Y ? 1 : 0) + (a.acc ? 1 : 0);
     if (a.Y) {
         // bf16 output [M rows][N] (N/2 with SwiGLU), one [32 tokens x 16 features] box per
         // store, 32-byte swizzle

@@ -79,7 +79,7 @@ cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream);
 
 // tcgen05 tensor-core kernel (prefill).  encode is cuTensorMapEncodeTiled.
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, int *launches = nullptr);
 
 // ---- failure detection self-test (selftest.cu) ----
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, int *status,

@@ -164,6 +164,11 @@ int bitnet_norm_transform_f32(const void *X_dev, int64_t M, int64_t K, const voi
  * bitnet_quantize_pack_weights.  acc_dev (int32 [M, N]) and Y_dev (bf16 [M, N]) are each
  * optional (NULL to skip); at least one must be given.  Large M runs on the tcgen05 tensor
  * cores, small M (decode) on a weight-streaming kernel; both give the same integers.
+ * When M > 8 but the output has few 256 x 256 tiles (fewer than half the GPU's SM pairs) and
+ * M * N <= 2^21, the tensor-core product splits K across SM pairs and sums the int32 partials in
+ * a library-owned scratch (8 MB per device, zero between calls); two such calls on one device
+ * must not run at the same time on the GPU (issue them on one stream, or order them).  The same
+ * holds for the forward and activation entries below, which use this product.
  */
 int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
                         const int32_t *rowsum_dev, int64_t M, int64_t K, const void *Wp_dev,

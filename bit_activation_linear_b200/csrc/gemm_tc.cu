@@ -40,6 +40,9 @@
 //                them with bulk tensor stores.  (Direct stores of one row per thread touch 32
 //                lines per instruction; on B200 they held up the unpack warps' shared-memory
 //                stores for ~6000 cycles per tile.)
+// Work: a persistent grid of pairs walks units; a unit is one tile (one pass over K) or, with
+// few tiles, one K chunk of a tile whose int32 sums are added atomically into a scratch and
+// finished by splitk_finish_kernel (see the K split section below).
 // Commits multicast to both CTAs; every wait is bounded: after ~1 s a role records
 // BITNET_ERR_TIMEOUT and stops; in-flight copies and MMAs are drained and both CTAs meet at a
 // cluster barrier before tensor memory is released.  No TMA multicast is used.

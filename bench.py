@@ -27,6 +27,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -116,7 +117,9 @@ class ClockSampler:
         self.path = None
 
     def start(self):
-        out_dir = os.path.join(ROOT, "gpurun_out")
+        # the raw samples go to $BITNET_BENCH_OUT (default: the system temporary directory); the
+        # JSON line carries their summary
+        out_dir = os.environ.get("BITNET_BENCH_OUT", tempfile.gettempdir())
         os.makedirs(out_dir, exist_ok=True)
         self.path = os.path.join(out_dir, f"bench_clocks_rank{self.idx}.csv")
         try:

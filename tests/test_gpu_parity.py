@@ -155,6 +155,7 @@ def staged_product(B, M, K, N, bits, seed):
     (8, 16384, 520), (4, 32768, 16),                        # (17 steps: uneven split)
     (7, 4096, 8200),                                        # decode, 4-row groups
     (9, 256, 256), (130, 384, 136), (300, 2048, 264),       # tensor-core kernel, ragged tiles
+    (64, 8192, 2048), (17, 4096, 1032),                     # tensor cores with the K split
     (256, 1024, 1024), (513, 128, 8),
     (1000, 640, 520),                                       # several tiles, 2.5 K stages
 ])

@@ -4,16 +4,18 @@
 A step is one pass of the whole forward over one batch of synthetic input: absmean
 ternarisation + packing of the latent weights (2 kernels), the fused Hadamard + absmax INT8
 quantisation of the tokens (1 kernel) and the ternary x int8 tensor-core product with the bf16
-rescale (1 kernel).  Default workload: the Wo-shaped layer of a 2B-class model
-(M = 4096 tokens, K = N = 2048, H-BitLinear, INT8 activations).
+rescale (1 kernel).  Default workload: the 7B-scale down projection, the largest layer of the
+pages' workloads that one GPU holds (M = 16384 tokens, K = 16384, N = 4096, H-BitLinear, INT4
+activations).
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier and
 cuda.synchronize on both sides, timed with CUDA events on the launching stream, max over ranks.
 Inputs are rotated over several copies whose total exceeds twice the L2 cache, so no step finds
 its inputs in L2.  Each copy's step is one CUDA graph, so host launch overhead does not starve
 the GPU: the weight ternarisation and the activation quantisation run side by side on two
-streams (they are independent), then the tensor-core product, bracketed by two timing events
-that are nodes of the same graph; they give the product's live duration for the roofline figure.
+streams (they are independent), then the tensor-core product.  The last few timed steps replay
+a copy of their graph in which two timing events bracket the product; those events give the
+product's live duration for the roofline figure.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the data
@@ -41,7 +43,7 @@ sys.path.insert(0, ROOT)
 from bit_activation_linear_b200 import synth  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic_wo_2048.json")
+PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
 METRIC = "H-BitLinear tokens/s and effective int8 TOPS (% of roofline) on 1 B200"
@@ -85,11 +87,12 @@ def kernel_work(wl, base3: bool = False, rotate: bool = False):
 
 
 def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch (read + write) from the committed ncu capture, or None when the
-    capture is for another workload or the kernel's source changed since it was taken."""
+    """DRAM bytes per launch (read + write) from the committed ncu capture of this workload
+    (profiles/ncu_traffic_<workload>.json), or None when there is none or the kernel's source
+    changed since it was taken."""
     import hashlib
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(os.path.join(PROFILES, f"ncu_traffic_{workload}.json")) as f:
             cap = json.load(f)
     except (OSError, ValueError):
         return None
@@ -372,44 +375,43 @@ def run_gpu(args, wl, rank, world, device):
 
     # One CUDA graph per input copy holds the whole step.  Timing-event nodes inside a graph
     # cost ~5 us per step on B200, so the timed loop replays event-free graphs, except for its
-    # last copies x SAMPLES steps: each of those replays, once, its own copy of the step graph
+    # last n_timed (at most SAMPLES) steps: each of those replays its own copy of the step graph
     # whose product is bracketed by two timing events.  Those events give the product's live
-    # duration inside the timed region.
+    # duration inside the timed region, at a fixed cost of a few microseconds per run.
     SAMPLES = 4
-    graphs, timed = [], []
+    graphs = []
     for b in bufs:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             prep(b)
             gemm(b)
         graphs.append(g)
-        copy_timed = []
-        for _ in range(SAMPLES):
-            gt = torch.cuda.CUDAGraph()
-            ev = (torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True))
-            with torch.cuda.graph(gt, stream=stream):
-                prep(b)
-                ev[0].record(stream)
-                gemm(b)
-                ev[1].record(stream)
-            copy_timed.append((gt, ev))
-        timed.append(copy_timed)
+    n_timed = min(args.steps, SAMPLES)
+    first_timed = args.steps - n_timed
+    timed = {}  # step index -> (graph, (start event, end event))
+    for i in range(first_timed, args.steps):
+        b = bufs[i % copies]
+        gt = torch.cuda.CUDAGraph()
+        ev = (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True))
+        with torch.cuda.graph(gt, stream=stream):
+            prep(b)
+            ev[0].record(stream)
+            gemm(b)
+            ev[1].record(stream)
+        timed[i] = (gt, ev)
     torch.cuda.synchronize(device)
-    n_timed = min(args.steps, copies * SAMPLES)
 
     def step(i, sampled=False):
-        if sampled:  # the j-th sampled step of copy i % copies uses that copy's j-th timed graph
-            j = (i - (args.steps - n_timed)) // copies
-            timed[i % copies][j][0].replay()
+        if sampled:
+            timed[i][0].replay()
         else:
             graphs[i % copies].replay()
 
     for i in range(args.warmup):
         step(i)
-    for copy_timed in timed:  # first replays upload the sampled graphs outside the timed region
-        for gt, _ in copy_timed:
-            gt.replay()
+    for gt, _ in timed.values():  # first replays upload the sampled graphs outside the timed region
+        gt.replay()
     torch.cuda.synchronize(device)
     B.bitnet_sync_status(stream)
 
@@ -424,7 +426,7 @@ def run_gpu(args, wl, rank, world, device):
     torch.cuda._sleep(int(2e7))
     t_start.record(stream)
     for i in range(args.steps):
-        step(i, sampled=i >= args.steps - n_timed)
+        step(i, sampled=i >= first_timed)
     t_end.record(stream)
     torch.cuda.synchronize(device)
     barrier()
@@ -433,11 +435,7 @@ def run_gpu(args, wl, rank, world, device):
 
     elapsed_ms = t_start.elapsed_time(t_end)
     # the product's duration in each sampled step (all inside the timed region)
-    samples = []
-    for i in range(args.steps - n_timed, args.steps):
-        j = (i - (args.steps - n_timed)) // copies
-        ev = timed[i % copies][j][1]
-        samples.append(ev[0].elapsed_time(ev[1]))
+    samples = [ev[0].elapsed_time(ev[1]) for _, ev in timed.values()]
     gemm_ms = statistics.mean(samples)
     elapsed_ms = aggregate_max(elapsed_ms, device)
     gemm_ms = aggregate_max(gemm_ms, device)
@@ -466,7 +464,7 @@ def run_gpu(args, wl, rank, world, device):
     ms_per_step = elapsed_ms / args.steps
 
     # end to end through the public API: pinned host X and W in, Y out, every step
-    e2e = run_e2e(args, wl, B, stream, device, X0, W0)
+    e2e = None if args.no_e2e else run_e2e(args, wl, B, stream, device, X0, W0)
 
     if rank == 0:
         peaks, peak_kind = load_peaks()
@@ -526,11 +524,16 @@ def run_gpu(args, wl, rank, world, device):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "int8",
+            # the activation code width; the tensor cores contract int8 operands (INT4 codes are
+            # widened on chip) into int32 accumulators
+            "dtype": f"int{wl.act_bits}",
             "data": "synthetic",
             "effective_tops": world * wl.ops / (ms_per_step * 1e-3) / 1e12,
             "config": {"workload": wl.name, "M": M, "K": K, "N": N, "hadamard": wl.hadamard,
-                       "act_bits": wl.act_bits, "rmsnorm": bool(args.rmsnorm),
+                       "act_bits": wl.act_bits,
+                       "contraction": "ternary weights x int8 operands (tcgen05 kind::i8), "
+                                      "int32 accumulate, bf16 out",
+                       "rmsnorm": bool(args.rmsnorm),
                        "activation": args.activation,
                        "weights": "base3" if args.base3 else "2bit",
                        "act_scale": "absmean" if args.absmean4 else "absmax",
@@ -655,7 +658,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
-    ap.add_argument("--workload", default="wo_2048", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="down_7b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--activation", default="none", choices=["none", "relu2", "swiglu"],
                     help="activation in the product's epilogue (squared ReLU, SwiGLU)")
@@ -671,6 +674,8 @@ def main():
                     help="weight + activation Hadamard rotation: ternarise the rotated weight "
                          "rows (H-BitLinear workloads)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (e.g. to keep a profiler capture small)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:

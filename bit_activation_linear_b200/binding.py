@@ -21,6 +21,7 @@ _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
 ACT_RELU2, ACT_SWIGLU = 1, 2  # bitnet_activation
+PATH_DECODE, PATH_TC, PATH_TC_KSPLIT = 1, 2, 3  # bitnet_product_path
 
 
 class BitnetError(RuntimeError):
@@ -59,6 +60,9 @@ _SIGS = {
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "bitnet_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                                  ctypes.c_int]),
+    "bitnet_product_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_int)]),
     "bitnet_bitlinear_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
@@ -194,6 +198,14 @@ def bitnet_act_codes_bytes(M: int, K: int, act_bits: int) -> int:
 
 def bitnet_workspace_bytes(M: int, K: int, N: int, act_bits: int) -> int:
     return int(load_library().bitnet_workspace_bytes(M, K, N, act_bits))
+
+
+def bitnet_product_plan(M: int, K: int, N: int, act_bits: int):
+    """(path, k_split) of the product of this shape on the current device (PATH_* values)."""
+    path, split = ctypes.c_int(0), ctypes.c_int(0)
+    _rc(load_library().bitnet_product_plan(M, K, N, int(act_bits), ctypes.byref(path),
+                                           ctypes.byref(split)), "bitnet_product_plan")
+    return path.value, split.value
 
 
 def bitnet_quantize_pack_weights(W: torch.Tensor, Wp: torch.Tensor | None = None,

@@ -425,6 +425,26 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
                      acc_dev, Y_dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path,
+                        int *k_split) {
+    int rc = check_shape(M, K, N, true, true);
+    if (rc) return rc;
+    if (act_bits != 8 && act_bits != 4)
+        return fail(BITNET_ERR_INVALID, "act_bits = %d must be 8 or 4", act_bits);
+    if (!path || !k_split) return fail(BITNET_ERR_INVALID, "null pointer argument");
+    DeviceState *st = nullptr;
+    if ((rc = device_state(&st))) return rc;
+    if (M <= kGemvMaxTokens) {
+        *path = BITNET_PATH_DECODE;
+        *k_split = 1;
+        return BITNET_OK;
+    }
+    const int split = ternary_gemm_tc_split(M, N, K, act_bits, st->num_sms);
+    *path = split > 1 ? BITNET_PATH_TC_KSPLIT : BITNET_PATH_TC;
+    *k_split = split;
+    return BITNET_OK;
+}
+
 size_t bitnet_workspace_bytes(int64_t M, int64_t K, int64_t N, int act_bits) {
     (void)N;
     if (M <= 0 || K <= 0) return 0;

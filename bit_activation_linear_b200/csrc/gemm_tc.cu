@@ -708,6 +708,14 @@ static CUresult encode_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+int ternary_gemm_tc_split(int64_t M, int64_t N, int64_t K, int act_bits, int num_sms) {
+    using namespace tc;
+    const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
+    return choose_split(tiles, M, N, K,
+                        act_bits == 8 ? max_pairs<8, OUT_PARTIAL>(num_sms)
+                                      : max_pairs<4, OUT_PARTIAL>(num_sms));
+}
+
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream, int *launches) {
     using namespace tc;

@@ -80,6 +80,8 @@ cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream);
 // tcgen05 tensor-core kernel (prefill).  encode is cuTensorMapEncodeTiled.
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream, int *launches = nullptr);
+// The K split launch_ternary_gemm_tc takes for this shape on the current device (1: one pass).
+int ternary_gemm_tc_split(int64_t M, int64_t N, int64_t K, int act_bits, int num_sms);
 
 // ---- failure detection self-test (selftest.cu) ----
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, int *status,

@@ -176,6 +176,23 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
                         void *Y_dev, bitnet_stream_t stream);
 
 /*
+ * Which kernel the product of an M x K by N x K shape takes on the current device (a query of
+ * the library; the pages have no counterpart).  Every path gives the same integers.
+ *   *path    BITNET_PATH_DECODE    weight-streaming kernel (M <= 8 tokens);
+ *            BITNET_PATH_TC        tensor-core kernel, one pass over K per 256 x 256 tile;
+ *            BITNET_PATH_TC_KSPLIT tensor-core kernel with K cut into *k_split chunks.
+ *   *k_split chunks of K per output tile (1 unless BITNET_PATH_TC_KSPLIT).
+ * Shape and act_bits rules and errors as bitnet_ternary_gemm; enqueues nothing.
+ */
+typedef enum {
+    BITNET_PATH_DECODE = 1,
+    BITNET_PATH_TC = 2,
+    BITNET_PATH_TC_KSPLIT = 3
+} bitnet_product_path;
+
+int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path, int *k_split);
+
+/*
  * Activations fused into the product's epilogue, for the up / gate projections that feed the
  * FFN (BitNet b1.58 2B4T article, section 一.3: squared ReLU; BitNet v2 write-up: SwishGLU).
  * With y = float(acc) * (scales[m] * gamma) as in bitnet_ternary_gemm:

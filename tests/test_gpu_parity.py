@@ -9,6 +9,8 @@ Tolerances (written here, from the contract of the forward):
   * bf16 output: elementwise relative error <= 1e-2 against the oracle fed the same codes, and
     ||Y - Y_ref||_F / ||Y_ref||_F <= 1e-2 against the fully independent oracle.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -171,25 +173,98 @@ def test_product_int32_exact_and_bf16(B, M, K, N, bits):
     assert np.all(y[y_ref == 0] == 0)
 
 
+def sample_rows(M, count, seed):
+    """A seeded sorted sample of token rows that always holds the first and the last row (the
+    ragged tail of the last tile)."""
+    if count is None or count >= M:
+        return np.arange(M)
+    rows = np.random.default_rng(seed).choice(np.arange(1, M - 1), size=count - 2, replace=False)
+    return np.sort(np.concatenate([[0, M - 1], rows]))
+
+
+def codes_rows(codes, rows, K, bits):
+    c = codes[torch.from_numpy(rows).to(codes.device)].cpu().numpy()
+    return c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+
+
+# The one-pass tensor-core product at the sizes the benchmark runs: many K stages per tile
+# (the operand rings wrap), more tiles than SM pairs (the persistent tile loop and both
+# accumulator buffers of tensor memory are used), ragged token and feature tails, and a half
+# last stage (K % 256 == 128).  int32 bit-exact on a seeded sample of rows x all features;
+# bf16 elementwise on the same rows.
+@pytest.mark.parametrize("M,K,N,bits,name", [
+    (4096, 2048, 2048, 8, "wo_2048"),
+    (8192, 8192, 2048, 4, "wdown_8192"),
+    (16384, 16384, 4096, 4, "down_7b"),
+    (4000, 2048, 2056, 8, None),
+    (3000, 1152, 3080, 4, None),
+])
+def test_product_one_pass_full_size_bit_exact(B, M, K, N, bits, name):
+    path, split = B.bitnet_product_plan(M, K, N, bits)
+    assert (path, split) == (B.PATH_TC, 1), "this shape must take the one-pass kernel"
+    if name is not None:
+        wl = synth.WORKLOADS[name]
+        X, W = wl.activations(seed=3), wl.weights(seed=3)
+    else:
+        X = synth.sharp_activations(M, K, seed=M + K)
+        W = synth.latent_weights(N, K, seed=N + K)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    hadamard = (K & (K - 1)) == 0
+    Xd = dev_bf16(X)
+    del X
+    codes, scales, rowsum = B.bitnet_act_quant(Xd, hadamard, bits)
+    acc, Y = B.bitnet_ternary_gemm(codes, scales, rowsum, K, Wp, gamma, bits, want_acc=True,
+                                   want_y=True)
+    B.bitnet_sync_status()
+    rows = sample_rows(M, 64, seed=M)
+    sel = torch.from_numpy(rows).cuda()
+    c = codes_rows(codes, rows, K, bits)
+    q, bad = oracle.unpack_ternary(Wp.cpu().numpy().view(np.uint32), K)
+    assert bad == 0
+    acc_ref = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(acc[sel].cpu().numpy().astype(np.int64), acc_ref)
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc_ref, scales[sel].cpu().numpy(),
+                                              np.float32(gamma.item())))
+    y = oracle.bf16_to_f64(to_np_bits(Y[sel]))
+    rel = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), 1e-30)
+    assert np.all((rel <= Y_REL) | (y_ref == 0)), rel.max()
+    assert np.all(y[y_ref == 0] == 0)
+
+
 # ----------------------------------------------------------------------------------------
 # the whole layer against the independent oracle, on every workload shape
 # ----------------------------------------------------------------------------------------
 
-def forward_case(B, wl, sample_rows, seed=0):
+def forward_case(B, wl, sample_count, seed=0):
+    """The GPU forward against the fully independent oracle on sampled rows.
+
+    Besides the Frobenius bound, every sampled element is checked: the GPU's codes may differ
+    from the oracle's by +-1 at near-ties (the GPU's fp32 transform is not the oracle's double
+    one), and each such code moves an accumulator by at most 1, i.e. y by at most d * gamma.
+    So |y - y_ref| <= Y_REL |y_ref| + flips(m) * d_m * gamma, flips(m) being the number of
+    codes of row m that differ (themselves held to the code tolerance)."""
     X = wl.activations(seed=seed)
     W = wl.weights(seed=seed)
     Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
     fwd = B.bitnet_hbitlinear_forward if wl.hadamard else B.bitnet_bitlinear_forward
-    Y = fwd(dev_bf16(X), Wp, gamma, wl.act_bits)
+    Xd = dev_bf16(X)
+    Y = fwd(Xd, Wp, gamma, wl.act_bits)
+    codes, _, _ = B.bitnet_act_quant(Xd, wl.hadamard, wl.act_bits)  # the forward's own codes
     B.bitnet_sync_status()
-    rows = np.arange(wl.M) if sample_rows is None else np.sort(
-        np.random.default_rng(seed).choice(wl.M, size=sample_rows, replace=False))
+    rows = sample_rows(wl.M, sample_count, seed)
     ref = oracle.bitlinear_forward(X[rows], W, wl.hadamard, wl.act_bits)
     assert np.float32(gamma.item()) == ref["gamma"]
+    c = codes_rows(codes, rows, wl.K, wl.act_bits)
+    _, _, pre, _ = oracle.quant_act(ref["z"].astype(np.float32), wl.act_bits)
+    check_codes(c, ref["codes"], pre)
+    flips = (c != ref["codes"]).sum(axis=1)
     y = oracle.bf16_to_f64(to_np_bits(Y)[rows])
     y_ref = oracle.bf16_to_f64(ref["y"])
     fro = np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref)
     assert fro <= Y_REL, fro
+    slack = flips[:, None] * ref["d"][:, None].astype(np.float64) * float(ref["gamma"])
+    bound = Y_REL * np.abs(y_ref) + slack * (1 + 1e-6)
+    assert np.all(np.abs(y - y_ref) <= bound), np.abs(y - y_ref).max()
     return fro
 
 
@@ -207,6 +282,164 @@ def test_forward_end_to_end(B, name, rows):
 @pytest.mark.parametrize("name,rows", [("down_7b", 6), ("up_7b", 8)])
 def test_forward_end_to_end_7b(B, name, rows):
     forward_case(B, synth.WORKLOADS[name], rows)
+
+
+# ----------------------------------------------------------------------------------------
+# the method's edge cases on the GPU
+# ----------------------------------------------------------------------------------------
+
+def bf16_exact(a):
+    """bf16 bits of values that bf16 holds exactly (asserted)."""
+    a = np.asarray(a, np.float32)
+    bits = synth.f32_to_bf16_bits(a)
+    assert np.array_equal(oracle.bf16_to_f64(bits), a.astype(np.float64))
+    return bits
+
+
+def test_weights_on_the_ternary_threshold(B):
+    """Weights exactly at |w| = gamma / 2 and at the bf16 neighbours of that value.
+
+    3/8 of the weights are +-1, half are +-1/4 and 1/8 are zero, so gamma = 1/2 exactly and
+    1/4 lies on the threshold: w / gamma = 0.5 rounds to the even 0.  Triples (1/4 + 2^-9,
+    1/4 - 2^-10, 1/4 - 2^-10) keep the sum, and so gamma, unchanged: the first is the bf16 value
+    just above the threshold (code +-1), the others just below it (code 0)."""
+    N, K = 64, 256
+    rng = np.random.default_rng(21)
+    kinds = np.array([1.0] * 3 + [0.25] * 4 + [0.0])          # per 8 weights
+    w = np.stack([rng.permutation(kinds) for _ in range(N * K // 8)]).reshape(N, K)
+    flat = w.reshape(-1)
+    quarter = np.flatnonzero(flat == 0.25)
+    trip = rng.choice(quarter, size=(300, 3), replace=False)
+    flat[trip[:, 0]] = 0.25 + 2.0 ** -9
+    flat[trip[:, 1:]] = 0.25 - 2.0 ** -10
+    sign = np.where(rng.random(flat.shape) < 0.5, -1.0, 1.0)
+    W = bf16_exact((flat * sign).reshape(N, K))
+    g_ref = oracle.absmean_gamma(W)
+    assert g_ref == np.float32(0.5)
+    q_ref = oracle.ternarize(W, g_ref)
+    a = np.abs(oracle.bf16_to_f64(W))
+    assert np.all(q_ref[a == 0.25] == 0) and np.all(q_ref[a == 0.25 - 2.0 ** -10] == 0)
+    assert np.all(np.abs(q_ref[a == 0.25 + 2.0 ** -9]) == 1)
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    B.bitnet_sync_status()
+    assert np.float32(gamma.item()) == g_ref
+    np.testing.assert_array_equal(Wp.cpu().numpy().view(np.uint32).reshape(N, K // 16),
+                                  oracle.pack_ternary(q_ref))
+
+
+def test_weights_near_the_threshold_of_a_random_gamma(B):
+    """A random matrix whose gamma is not a power of two, with probes at the bf16 values around
+    gamma / 2, where the fp32 division w / gamma decides between 0 and +-1 by one rounding."""
+    N, K = 256, 1024
+    W = synth.latent_weights(N, K, seed=33)
+    probes = np.random.default_rng(33).choice(N * K, size=4096, replace=False)
+    for _ in range(6):  # settle gamma: the probes' own magnitudes move it slightly
+        g = float(oracle.absmean_gamma(W))
+        h = np.float32(g / 2)
+        nb = synth.f32_to_bf16_bits(np.array([h], np.float32)).astype(np.int32)[0] & 0x7FFF
+        cand = np.array([nb - 2, nb - 1, nb, nb + 1, nb + 2], np.int32)
+        mags = cand[np.arange(probes.size) % 5]
+        signs = np.where(np.arange(probes.size) % 2 == 0, 0, 0x8000)
+        flat = W.reshape(-1).copy()
+        flat[probes] = (mags | signs).astype(np.uint16)
+        W = flat.reshape(N, K)
+    g_ref = oracle.absmean_gamma(W)
+    q_ref = oracle.ternarize(W, g_ref)
+    a = np.abs(oracle.bf16_to_f64(W.reshape(-1)[probes]))
+    qa = np.abs(q_ref.reshape(-1)[probes])
+    # the probes straddle the threshold: some decide 0, some +-1, within two bf16 steps
+    assert (qa == 0).any() and (qa == 1).any()
+    assert a.max() / a.min() < 1.04
+    Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+    B.bitnet_sync_status()
+    assert np.float32(gamma.item()) == g_ref
+    np.testing.assert_array_equal(Wp.cpu().numpy().view(np.uint32).reshape(N, K // 16),
+                                  oracle.pack_ternary(q_ref))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_activation_codes_at_exact_ties_plain(B, bits):
+    """Plain rows with max |x| = Q/2 or Q/4, so s = 2 or 4 exactly, and every other x equal to
+    (k + 1/2) / s: x * s lands exactly on a .5 for each of them.  The codes must round half to
+    even, as the oracle does, with zero differences."""
+    Q = 127 if bits == 8 else 7
+    K = 256
+    rng = np.random.default_rng(bits)
+    rows = []
+    for s in (2, 4):
+        x = (rng.integers(-Q, Q, size=K) + 0.5) / s       # x * s = k + 1/2, |k + 1/2| < Q
+        x[rng.integers(K)] = Q / s
+        rows.append(x)
+    X = bf16_exact(np.stack(rows))
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), False, bits)
+    B.bitnet_sync_status()
+    z = oracle.bf16_to_f64(X).astype(np.float32)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
+    assert (pre - np.floor(pre) == 0.5).sum() > K  # most elements are exact ties
+    np.testing.assert_array_equal(codes_rows(codes, np.arange(2), K, bits), c_ref)
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
+
+
+def hadamard_rows_from_z(z_rows, K):
+    """x = H z / sqrt(K), so that the transform gives back z exactly (H H = K I)."""
+    H = np.array([[(-1) ** bin(i & j).count("1") for j in range(K)] for i in range(K)], np.float64)
+    return (np.asarray(z_rows, np.float64) @ H) / math.sqrt(K)
+
+
+def test_activation_codes_at_exact_ties_hadamard(B):
+    """H-BitLinear rows built so that z = 63.5 e_0 + 0.25 e_a + 0.75 e_b (signs varied): every x is
+    a bf16 value, the fp32 transform is exact, s = 127 / 63.5 = 2, and z * s = 127, 0.5, 1.5,
+    which round to 127, 0 and 2."""
+    K = 256
+    rng = np.random.default_rng(5)
+    zs = []
+    for t in range(12):
+        z = np.zeros(K)
+        a, b = rng.choice(np.arange(1, K), size=2, replace=False)
+        z[0] = 63.5 * (1 if t % 2 == 0 else -1)
+        z[a] = 0.25 * (1 if t % 3 else -1)
+        z[b] = 0.75 * (1 if t % 4 < 2 else -1)
+        zs.append(z)
+    X = bf16_exact(hadamard_rows_from_z(zs, K))
+    Xd = dev_bf16(X)
+    Z = B.bitnet_fwht_f32(Xd).cpu().numpy().astype(np.float64)
+    np.testing.assert_array_equal(Z, np.array(zs))
+    codes, scales, rowsum = B.bitnet_act_quant(Xd, True, 8)
+    B.bitnet_sync_status()
+    ref = oracle.bitlinear_forward(X, synth.latent_weights(8, K, seed=1), True, 8)
+    c = codes.cpu().numpy().view(np.int8)
+    np.testing.assert_array_equal(c, ref["codes"])
+    expect = np.rint(np.array(zs) * 2).astype(np.int8)  # numpy rint: half to even
+    np.testing.assert_array_equal(c, expect)
+    assert set(np.unique(np.abs(expect))) == {0, 2, 127}
+    np.testing.assert_array_equal(scales.cpu().numpy(), ref["d"])
+
+
+@pytest.mark.parametrize("K", [256, 2048, 8192])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_single_spike_and_constant_rows(B, K, bits):
+    """x = c * (column j of H): z = c sqrt(K) e_j, one non-zero; a constant row is the j = 0
+    case.  Codes are the oracle's (Q or the clipped absmean code at j, zero elsewhere), bit for
+    bit, and the scales match."""
+    js = [0, 1, K // 2 + 3, K - 1]
+    rows = []
+    for t, j in enumerate(js):
+        col = np.array([(-1) ** bin(i & j).count("1") for i in range(K)], np.float64)
+        rows.append((0.5 if t % 2 == 0 else -0.125) * col)
+    rows.append(np.full(K, 0.75))                          # constant row
+    X = bf16_exact(np.stack(rows))
+    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), True, bits)
+    B.bitnet_sync_status()
+    ref = oracle.bitlinear_forward(X, synth.latent_weights(8, K, seed=2), True, bits)
+    c = codes_rows(codes, np.arange(len(rows)), K, bits)
+    np.testing.assert_array_equal(c, ref["codes"])
+    for t, j in enumerate(js + [0]):
+        nz = np.flatnonzero(c[t])
+        assert list(nz) == [j]
+    # 1/sqrt(K) is inexact for odd powers of two: the scale may differ in its last bit
+    np.testing.assert_allclose(scales.cpu().numpy(), ref["d"], rtol=1e-6)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), c.astype(np.int64).sum(axis=1))
 
 
 def test_forward_equals_staged_calls(B):

@@ -301,6 +301,36 @@ def test_quant_brute_force_nearest_and_extremes(bits, Q):
     assert np.all(err[live] <= 0.5 * d[live, None] * (1 + 1e-6))
 
 
+@pytest.mark.parametrize("bits,Q", [(8, 127), (4, 7)])
+def test_quant_pre_at_exact_ties(bits, Q):
+    """Rows whose max |z| is Q/2 or Q/4 have s = 2 or 4 exactly, so z * s is exact and known:
+    ``pre`` must equal those closed-form values and every x.5 must round to the even integer.
+    A dropped factor, a wrong scale or a round-half-away rule fails here."""
+    z = np.zeros((3, 16), np.float32)
+    # s = 2: pre = 2 z
+    z[0, :10] = [Q / 2, 0.25, 0.75, -0.25, -0.75, 1.25, -1.75, 0.125, 1.0, -Q / 2]
+    # s = 4: pre = 4 z
+    z[1, :8] = [Q / 4, 0.125, 0.375, 0.625, -0.875, 0.0625, -Q / 4, 0.25]
+    z[2, 0] = -Q / 2                      # one non-zero: pre = -Q at 0, zero elsewhere
+    codes, d, pre, rowsum = oracle.quant_act(z, bits)
+    exp_pre = np.zeros((3, 16))
+    exp_pre[0, :10] = [Q, 0.5, 1.5, -0.5, -1.5, 2.5, -3.5, 0.25, 2.0, -Q]
+    exp_pre[1, :8] = [Q, 0.5, 1.5, 2.5, -3.5, 0.25, -Q, 1.0]
+    exp_pre[2, 0] = -Q
+    np.testing.assert_array_equal(pre, exp_pre)
+    exp_codes = np.zeros((3, 16), np.int64)
+    exp_codes[0, :10] = [Q, 0, 2, 0, -2, 2, -4, 0, 2, -Q]     # ties to even
+    exp_codes[1, :8] = [Q, 0, 2, 2, -4, 0, -Q, 1]
+    exp_codes[2, 0] = -Q
+    np.testing.assert_array_equal(codes, exp_codes)
+    np.testing.assert_array_equal(rowsum, exp_codes.sum(axis=1))
+    np.testing.assert_array_equal(d, np.float32([Q / 2, Q / 4, Q / 2]) / np.float32(Q))
+    # on random rows pre stays within half a step of its code
+    z = np.random.default_rng(bits + 40).laplace(size=(8, 512)).astype(np.float32)
+    codes, _, pre, _ = oracle.quant_act(z, bits)
+    assert np.all(np.abs(pre - codes) <= 0.5 + 1e-6)
+
+
 # ---- variant INT4 quantiser with an absmean scale (a reading: the pages name the INT4 strategy
 # without its formula; the form is that of the weights' absmean) ----
 

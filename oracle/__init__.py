@@ -69,7 +69,8 @@ def lib():
                 "oracle_fwht": (None, [vp, i64, i64, vp]),
                 "oracle_rmsnorm": (None, [vp, i64, i64, vp, f64, vp]),
                 "oracle_bitlinear_forward_norm": (i32, [vp, i64, i64, vp, i64, i32, i32, i32,
-                                                        vp, f64, vp, vp, vp, vp, vp, vp, vp]),
+                                                        i32, vp, f64, vp, vp, vp, vp, vp, vp,
+                                                        vp]),
                 "oracle_quant_act": (None, [vp, i64, i64, i32, vp, vp, vp, vp]),
                 "oracle_quant_act_absmean4": (None, [vp, i64, i64, vp, vp, vp, vp]),
                 "oracle_pack_int4": (None, [vp, i64, i64, vp]),
@@ -234,11 +235,19 @@ def fwht(x: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
-# Step 3: per-token absmax quantisation  (2B4T article, 一.2; BitNet v2 write-up, INT8/INT4)
+# Step 3: per-token quantisation  (2B4T article, 一.2: absmax for 8-bit activations; BitNet v2
+# write-up, INT8/INT4 paragraph: each width takes its own strategy -- absmean for INT4, the
+# reading taken here)
 # --------------------------------------------------------------------------------------
 
+def quant_act_for_bits(z_f32: np.ndarray, bits: int):
+    """The forward's quantiser for the width: absmax to INT8 (bits 8), absmean to INT4 (bits 4).
+    Returns (codes, d, pre, rowsum) as quant_act."""
+    return quant_act(z_f32, 8) if bits == 8 else quant_act_absmean4(z_f32)
+
+
 def quant_act(z_f32: np.ndarray, bits: int):
-    """Per-token absmax codes decided in fp32.
+    """Per-token absmax codes decided in fp32 (INT8; with bits 4, the absmax INT4 variant).
 
     Returns (codes int8 [M, K], d float32 [M], pre float64 [M, K], rowsum int64 [M]) where
     ``pre`` is the unrounded z * Q / max|z| in double.
@@ -254,8 +263,8 @@ def quant_act(z_f32: np.ndarray, bits: int):
 
 
 def quant_act_absmean4(z_f32: np.ndarray):
-    """Variant INT4 codes with a per-token absmean scale (the mean |z| maps to code sqrt(7)),
-    decided in fp32 and clipped to [-8, 7].
+    """INT4 codes with a per-token absmean scale (the mean |z| maps to code sqrt(7)), decided in
+    fp32 and clipped to [-8, 7]: the forward's INT4 quantiser.
 
     Returns (codes int8 [M, K], d float32 [M], pre float64 [M, K], rowsum int64 [M]) where
     ``pre`` is z * s in double, the value the rounding decides on.
@@ -346,8 +355,10 @@ def dequant_act(acc: np.ndarray, d: np.ndarray, gamma, act: int) -> np.ndarray:
 
 
 def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bits: int,
-                      norm_gain: np.ndarray | None = None, norm_eps: float | None = None):
-    """Y = (H-)BitLinear(X) from bf16 X [M, K] and latent bf16 W [N, K].  With norm_eps given,
+                      norm_gain: np.ndarray | None = None, norm_eps: float | None = None,
+                      int4_absmax: bool = False):
+    """Y = (H-)BitLinear(X) from bf16 X [M, K] and latent bf16 W [N, K].  bits 8: absmax INT8
+    codes; bits 4: absmean INT4 codes (int4_absmax: the absmax variant).  With norm_eps given,
     every token row is RMS-normalised first (gain norm_gain, bf16 bits [K], or unit gain).
 
     Returns a dict with every stage: gamma, q, z, codes, d, acc, y (uint16 bf16 bits).
@@ -365,7 +376,8 @@ def bitlinear_forward(x_bf16: np.ndarray, w_bf16: np.ndarray, hadamard: bool, bi
     acc = np.empty((M, N), dtype=np.int64)
     g = None if norm_gain is None else np.ascontiguousarray(norm_gain, dtype=np.uint16)
     rc = lib().oracle_bitlinear_forward_norm(
-        _p(X), M, K, _p(W), N, int(bool(hadamard)), int(bits), int(norm_eps is not None),
+        _p(X), M, K, _p(W), N, int(bool(hadamard)), int(bits), int(bool(int4_absmax)),
+        int(norm_eps is not None),
         None if g is None else _p(g), float(norm_eps or 0.0),
         _p(Y), _p(gamma), _p(q), _p(z), _p(codes), _p(d), _p(acc))
     if rc != 0:

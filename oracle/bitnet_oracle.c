@@ -30,10 +30,14 @@
  * Readings taken where the pages print no formula (each is listed in the design notes):
  *   gamma = fp32(max(mean|W|, 1e-5)) with the mean in double; q = clip(rint(w / gamma), -1, 1)
  *   with an fp32 IEEE division and round-half-even; Hadamard = Sylvester order, scaled by
- *   1/sqrt(K) (orthonormal), size K; activation quantiser = per-token absmax with Q = 127
- *   (INT8) or Q = 7 (INT4), eps 1e-5, round-half-even, clip to [-Q-1, Q]; output =
- *   bf16_rn(acc * d * gamma) with d = max|z| / Q.  Variant INT4 quantiser (not the default):
- *   absmean scale, the mean |z| of a token mapped to code sqrt(7), clipped to [-8, 7].
+ *   1/sqrt(K) (orthonormal), size K; output = bf16_rn(acc * d * gamma).
+ *   Activation quantisers: the [v2] write-up says INT8 and INT4 "respectively" take their own
+ *   strategy, and names absmax for the 4-bit activations of the post-training baselines only;
+ *   the pages name two quantisation functions, absmax (8-bit activations, [2B4T] 一.2) and
+ *   absmean ([b1.58]).  So INT8 = per-token absmax, Q = 127, eps 1e-5, round-half-even, clip to
+ *   [-128, 127], d = max|z| / 127; INT4 = per-token absmean, the mean |z| of a token mapped to
+ *   code sqrt(7), eps 1e-5, clip to [-8, 7], d = mean|z| / sqrt(7).  Variant INT4 quantiser
+ *   (not the default): absmax with Q = 7.
  *   Variant weight + activation rotation (not the default): the rows of W are transformed by
  *   the same orthonormal Hadamard before the absmean ternarisation, W' = W H / sqrt(K), so that
  *   W' (H x / sqrt(K)) = W x; the rotated rows are rounded to fp32 once, then ternarised.
@@ -307,10 +311,11 @@ void oracle_fwht(const double *x, int64_t M, int64_t K, double *z) {
 }
 
 /* ------------------------------------------------------------------------------------- */
-/* Step 3: per-token absmax activation quantisation  [2B4T 一.2], [v2]                     */
+/* Step 3: per-token activation quantisation: absmax (INT8) [2B4T 一.2], absmean (INT4) [v2]    */
 /* ------------------------------------------------------------------------------------- */
 
-/* For each row: m = max|z|, s = Q / max(m, 1e-5), c = clip(rint(z * s), -Q-1, Q), d = max(m, 1e-5) / Q,
+/* Per-token absmax (INT8, and the INT4 variant).
+ * For each row: m = max|z|, s = Q / max(m, 1e-5), c = clip(rint(z * s), -Q-1, Q), d = max(m, 1e-5) / Q,
  * with Q = 127 for 8-bit and Q = 7 for 4-bit codes.  The codes are decided in IEEE fp32 on
  * fp32 inputs (the kernel's precision).  If pre != NULL it receives z * s in double, the
  * unrounded value, so a test can see how close each code was to a rounding boundary.
@@ -346,9 +351,9 @@ void oracle_quant_act(const float *z, int64_t M, int64_t K, int bits, int8_t *co
 }
 
 /*
- * Variant INT4 quantiser with an absmean scale [v2: the INT4 activation strategy is named but its
- * formula is not printed; the weights' absmean function of b1.58 / 2B4T 一.2 gives the form].
- * Reading: per token row, beta = mean |z| (in double, rounded to fp32 once), g = max(beta,
+ * INT4 quantiser with an absmean scale [v2: INT8 and INT4 each take their own strategy, whose
+ * formulas are not printed; the pages' other quantisation function, the weights' absmean of
+ * b1.58 / 2B4T 一.2, gives the form].  Reading: per token row, beta = mean |z| (in double, rounded to fp32 once), g = max(beta,
  * 1e-5); the mean magnitude is mapped to code sqrt(7): s = fl32(sqrt7 / g) with sqrt7 the fp32
  * value of sqrt(7); codes = clip(rint(fl32(z * s)), -8, 7), round half to even; d = fl32(g /
  * sqrt7).  Unlike absmax, values beyond 7/s are clipped.  pre (optional) = z * s in double, the
@@ -488,11 +493,13 @@ void oracle_dequant_act(const int64_t *acc, const float *d, float gamma, int64_t
 /* ------------------------------------------------------------------------------------- */
 
 /* Y = BitLinear(X) (hadamard == 0) or H-BitLinear(X) (hadamard != 0), from bf16 X [M][K] and
- * latent bf16 W [N][K].  Optional outputs expose each stage: gamma, ternary q [N][K], the
- * transformed activations z [M][K] (double, before quantisation), codes [M][K], d [M],
- * acc [M][N].  Returns 0, or -1 when a buffer cannot be allocated. */
+ * latent bf16 W [N][K].  bits = 8 quantises the tokens with absmax to INT8, bits = 4 with
+ * absmean to INT4 (int4_absmax != 0: the absmax variant with Q = 7 instead).  Optional outputs
+ * expose each stage: gamma, ternary q [N][K], the transformed activations z [M][K] (double,
+ * before quantisation), codes [M][K], d [M], acc [M][N].  Returns 0, or -1 when a buffer
+ * cannot be allocated. */
 int oracle_bitlinear_forward_norm(const uint16_t *X, int64_t M, int64_t K, const uint16_t *W,
-                                  int64_t N, int hadamard, int bits, int norm,
+                                  int64_t N, int hadamard, int bits, int int4_absmax, int norm,
                                   const uint16_t *norm_gain, double norm_eps, uint16_t *Y,
                                   float *gamma_out, int8_t *q_out, double *z_out,
                                   int8_t *codes_out, float *d_out, int64_t *acc_out);
@@ -501,14 +508,14 @@ int oracle_bitlinear_forward(const uint16_t *X, int64_t M, int64_t K, const uint
                              int64_t N, int hadamard, int bits, uint16_t *Y,
                              float *gamma_out, int8_t *q_out, double *z_out,
                              int8_t *codes_out, float *d_out, int64_t *acc_out) {
-    return oracle_bitlinear_forward_norm(X, M, K, W, N, hadamard, bits, 0, NULL, 0.0, Y,
+    return oracle_bitlinear_forward_norm(X, M, K, W, N, hadamard, bits, 0, 0, NULL, 0.0, Y,
                                          gamma_out, q_out, z_out, codes_out, d_out, acc_out);
 }
 
 /* As oracle_bitlinear_forward; with norm != 0 each token row is RMS-normalised first
  * (oracle_rmsnorm with norm_gain and norm_eps) and the double result feeds the transform. */
 int oracle_bitlinear_forward_norm(const uint16_t *X, int64_t M, int64_t K, const uint16_t *W,
-                                  int64_t N, int hadamard, int bits, int norm,
+                                  int64_t N, int hadamard, int bits, int int4_absmax, int norm,
                                   const uint16_t *norm_gain, double norm_eps, uint16_t *Y,
                                   float *gamma_out, int8_t *q_out, double *z_out,
                                   int8_t *codes_out, float *d_out, int64_t *acc_out) {
@@ -534,7 +541,8 @@ int oracle_bitlinear_forward_norm(const uint16_t *X, int64_t M, int64_t K, const
     else memcpy(z, x, (size_t)(M * K) * sizeof(double));
     for (int64_t i = 0; i < M * K; ++i) zf[i] = (float)z[i];
 
-    oracle_quant_act(zf, M, K, bits, c, d, NULL, NULL);
+    if (bits == 4 && !int4_absmax) oracle_quant_act_absmean4(zf, M, K, c, d, NULL, NULL);
+    else oracle_quant_act(zf, M, K, bits, c, d, NULL, NULL);
     oracle_gemm_i64(c, q, M, N, K, acc);
     oracle_dequant(acc, d, gamma, M, N, Y);
 

@@ -331,8 +331,8 @@ def test_quant_pre_at_exact_ties(bits, Q):
     assert np.all(np.abs(pre - codes) <= 0.5 + 1e-6)
 
 
-# ---- variant INT4 quantiser with an absmean scale (a reading: the pages name the INT4 strategy
-# without its formula; the form is that of the weights' absmean) ----
+# ---- the INT4 quantiser, with an absmean scale (a reading: the pages give INT8 and INT4 each their
+# own strategy without printing either formula; the form is that of the weights' absmean) ----
 
 SQRT7_F32 = np.float32(math.sqrt(7.0))
 
@@ -469,9 +469,11 @@ def test_dequant_against_exact_products():
 
 @pytest.mark.parametrize("bits", [8, 4])
 def test_forward_hadamard_column_input(bits):
-    """x = a * (column j of H): z = a sqrt(K) e_j, so the codes are +-Q at j only and
-    Y[n] = q[n, j] * a * sqrt(K) * gamma (up to bf16 rounding).  A transposed operand, a
-    dropped normalisation or a wrong sign fails here."""
+    """x = a * (column j of H): z = a sqrt(K) e_j, one non-zero.  INT8 (absmax): the code is
+    +-127 at j only and Y[n] = q[n, j] * a * sqrt(K) * gamma.  INT4 (absmean): mean |z| =
+    a / sqrt(K), so z_j * s = +-sqrt(7) K is clipped to 7 or -8, and Y[n] = code * q[n, j] *
+    (a / sqrt(K) / sqrt(7)) * gamma (up to bf16 rounding).  A transposed operand, a dropped
+    normalisation or a wrong sign fails here."""
     K, N = 256, 64
     H = sylvester_bits(K)
     a = 0.125
@@ -479,15 +481,19 @@ def test_forward_hadamard_column_input(bits):
     X = bf16_bits(np.stack([a * H[:, j] * (1 if t % 2 == 0 else -1) for t, j in enumerate(js)]))
     W = synth.latent_weights(N, K, seed=1)
     out = oracle.bitlinear_forward(X, W, hadamard=True, bits=bits)
-    Q = 127 if bits == 8 else 7
     gamma = float(out["gamma"])
     for t, j in enumerate(js):
         sgn = 1 if t % 2 == 0 else -1
+        if bits == 8:
+            code, step = sgn * 127, a * math.sqrt(K) / 127
+        else:
+            code, step = (7 if sgn > 0 else -8), a / math.sqrt(K) / math.sqrt(7)
         expect_codes = np.zeros(K, np.int8)
-        expect_codes[j] = sgn * Q
+        expect_codes[j] = code
         np.testing.assert_array_equal(out["codes"][t], expect_codes)
+        np.testing.assert_allclose(out["d"][t], step, rtol=1e-6)
         y = oracle.bf16_to_f64(out["y"][t])
-        ref = sgn * out["q"][:, j] * a * math.sqrt(K) * gamma
+        ref = code * out["q"][:, j] * step * gamma
         np.testing.assert_allclose(y, ref, rtol=2 ** -8, atol=0)
 
 

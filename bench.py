@@ -176,17 +176,17 @@ class ClockSampler:
 # the oracle as a CPU baseline (test infrastructure, timed as it stands)
 # ----------------------------------------------------------------------------------------
 
-def oracle_sample(wl, rows: int, seed: int = 0):
+def oracle_sample(wl, rows: int, seed: int = 0, int4_absmax: bool = False):
     """Time the oracle's forward on `rows` tokens (full weight preparation included once)."""
     import oracle
     X = wl.activations(seed=seed, rows=rows)
     W = wl.weights(seed=seed)
     t0 = time.perf_counter()
-    oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits)
+    oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits, int4_absmax=int4_absmax)
     return time.perf_counter() - t0
 
 
-def oracle_baseline(wl, target_s: float = 12.0):
+def oracle_baseline(wl, target_s: float = 12.0, int4_absmax: bool = False):
     """tokens/s of the oracle, measured on a bounded sample and scaled to one full step:
     t_step = t_prep + (M / r) * t_rows(r), tokens/s = M / t_step."""
     import oracle
@@ -196,10 +196,10 @@ def oracle_baseline(wl, target_s: float = 12.0):
     oracle.pack_ternary(oracle.ternarize(W, g))
     t_prep = time.perf_counter() - t0
     probe_rows = 16
-    t_probe = oracle_sample(wl, probe_rows) - t_prep
+    t_probe = oracle_sample(wl, probe_rows, int4_absmax=int4_absmax) - t_prep
     per_row = max(t_probe, 1e-6) / probe_rows
     rows = int(max(probe_rows, min(wl.M, (target_s - t_prep) / per_row)))
-    t_rows = oracle_sample(wl, rows) - t_prep
+    t_rows = oracle_sample(wl, rows, int4_absmax=int4_absmax) - t_prep
     t_step = t_prep + (wl.M / rows) * max(t_rows, 1e-9)
     return {"value": wl.M / t_step, "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
@@ -214,13 +214,14 @@ def run_reference(args, wl, rank, world):
     if rank != 0:
         return
     import oracle
+    int4_absmax = bool(getattr(args, "absmax4", False))
     budget_s = 150.0
     W = wl.weights()
     t0 = time.perf_counter()
     g = oracle.absmean_gamma(W)
     oracle.pack_ternary(oracle.ternarize(W, g))
     t_prep = time.perf_counter() - t0
-    t_probe = oracle_sample(wl, 8) - t_prep
+    t_probe = oracle_sample(wl, 8, int4_absmax=int4_absmax) - t_prep
     per_row = max(t_probe, 1e-6) / 8
     steps_total = args.steps + args.warmup
     rows = int(max(1, min(wl.M, (budget_s / steps_total - t_prep) / per_row)))
@@ -228,7 +229,7 @@ def run_reference(args, wl, rank, world):
     for i in range(steps_total):
         X = wl.activations(seed=i, rows=rows)
         t0 = time.perf_counter()
-        oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits)
+        oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits, int4_absmax=int4_absmax)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     t_rows = statistics.mean(times) - t_prep
@@ -330,8 +331,8 @@ def run_gpu(args, wl, rank, world, device):
         gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
 
     def quant(b):
-        if args.absmean4:  # the variant INT4 quantiser (absmean scale)
-            B.bitnet_act_quant_absmean4(b["X"], wl.hadamard, b["codes"], b["scales"], b["rowsum"])
+        if args.absmax4:  # the variant INT4 quantiser (absmax scale)
+            B.bitnet_act_quant_absmax4(b["X"], wl.hadamard, b["codes"], b["scales"], b["rowsum"])
             return
         if gain is not None:
             B.bitnet_act_quant_norm(b["X"], gain, 1e-5, wl.hadamard, wl.act_bits, b["codes"],
@@ -480,7 +481,7 @@ def run_gpu(args, wl, rank, world, device):
                 "achieved_gbs": w_bytes / (phase_ms[0] * 1e-3) / 1e9,
                 "frac": w_bytes / (phase_ms[0] * 1e-3) / 1e9 / hbm},
             ("fwht_quant" if wl.hadamard else "act_quant_plain")
-            + ("+rmsnorm" if args.rmsnorm else "") + ("+absmean4" if args.absmean4 else "")
+            + ("+rmsnorm" if args.rmsnorm else "") + ("+absmax4" if args.absmax4 else "")
             + " (alone, outside the timed steps)": {
                 "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,
                 "achieved_gbs": q_bytes / (phase_ms[1] * 1e-3) / 1e9,
@@ -536,7 +537,8 @@ def run_gpu(args, wl, rank, world, device):
                        "rmsnorm": bool(args.rmsnorm),
                        "activation": args.activation,
                        "weights": "base3" if args.base3 else "2bit",
-                       "act_scale": "absmean" if args.absmean4 else "absmax",
+                       "act_scale": ("absmean" if wl.act_bits == 4 and not args.absmax4
+                                     else "absmax"),
                        "weight_rotation": bool(args.rotate_weights),
                        "tokens_per_rank": M,
                        "parallelism": f"replicas{world}",
@@ -549,7 +551,7 @@ def run_gpu(args, wl, rank, world, device):
             "clocks": clocks,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = oracle_baseline(wl, args.cpu_seconds)
+            line["cpu_baseline"] = oracle_baseline(wl, args.cpu_seconds, args.absmax4)
         elif not args.no_cpu_baseline:
             line["cpu_baseline"] = None
         print(json.dumps(line), flush=True)
@@ -585,9 +587,9 @@ def run_e2e(args, wl, B, stream, device, X0, W0):
         gain = synth.to_torch_bf16(synth.f32_to_bf16_bits(g)).to(device)
 
     def fwd(b):
-        if args.absmean4:
-            B.bitnet_bitlinear_forward_absmean4(b["Xd"], b["Wp"], b["gamma"], wl.hadamard,
-                                                Y=b["Yd"], ws=b["ws"])
+        if args.absmax4:
+            B.bitnet_bitlinear_forward_absmax4(b["Xd"], b["Wp"], b["gamma"], wl.hadamard,
+                                               Y=b["Yd"], ws=b["ws"])
         elif args.base3:
             B.bitnet_bitlinear_forward_base3(b["Xd"], b["Wp"], b["gamma"], wl.hadamard, act,
                                              Y=b["Yd"], ws=b["ws"])
@@ -667,8 +669,8 @@ def main():
     ap.add_argument("--base3", action="store_true",
                     help="store the weights five to a byte (base 3) for the decode product "
                          "(at most 8 tokens, INT8 activations)")
-    ap.add_argument("--absmean4", action="store_true",
-                    help="variant INT4 activation quantiser with a per-token absmean scale "
+    ap.add_argument("--absmax4", action="store_true",
+                    help="variant INT4 activation quantiser with a per-token absmax scale "
                          "(INT4 workloads)")
     ap.add_argument("--rotate-weights", action="store_true",
                     help="weight + activation Hadamard rotation: ternarise the rotated weight "
@@ -685,9 +687,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     wl = synth.WORKLOADS[args.workload]
-    if args.absmean4 and (wl.act_bits != 4 or args.rmsnorm or args.base3 or
-                          args.activation != "none"):
-        ap.error("--absmean4 serves INT4 workloads, without --rmsnorm, --base3 or --activation")
+    if args.absmax4 and (wl.act_bits != 4 or args.rmsnorm or args.base3 or
+                         args.activation != "none"):
+        ap.error("--absmax4 serves INT4 workloads, without --rmsnorm, --base3 or --activation")
     if args.rotate_weights and (not wl.hadamard or args.base3):
         ap.error("--rotate-weights serves H-BitLinear workloads with the 2-bit weights")
     if args.base3 and (wl.M > 8 or wl.act_bits != 8 or args.rmsnorm):

@@ -99,10 +99,10 @@ _SIGS = {
                                                             ctypes.c_int64, ctypes.c_void_p,
                                                             ctypes.c_void_p, ctypes.c_void_p,
                                                             ctypes.c_size_t, ctypes.c_void_p]),
-    "bitnet_act_quant_absmean4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+    "bitnet_act_quant_absmax4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p]),
-    "bitnet_bitlinear_forward_absmean4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
+    "bitnet_bitlinear_forward_absmax4": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64,
                                                          ctypes.c_int64, ctypes.c_void_p,
                                                          ctypes.c_void_p, ctypes.c_int64,
                                                          ctypes.c_int, ctypes.c_void_p,
@@ -249,7 +249,8 @@ def bitnet_quantize_pack_weights_noalloc(W: torch.Tensor, Wp: torch.Tensor | Non
 
 def bitnet_act_quant(X: torch.Tensor, hadamard: bool, act_bits: int, codes=None, scales=None,
                      rowsum=None, stream=None):
-    """Per-token (Hadamard +) absmax quantisation.  Returns (codes, scales, rowsum)."""
+    """Per-token (Hadamard +) quantisation: absmax INT8 or absmean INT4.  Returns (codes,
+    scales, rowsum)."""
     L = load_library()
     _check(X, "X", torch.bfloat16, 2)
     M, K = X.shape
@@ -483,10 +484,10 @@ def bitnet_quantize_pack_weights_rotated(W: torch.Tensor, Wp: torch.Tensor | Non
     return Wp, gamma
 
 
-def bitnet_act_quant_absmean4(X: torch.Tensor, hadamard: bool, codes=None, scales=None,
-                              rowsum=None, stream=None):
-    """Variant INT4 quantiser with a per-token absmean scale.  Returns (codes uint8 [M, K/2]
-    nibbles, scales, rowsum), consumed by the product with act_bits 4."""
+def bitnet_act_quant_absmax4(X: torch.Tensor, hadamard: bool, codes=None, scales=None,
+                             rowsum=None, stream=None):
+    """Variant INT4 quantiser with a per-token absmax scale (Q = 7).  Returns (codes uint8
+    [M, K/2] nibbles, scales, rowsum), consumed by the product with act_bits 4."""
     L = load_library()
     _check(X, "X", torch.bfloat16, 2)
     M, K = X.shape
@@ -499,14 +500,14 @@ def bitnet_act_quant_absmean4(X: torch.Tensor, hadamard: bool, codes=None, scale
     _nbytes_at_least(codes, int(L.bitnet_act_codes_bytes(M, K, 4)), "codes")
     _nbytes_at_least(scales, 4 * M, "scales")
     _nbytes_at_least(rowsum, 4 * M, "rowsum")
-    _rc(L.bitnet_act_quant_absmean4(X.data_ptr(), M, K, int(bool(hadamard)), codes.data_ptr(),
-                                    scales.data_ptr(), rowsum.data_ptr(), _stream(stream)),
-        "bitnet_act_quant_absmean4")
+    _rc(L.bitnet_act_quant_absmax4(X.data_ptr(), M, K, int(bool(hadamard)), codes.data_ptr(),
+                                   scales.data_ptr(), rowsum.data_ptr(), _stream(stream)),
+        "bitnet_act_quant_absmax4")
     return codes, scales, rowsum
 
 
-def bitnet_bitlinear_forward_absmean4(X, Wp, gamma, hadamard: bool, Y=None, ws=None, stream=None):
-    """Y = (H-)BitLinear(X) with the absmean INT4 activation quantiser."""
+def bitnet_bitlinear_forward_absmax4(X, Wp, gamma, hadamard: bool, Y=None, ws=None, stream=None):
+    """Y = (H-)BitLinear(X) with the variant absmax INT4 activation quantiser."""
     L = load_library()
     _check(X, "X", torch.bfloat16, 2)
     _check(Wp, "Wp")
@@ -520,10 +521,10 @@ def bitnet_bitlinear_forward_absmean4(X, Wp, gamma, hadamard: bool, Y=None, ws=N
     need = int(L.bitnet_workspace_bytes(M, K, N, 4))
     if ws is None:
         ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
-    _rc(L.bitnet_bitlinear_forward_absmean4(X.data_ptr(), M, K, Wp.data_ptr(), gamma.data_ptr(),
-                                            N, int(bool(hadamard)), Y.data_ptr(), ws.data_ptr(),
-                                            ws.numel() * ws.element_size(), _stream(stream)),
-        "bitnet_bitlinear_forward_absmean4")
+    _rc(L.bitnet_bitlinear_forward_absmax4(X.data_ptr(), M, K, Wp.data_ptr(), gamma.data_ptr(),
+                                           N, int(bool(hadamard)), Y.data_ptr(), ws.data_ptr(),
+                                           ws.numel() * ws.element_size(), _stream(stream)),
+        "bitnet_bitlinear_forward_absmax4")
     return Y
 
 

@@ -1,12 +1,13 @@
 // actquant.cu -- steps 2 and 3 of the forward: the online Hadamard transform of every token
-// row (H-BitLinear) fused with per-token absmax quantisation to INT8 or INT4.
+// row (H-BitLinear) fused with per-token quantisation, absmax to INT8 or absmean to INT4.
 //
 // BitNet v2 write-up, paragraphs on H-BitLinear: before the activations of Wo and Wdown are
 // quantised, each token row is multiplied by a Hadamard matrix (entries +-1, mutually
 // orthogonal rows), which turns the sharp, outlier-heavy distribution into a near-Gaussian
 // one.  BitNet b1.58 2B4T article, section 一.2: activations are quantised per token with
-// absmax to 8 bits; the BitNet v2 write-up adds a native 4-bit variant.  Readings: H_K in
-// Sylvester order scaled by 1/sqrt(K); Q = 127 or 7; eps 1e-5; round half to even.
+// absmax to 8 bits; the BitNet v2 write-up adds native 4-bit activations, each width with its
+// own strategy: INT4 takes the absmean form (mean |z| -> code sqrt(7), clip [-8, 7]).  Readings:
+// H_K in Sylvester order scaled by 1/sqrt(K); eps 1e-5; round half to even.
 //
 // Kernel design (HBM-bound: 2 bytes in, 1 or 0.5 byte out per element):
 //   One "team" of TEAM = 2^t threads owns one token row of K = 2^k elements, V = 2^v values per
@@ -96,12 +97,12 @@ __device__ __forceinline__ void team_sync(int team) {
     }
 }
 
-// sqrt(7) rounded to fp32: the code the mean |z| of a token maps to in the absmean INT4 variant
+// sqrt(7) rounded to fp32: the code the mean |z| of a token maps to in the absmean INT4 quantiser
 constexpr float kSqrt7 = 2.6457513110645906f;
 
-// ABSMEAN: the variant INT4 quantiser (BITS == 4 only): the scale comes from the mean |z| of
-// the token (summed in double) instead of max |z|, s = sqrt7 / max(mean, 1e-5), and codes are
-// clipped to [-8, 7].
+// ABSMEAN: the INT4 quantiser (BITS == 4 only): the scale comes from the mean |z| of the token
+// (summed in double) instead of max |z|, s = sqrt7 / max(mean, 1e-5), and codes are clipped to
+// [-8, 7].  BITS == 4 without ABSMEAN is the variant absmax INT4 quantiser (Q = 7).
 template <class P, int BITS, bool ZOUT, bool NORM, bool ABSMEAN = false>
 __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
     fwht_quant_kernel(const uint8_t *__restrict__ X, int M, float rsqrt_k,
@@ -295,7 +296,7 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
         }
     } else {
         constexpr int W = TEAM < 32 ? TEAM : 32;
-        static_assert(!ABSMEAN || BITS == 4, "the absmean variant is an INT4 quantiser");
+        static_assert(!ABSMEAN || BITS == 4, "the absmean rule is an INT4 quantiser");
         float g;
         if constexpr (ABSMEAN) {
 #pragma unroll
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(256)
         }
         return;
     }
-    static_assert(!ABSMEAN || BITS == 4, "the absmean variant is an INT4 quantiser");
+    static_assert(!ABSMEAN || BITS == 4, "the absmean rule is an INT4 quantiser");
     float mx = 0.f;
     double sa = 0.0;  // ABSMEAN: sum |y| in double (see fwht_quant_kernel)
     for (int64_t c = lane; c < nchunk; c += 32) {
@@ -561,18 +562,18 @@ static cudaError_t launch_fwht_n(const void *X, int64_t M, int act_bits, const N
                                  void *codes, float *scales, int32_t *rowsum, float *zout,
                                  int *status, cudaStream_t stream) {
     using P = typename FwhtConfig<LOGK>::P;
-    if (act_bits == kActInt4Absmean) {
+    if (act_bits == kActInt4Absmax) {
         if constexpr (NORM) return cudaErrorInvalidValue;  // not offered with the norm
         else
-            return launch_fwht_t<P, 4, false, false, true>(X, M, nrm, codes, scales, rowsum,
-                                                            nullptr, status, stream);
+            return launch_fwht_t<P, 4, false, false, false>(X, M, nrm, codes, scales, rowsum,
+                                                             nullptr, status, stream);
     }
     if (zout)
         return launch_fwht_t<P, 8, true, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
                                                stream);
     if (act_bits == 4)
-        return launch_fwht_t<P, 4, false, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
-                                                stream);
+        return launch_fwht_t<P, 4, false, NORM, true>(X, M, nrm, codes, scales, rowsum, zout,
+                                                      status, stream);
     return launch_fwht_t<P, 8, false, NORM>(X, M, nrm, codes, scales, rowsum, zout, status,
                                             stream);
 }
@@ -607,12 +608,12 @@ cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
 #undef BITNET_FWHT_CASE
 }
 
-template <int BITS, bool NORM, bool ZOUT>
+template <int BITS, bool NORM, bool ZOUT, bool ABSMEAN = false>
 static cudaError_t launch_plain_t(const void *X, int64_t M, int64_t K, const NormArgs &nrm,
                                   void *codes, float *scales, int32_t *rowsum, float *zout,
                                   cudaStream_t stream) {
     const int64_t blocks = (M + 7) / 8;
-    act_quant_plain_kernel<BITS, NORM, ZOUT><<<(unsigned)blocks, 256, 0, stream>>>(
+    act_quant_plain_kernel<BITS, NORM, ZOUT, ABSMEAN><<<(unsigned)blocks, 256, 0, stream>>>(
         reinterpret_cast<const uint4 *>(X), M, K, reinterpret_cast<const uint4 *>(nrm.gain),
         nrm.eps, reinterpret_cast<uint8_t *>(codes), scales, rowsum, zout);
     return cudaGetLastError();
@@ -621,22 +622,20 @@ static cudaError_t launch_plain_t(const void *X, int64_t M, int64_t K, const Nor
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,
                                    const NormArgs &nrm, void *codes, float *scales,
                                    int32_t *rowsum, float *zout, cudaStream_t stream) {
-    if (act_bits == kActInt4Absmean) {
+    if (act_bits == kActInt4Absmax) {
         if (nrm.on || zout) return cudaErrorInvalidValue;
-        const int64_t blocks = (M + 7) / 8;
-        act_quant_plain_kernel<4, false, false, true><<<(unsigned)blocks, 256, 0, stream>>>(
-            reinterpret_cast<const uint4 *>(X), M, K, nullptr, 0.f,
-            reinterpret_cast<uint8_t *>(codes), scales, rowsum, nullptr);
-        return cudaGetLastError();
+        return launch_plain_t<4, false, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
     }
     if (zout)  // the normalised rows themselves (the parity entry); only with a norm
         return launch_plain_t<8, true, true>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
     if (nrm.on)
         return act_bits == 4
-                   ? launch_plain_t<4, true, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream)
+                   ? launch_plain_t<4, true, false, true>(X, M, K, nrm, codes, scales, rowsum,
+                                                          zout, stream)
                    : launch_plain_t<8, true, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
     return act_bits == 4
-               ? launch_plain_t<4, false, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream)
+               ? launch_plain_t<4, false, false, true>(X, M, K, nrm, codes, scales, rowsum, zout,
+                                                       stream)
                : launch_plain_t<8, false, false>(X, M, K, nrm, codes, scales, rowsum, zout, stream);
 }
 

@@ -152,7 +152,7 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
 int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const float *gamma,
                  int64_t N, int act_bits, void *Y, void *ws, size_t ws_bytes, int hadamard,
                  cudaStream_t stream, const NormArgs &nrm = NormArgs(), int activation = 0,
-                 bool absmean4 = false) {
+                 bool absmax4 = false) {
     int rc = check_shape(M, K, N, true, true);
     if (rc) return rc;
     if (act_bits != 8 && act_bits != 4)
@@ -171,7 +171,7 @@ int forward_impl(const void *X, int64_t M, int64_t K, const void *Wp, const floa
     float *scales = reinterpret_cast<float *>(w + round256(bitnet_act_codes_bytes(M, K, act_bits)));
     int32_t *rowsum = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(scales) +
                                                   round256((size_t)M * sizeof(float)));
-    if ((rc = act_quant_impl(st, X, M, K, hadamard, absmean4 ? kActInt4Absmean : act_bits, codes,
+    if ((rc = act_quant_impl(st, X, M, K, hadamard, absmax4 ? kActInt4Absmax : act_bits, codes,
                              scales, rowsum, nullptr, stream, nrm)))
         return rc;
     // the quantiser above was launched in stream order after whatever wrote Wp
@@ -500,7 +500,7 @@ int bitnet_quantize_pack_weights_rotated(const void *W_dev, int64_t N, int64_t K
                     2, "ternarize_pack_f32");
 }
 
-int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadamard,
+int bitnet_act_quant_absmax4(const void *X_dev, int64_t M, int64_t K, int hadamard,
                               void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
                               bitnet_stream_t stream) {
     int rc = check_shape(M, K, 8, true, false);
@@ -511,11 +511,11 @@ int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadam
         return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
     DeviceState *st = nullptr;
     if ((rc = device_state(&st))) return rc;
-    return act_quant_impl(st, X_dev, M, K, hadamard ? 1 : 0, kActInt4Absmean, codes_dev,
+    return act_quant_impl(st, X_dev, M, K, hadamard ? 1 : 0, kActInt4Absmax, codes_dev,
                           scales_dev, rowsum_dev, nullptr, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int bitnet_bitlinear_forward_absmean4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+int bitnet_bitlinear_forward_absmax4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
                                       const float *gamma_dev, int64_t N, int hadamard, void *Y_dev,
                                       void *ws_dev, size_t ws_bytes, bitnet_stream_t stream) {
     return forward_impl(X_dev, M, K, Wp_dev, gamma_dev, N, 4, Y_dev, ws_dev, ws_bytes,

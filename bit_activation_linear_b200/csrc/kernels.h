@@ -38,9 +38,10 @@ struct NormArgs {
 cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
                               const NormArgs &nrm, void *codes, float *scales, int32_t *rowsum,
                               float *zout, int *status, cudaStream_t stream);
-// act_bits value that selects the variant INT4 quantiser with an absmean scale (INT4 codes,
-// layout as act_bits 4); the launchers reject it together with a norm or a z output.
-constexpr int kActInt4Absmean = 0x104;
+// act_bits 8: absmax INT8; act_bits 4: absmean INT4 (the mean |z| of a token maps to code
+// sqrt(7), clipped to [-8, 7]).  kActInt4Absmax selects the variant absmax INT4 quantiser (Q = 7;
+// INT4 codes, layout as act_bits 4); the launchers reject it together with a norm or a z output.
+constexpr int kActInt4Absmax = 0x204;
 
 // Quantise without a transform; K % 128 == 0.  zout != nullptr (with nrm.on) writes the
 // normalised rows in fp32 instead of codes.

@@ -9,8 +9,8 @@
  *                                              article, section 一.2 (BitLinear, W1.58A8)];
  *   2. in H-BitLinear every token row gets an online Hadamard transform  [BitNet v2 write-up,
  *      paragraphs on H-BitLinear; BitNet v2 abstract];
- *   3. every token row is quantised with absmax to INT8 (or INT4)  [2B4T article, 一.2;
- *      BitNet v2 write-up, 8-bit / 4-bit activation paragraph];
+ *   3. every token row is quantised, with absmax to INT8 or with absmean to INT4  [2B4T
+ *      article, 一.2; BitNet v2 write-up, 8-bit / 4-bit activation paragraph];
  *   4. a ternary x integer product accumulates in int32 and is rescaled to bf16
  *      [2B4T article, 一.2: multiplying by 1 adds, by -1 subtracts, by 0 skips].
  *
@@ -115,8 +115,15 @@ size_t bitnet_act_codes_bytes(int64_t M, int64_t K, int act_bits);
  * Per token row m (BitNet v2 write-up, H-BitLinear; 2B4T article, 一.2):
  *   z = (1/sqrt(K)) H_K x  when hadamard != 0 (H_K in Sylvester order, H_2n = [[H,H],[H,-H]],
  *       computed in fp32 by a fast Walsh-Hadamard transform), else z = x;
- *   mx = max(max_k |z_k|, 1e-5); s = Q / mx (IEEE fp32); codes = round_half_even(z * s),
- *   Q = 127 (act_bits 8) or 7 (act_bits 4);  scales[m] = mx / Q;  rowsum[m] = sum_k codes.
+ *   act_bits 8 (absmax; 2B4T article, 一.2): mx = max(max_k |z_k|, 1e-5); s = 127 / mx (IEEE
+ *       fp32); codes = round_half_even(z * s); scales[m] = mx / 127;
+ *   act_bits 4 (absmean; the BitNet v2 write-up gives INT8 and INT4 each their own strategy,
+ *       formulas not printed, and the pages' other quantisation function is absmean):
+ *       g = fp32(max(mean_k |z_k|, 1e-5)) (sum in double); s = sqrt7 / g with sqrt7 the fp32
+ *       value of sqrt(7) (the mean magnitude maps to code sqrt 7, so a Gaussian row spans the
+ *       4-bit range to about 2.3 standard deviations); codes = clip(round_half_even(z * s),
+ *       -8, 7); scales[m] = g / sqrt7;
+ *   rowsum[m] = sum_k codes.
  * X_dev       bf16 [M, K].
  * codes_dev   out: int8 [M, K] (act_bits 8) or [M, K/2] bytes (act_bits 4: every 8 codes
  *             k0..k0+7 fill 4 bytes, byte j = code k0+j in the low nibble and k0+4+j in the
@@ -272,32 +279,29 @@ int bitnet_quantize_pack_weights_rotated(const void *W_dev, int64_t N, int64_t K
                                          bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
-/* Variant INT4 quantiser with an absmean scale                                              */
+/* Variant INT4 quantiser with an absmax scale                                               */
 /* ---------------------------------------------------------------------------------------- */
 
 /*
- * The BitNet v2 write-up names a 4-bit activation strategy but its formula is not printed; the
- * default INT4 path (act_bits 4) uses absmax like INT8.  This variant takes the form of the
- * weights' absmean function ("The Era of 1-bit LLMs" summary, 方法论; 2B4T article, 一.2) for the
- * activations instead.  Per token row, with z = (1/sqrt(K)) H_K x (hadamard != 0) or z = x:
- *   beta = mean_k |z_k| (summed in double), g = fp32(max(beta, 1e-5)),
- *   s = sqrt7 / g (sqrt7 = fp32 value of sqrt(7), IEEE fp32 division): the mean magnitude maps to
- *   code sqrt(7), so a Gaussian row spans the 4-bit range to about 2.3 standard deviations;
- *   codes = clip(round_half_even(z * s), -8, 7)  (values beyond the range are clipped);
- *   scales[m] = g / sqrt7;  rowsum[m] = sum_k codes.
+ * The INT4 path (act_bits 4) uses the absmean rule above.  This variant quantises to INT4 with
+ * absmax instead, the INT8 rule with Q = 7 (the BitNet v2 write-up names absmax for the 4-bit
+ * activations of the post-training baselines it compares against).  Per token row, with
+ * z = (1/sqrt(K)) H_K x (hadamard != 0) or z = x:
+ *   mx = max(max_k |z_k|, 1e-5); s = 7 / mx (IEEE fp32); codes = round_half_even(z * s) in
+ *   [-7, 7]; scales[m] = mx / 7; rowsum[m] = sum_k codes.
  * Outputs in the INT4 layout of bitnet_act_quant (act_bits 4), so bitnet_ternary_gemm with
  * act_bits 4 consumes them.  Shapes, alignment and errors as bitnet_act_quant.
  */
-int bitnet_act_quant_absmean4(const void *X_dev, int64_t M, int64_t K, int hadamard,
-                              void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
-                              bitnet_stream_t stream);
+int bitnet_act_quant_absmax4(const void *X_dev, int64_t M, int64_t K, int hadamard,
+                             void *codes_dev, float *scales_dev, int32_t *rowsum_dev,
+                             bitnet_stream_t stream);
 
-/* The whole layer with this quantiser: bitnet_act_quant_absmean4, then the product with act_bits
+/* The whole layer with this quantiser: bitnet_act_quant_absmax4, then the product with act_bits
  * 4.  ws_bytes >= bitnet_workspace_bytes(M, K, N, 4); other arguments as
  * bitnet_bitlinear_forward. */
-int bitnet_bitlinear_forward_absmean4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
-                                      const float *gamma_dev, int64_t N, int hadamard, void *Y_dev,
-                                      void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
+int bitnet_bitlinear_forward_absmax4(const void *X_dev, int64_t M, int64_t K, const void *Wp_dev,
+                                     const float *gamma_dev, int64_t N, int hadamard, void *Y_dev,
+                                     void *ws_dev, size_t ws_bytes, bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* Base-3 weights for decode                                                                */

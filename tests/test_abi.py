@@ -148,14 +148,14 @@ def test_base3_entries_size_and_rejections_before_the_device(lib):
     assert lib.bitnet_quantize_pack_weights_base3(p, 256, 256, p, p, p, 0, None) == -5
 
 
-def test_absmean4_entries_reject_bad_arguments_before_the_device(lib):
+def test_absmax4_entries_reject_bad_arguments_before_the_device(lib):
     p = ctypes.c_void_p(16)
-    assert lib.bitnet_act_quant_absmean4(p, 4, 200, 1, p, p, p, None) == -1      # K % 128
-    assert lib.bitnet_act_quant_absmean4(p, 0, 256, 1, p, p, p, None) == -1      # M < 1
-    assert lib.bitnet_act_quant_absmean4(None, 4, 256, 1, p, p, p, None) == -1   # null X
+    assert lib.bitnet_act_quant_absmax4(p, 4, 200, 1, p, p, p, None) == -1      # K % 128
+    assert lib.bitnet_act_quant_absmax4(p, 0, 256, 1, p, p, p, None) == -1      # M < 1
+    assert lib.bitnet_act_quant_absmax4(None, 4, 256, 1, p, p, p, None) == -1   # null X
     q = ctypes.c_void_p(24)
-    assert lib.bitnet_act_quant_absmean4(q, 4, 256, 1, p, p, p, None) == -1      # misaligned
-    assert lib.bitnet_bitlinear_forward_absmean4(p, 4, 256, p, p, 256, 1, p, p, 0, None) == -5
+    assert lib.bitnet_act_quant_absmax4(q, 4, 256, 1, p, p, p, None) == -1      # misaligned
+    assert lib.bitnet_bitlinear_forward_absmax4(p, 4, 256, p, p, 256, 1, p, p, 0, None) == -5
 
 
 def test_rotated_weight_entries_size_and_rejections_before_the_device(lib):

@@ -99,7 +99,7 @@ def test_hadamard_quant_codes(B, K, bits):
     Xd = dev_bf16(X)
     z = B.bitnet_fwht_f32(Xd).cpu().numpy()
     codes, scales, rowsum = B.bitnet_act_quant(Xd, True, bits)
-    c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act_for_bits(z, bits)
     c = codes.cpu().numpy()
     c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
     n_diff = check_codes(c, c_ref, pre)
@@ -113,14 +113,19 @@ def test_hadamard_quant_codes(B, K, bits):
 def test_plain_quant_codes_exact(B, K, bits):
     M = 21
     X = synth.gaussian_activations(M, K, seed=K + bits)
+    X[3] = 0  # a zero row: zero codes, guarded scale
     codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), False, bits)
     z = oracle.bf16_to_f64(X).astype(np.float32)
-    c_ref, d_ref, _, rs_ref = oracle.quant_act(z, bits)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act_for_bits(z, bits)
     c = codes.cpu().numpy()
     c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
-    np.testing.assert_array_equal(c, c_ref)
-    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    assert check_codes(c, c_ref, pre) == 0
+    if bits == 8:
+        np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    else:  # the absmean sum is taken in double in another order: the scale may move by an ulp
+        np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
     np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
+    assert not c[3].any()
 
 
 def test_quant_zero_rows(B):
@@ -255,7 +260,7 @@ def forward_case(B, wl, sample_count, seed=0):
     ref = oracle.bitlinear_forward(X[rows], W, wl.hadamard, wl.act_bits)
     assert np.float32(gamma.item()) == ref["gamma"]
     c = codes_rows(codes, rows, wl.K, wl.act_bits)
-    _, _, pre, _ = oracle.quant_act(ref["z"].astype(np.float32), wl.act_bits)
+    _, _, pre, _ = oracle.quant_act_for_bits(ref["z"].astype(np.float32), wl.act_bits)
     check_codes(c, ref["codes"], pre)
     flips = (c != ref["codes"]).sum(axis=1)
     y = oracle.bf16_to_f64(to_np_bits(Y)[rows])
@@ -361,7 +366,8 @@ def test_weights_near_the_threshold_of_a_random_gamma(B):
 def test_activation_codes_at_exact_ties_plain(B, bits):
     """Plain rows with max |x| = Q/2 or Q/4, so s = 2 or 4 exactly, and every other x equal to
     (k + 1/2) / s: x * s lands exactly on a .5 for each of them.  The codes must round half to
-    even, as the oracle does, with zero differences."""
+    even, as the oracle does, with zero differences.  (INT4: the absmax variant, whose scale a
+    row's maximum fixes.)"""
     Q = 127 if bits == 8 else 7
     K = 256
     rng = np.random.default_rng(bits)
@@ -371,7 +377,10 @@ def test_activation_codes_at_exact_ties_plain(B, bits):
         x[rng.integers(K)] = Q / s
         rows.append(x)
     X = bf16_exact(np.stack(rows))
-    codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), False, bits)
+    if bits == 8:
+        codes, scales, rowsum = B.bitnet_act_quant(dev_bf16(X), False, 8)
+    else:
+        codes, scales, rowsum = B.bitnet_act_quant_absmax4(dev_bf16(X), False)
     B.bitnet_sync_status()
     z = oracle.bf16_to_f64(X).astype(np.float32)
     c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
@@ -529,11 +538,14 @@ def test_norm_quant_codes_exact_on_the_gpu_rows(B, K, hadamard, bits):
     Xd, gd = dev_bf16(X), dev_gain(g)
     z = B.bitnet_norm_transform_f32(Xd, gd, NORM_EPS, hadamard).cpu().numpy()
     codes, scales, rowsum = B.bitnet_act_quant_norm(Xd, gd, NORM_EPS, hadamard, bits)
-    c_ref, d_ref, pre, rs_ref = oracle.quant_act(z, bits)
+    c_ref, d_ref, pre, rs_ref = oracle.quant_act_for_bits(z, bits)
     c = codes.cpu().numpy()
     c = c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
     assert check_codes(c, c_ref, pre) == 0
-    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    if bits == 8:
+        np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+    else:  # absmean: a double sum in another order
+        np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
     np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
 
 
@@ -728,16 +740,16 @@ def test_base3_product_equals_two_bit_product(B):
 
 
 # ----------------------------------------------------------------------------------------
-# variant INT4 quantiser with a per-token absmean scale
+# INT4: the absmean rule of act_bits 4 (the clip is exercised), and the absmax variant
 # ----------------------------------------------------------------------------------------
 
 @pytest.mark.parametrize("K", [128, 256, 2048, 4096, 8192, 16384, 32768])
-def test_absmean4_hadamard_codes(B, K):
+def test_int4_absmean_hadamard_codes(B, K):
     M = 37 if K <= 8192 else 9
     X = synth.sharp_activations(M, K, seed=5 * K + 1)
     Xd = dev_bf16(X)
     z = B.bitnet_fwht_f32(Xd).cpu().numpy()
-    codes, scales, rowsum = B.bitnet_act_quant_absmean4(Xd, True)
+    codes, scales, rowsum = B.bitnet_act_quant(Xd, True, 4)
     B.bitnet_sync_status()
     c_ref, d_ref, pre, _ = oracle.quant_act_absmean4(z)
     c = oracle.unpack_int4(codes.cpu().numpy().view(np.uint8), K)
@@ -748,39 +760,49 @@ def test_absmean4_hadamard_codes(B, K):
     assert (c == 7).any() or (c == -8).any()  # the clip is exercised
 
 
-@pytest.mark.parametrize("K", [128, 640, 4096])
-def test_absmean4_plain_codes(B, K):
-    M = 19
-    X = synth.gaussian_activations(M, K, seed=K + 17)
-    X[3] = 0  # a zero row: zero codes, guarded scale
-    codes, scales, rowsum = B.bitnet_act_quant_absmean4(dev_bf16(X), False)
+@pytest.mark.parametrize("K", [128, 256, 2048, 8192, 16384])
+def test_absmax4_hadamard_codes(B, K):
+    M = 37 if K <= 8192 else 9
+    X = synth.sharp_activations(M, K, seed=5 * K + 2)
+    Xd = dev_bf16(X)
+    z = B.bitnet_fwht_f32(Xd).cpu().numpy()
+    codes, scales, rowsum = B.bitnet_act_quant_absmax4(Xd, True)
     B.bitnet_sync_status()
-    z = oracle.bf16_to_f64(X).astype(np.float32)
-    c_ref, d_ref, pre, rs_ref = oracle.quant_act_absmean4(z)
+    c_ref, d_ref, pre, _ = oracle.quant_act(z, 4)
     c = oracle.unpack_int4(codes.cpu().numpy().view(np.uint8), K)
     assert check_codes(c, c_ref, pre) == 0
     np.testing.assert_allclose(scales.cpu().numpy(), d_ref, rtol=1e-6)
+    np.testing.assert_array_equal(rowsum.cpu().numpy(), c.astype(np.int64).sum(axis=1))
+
+
+@pytest.mark.parametrize("K", [128, 640, 4096])
+def test_absmax4_plain_codes(B, K):
+    M = 19
+    X = synth.gaussian_activations(M, K, seed=K + 17)
+    X[3] = 0  # a zero row: zero codes, guarded scale
+    codes, scales, rowsum = B.bitnet_act_quant_absmax4(dev_bf16(X), False)
+    B.bitnet_sync_status()
+    z = oracle.bf16_to_f64(X).astype(np.float32)
+    c_ref, d_ref, _, rs_ref = oracle.quant_act(z, 4)
+    c = oracle.unpack_int4(codes.cpu().numpy().view(np.uint8), K)
+    np.testing.assert_array_equal(c, c_ref)
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
     np.testing.assert_array_equal(rowsum.cpu().numpy(), rs_ref)
     assert not c[3].any()
 
 
 @pytest.mark.parametrize("name,rows", [("wdown_8192", 16), ("tiny", None)])
-def test_absmean4_forward_end_to_end(B, name, rows):
+def test_absmax4_forward_end_to_end(B, name, rows):
     wl = synth.WORKLOADS[name]
     X, W = wl.activations(seed=6), wl.weights(seed=6)
     Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
-    Y = B.bitnet_bitlinear_forward_absmean4(dev_bf16(X), Wp, gamma, wl.hadamard)
+    Y = B.bitnet_bitlinear_forward_absmax4(dev_bf16(X), Wp, gamma, wl.hadamard)
     B.bitnet_sync_status()
-    sel = np.arange(wl.M) if rows is None else np.sort(
-        np.random.default_rng(6).choice(wl.M, size=rows, replace=False))
-    x = oracle.bf16_to_f64(X[sel])
-    z = (oracle.fwht(x) if wl.hadamard else x).astype(np.float32)
-    codes, d, _, _ = oracle.quant_act_absmean4(z)
-    g = oracle.absmean_gamma(W)
-    assert np.float32(gamma.item()) == g
-    acc = oracle.gemm_i64(codes, oracle.ternarize(W, g))
-    y_ref = oracle.bf16_to_f64(oracle.dequant(acc, d, g))
+    sel = sample_rows(wl.M, rows, 6)
+    ref = oracle.bitlinear_forward(X[sel], W, wl.hadamard, 4, int4_absmax=True)
+    assert np.float32(gamma.item()) == ref["gamma"]
     y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
+    y_ref = oracle.bf16_to_f64(ref["y"])
     assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
 
 
@@ -823,7 +845,7 @@ def test_rotated_forward_end_to_end(B, name, rows):
     sel = np.arange(wl.M) if rows is None else np.sort(
         np.random.default_rng(8).choice(wl.M, size=rows, replace=False))
     z = oracle.fwht(oracle.bf16_to_f64(X[sel])).astype(np.float32)
-    codes, d, _, _ = oracle.quant_act(z, wl.act_bits)
+    codes, d, _, _ = oracle.quant_act_for_bits(z, wl.act_bits)
     Wr = oracle.rotate_weights(W)
     g = oracle.absmean_gamma_f32(Wr)
     assert abs(np.float32(gamma.item()) / g - 1) <= 1e-6

@@ -73,6 +73,9 @@ def lib():
                                                         vp]),
                 "oracle_quant_act": (None, [vp, i64, i64, i32, vp, vp, vp, vp]),
                 "oracle_quant_act_absmean4": (None, [vp, i64, i64, vp, vp, vp, vp]),
+                "oracle_quant_states": (None, [vp, i64, i64, i64, i32, vp, vp, vp]),
+                "oracle_pack_bits": (None, [vp, i64, i64, i32, vp]),
+                "oracle_unpack_bits": (None, [vp, i64, i64, i32, vp]),
                 "oracle_pack_int4": (None, [vp, i64, i64, vp]),
                 "oracle_unpack_int4": (None, [vp, i64, i64, vp]),
                 "oracle_gemm_i64": (None, [vp, vp, i64, i64, i64, vp]),
@@ -293,6 +296,41 @@ def unpack_int4(b: np.ndarray, K: int) -> np.ndarray:
     M = b.shape[0]
     c = np.empty((M, K), dtype=np.int8)
     lib().oracle_unpack_int4(_p(b), M, K, _p(c))
+    return c
+
+
+# --------------------------------------------------------------------------------------
+# Low-bit Q / K / V states  (BitNet v2 write-up, Tables 2 and 3: the QKV states' bit width
+# varies; a 3-bit KV cache matches full precision)
+# --------------------------------------------------------------------------------------
+
+def quant_states(x_bf16: np.ndarray, group: int, bits: int = 3):
+    """Per-token (group = C) or per-head (group = head_dim) absmax codes of bf16 states [M, C],
+    Q = 2^(bits-1) - 1, decided in fp32.  Returns (codes int8 [M, C], d float32 [M, C/group],
+    pre float64 [M, C])."""
+    x = bf16_to_f64(x_bf16).astype(np.float32)
+    M, C = x.shape
+    codes = np.empty((M, C), dtype=np.int8)
+    d = np.empty((M, C // group), dtype=np.float32)
+    pre = np.empty((M, C), dtype=np.float64)
+    lib().oracle_quant_states(_p(x), M, C, int(group), int(bits), _p(codes), _p(d), _p(pre))
+    return codes, d, pre
+
+
+def pack_bits(c: np.ndarray, bits: int) -> np.ndarray:
+    """Rows of `bits`-bit codes as little-endian bit streams: [M, C * bits / 8] uint8."""
+    c = np.ascontiguousarray(c, dtype=np.int8)
+    M, C = c.shape
+    out = np.empty((M, C * bits // 8), dtype=np.uint8)
+    lib().oracle_pack_bits(_p(c), M, C, int(bits), _p(out))
+    return out
+
+
+def unpack_bits(b: np.ndarray, C: int, bits: int) -> np.ndarray:
+    b = np.ascontiguousarray(b, dtype=np.uint8).reshape(-1, C * bits // 8)
+    M = b.shape[0]
+    c = np.empty((M, C), dtype=np.int8)
+    lib().oracle_unpack_bits(_p(b), M, C, int(bits), _p(c))
     return c
 
 

@@ -37,7 +37,9 @@
  *   absmean ([b1.58]).  So INT8 = per-token absmax, Q = 127, eps 1e-5, round-half-even, clip to
  *   [-128, 127], d = max|z| / 127; INT4 = per-token absmean, the mean |z| of a token mapped to
  *   code sqrt(7), eps 1e-5, clip to [-8, 7], d = mean|z| / sqrt(7).  Variant INT4 quantiser
- *   (not the default): absmax with Q = 7.
+ *   (not the default): absmax with Q = 7.  Low-bit Q / K / V states ([v2] Tables 2-3 vary
+ *   their width): the absmax rule per token or per head with Q = 2^(bits-1) - 1, stored as a
+ *   little-endian bit stream of two's complement fields.
  *   Variant weight + activation rotation (not the default): the rows of W are transformed by
  *   the same orthonormal Hadamard before the absmean ternarisation, W' = W H / sqrt(K), so that
  *   W' (H x / sqrt(K)) = W x; the rotated rows are rounded to fp32 once, then ternarised.
@@ -486,6 +488,78 @@ void oracle_dequant_act(const int64_t *acc, const float *d, float gamma, int64_t
             }
         }
     }
+}
+
+/* ------------------------------------------------------------------------------------- */
+/* Low-bit Q / K / V states  [v2, Tables 2 and 3]                                           */
+/* ------------------------------------------------------------------------------------- */
+
+/* The write-up's Tables 2 and 3 vary the bit width of the attention's Q, K and V states (a 3-bit
+ * KV cache matches full precision); the quantiser's formula is not printed.  Reading: the
+ * activations' absmax rule per token, or per group of `group` consecutive features of a token
+ * (one attention head, group = head_dim), with Q = 2^(bits-1) - 1 (3 for 3 bits):
+ *   m = max |x| over the group, s = Q / max(m, 1e-5) (fp32 IEEE), c = clip(rint(fl32(x * s)),
+ *   -Q-1, Q) with round-half-even, d = max(m, 1e-5) / Q (fp32).
+ * x holds the bf16 states widened to fp32 (exact).  codes: int8 [M][C]; d: [M][C / group];
+ * pre (optional): x * Q / max(m, 1e-5) in double, the unrounded value.  C % group == 0. */
+void oracle_quant_states(const float *x, int64_t M, int64_t C, int64_t group, int bits,
+                         int8_t *codes, float *d, double *pre) {
+    const float Q = (float)((1 << (bits - 1)) - 1);
+    const float lo = -Q - 1.0f;
+    const int64_t G = C / group;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t g = 0; g < G; ++g) {
+            const float *row = x + m * C + g * group;
+            float mx = 0.0f;
+            for (int64_t k = 0; k < group; ++k) {
+                float a = fabsf(row[k]);
+                if (a > mx) mx = a;
+            }
+            float gm = mx < 1e-5f ? 1e-5f : mx;
+            volatile float s = Q / gm;
+            volatile float dq = gm / Q;
+            for (int64_t k = 0; k < group; ++k) {
+                volatile float v = row[k] * s;
+                float t = nearbyintf(v);
+                if (t > Q) t = Q;
+                if (t < lo) t = lo;
+                codes[m * C + g * group + k] = (int8_t)t;
+                if (pre) pre[m * C + g * group + k] = (double)row[k] * (double)Q / (double)gm;
+            }
+            d[m * G + g] = dq;
+        }
+    }
+}
+
+/* Storage of `bits`-bit codes: each row is a little-endian bit stream, code k of the row in bits
+ * bits*k .. bits*k + bits - 1 (two's complement), so a row takes C * bits / 8 bytes (C % 8 == 0).
+ * unpack sign-extends back to int8. */
+void oracle_pack_bits(const int8_t *c, int64_t M, int64_t C, int bits, uint8_t *out) {
+    const int64_t rb = C * bits / 8;
+    memset(out, 0, (size_t)(M * rb));
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < C; ++k) {
+            const unsigned v = (unsigned)c[m * C + k] & ((1u << bits) - 1u);
+            for (int b = 0; b < bits; ++b) {
+                const int64_t bit = k * bits + b;
+                if (v >> b & 1u) out[m * rb + bit / 8] |= (uint8_t)(1u << (bit % 8));
+            }
+        }
+}
+
+void oracle_unpack_bits(const uint8_t *in, int64_t M, int64_t C, int bits, int8_t *c) {
+    const int64_t rb = C * bits / 8;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < C; ++k) {
+            int v = 0;
+            for (int b = 0; b < bits; ++b) {
+                const int64_t bit = k * bits + b;
+                v |= (in[m * rb + bit / 8] >> (bit % 8) & 1) << b;
+            }
+            if (v >> (bits - 1) & 1) v -= 1 << bits;
+            c[m * C + k] = (int8_t)v;
+        }
 }
 
 /* ------------------------------------------------------------------------------------- */

@@ -653,3 +653,76 @@ def test_base3_rows_round_trip_and_size(K):
     row = np.concatenate([q[2] + 1, np.ones((-K) % 20, np.int64)])
     expect = (row.reshape(-1, 5) * np.array([81, 27, 9, 3, 1])).sum(axis=1)
     np.testing.assert_array_equal(words[2].view(np.uint8), expect.astype(np.uint8))
+
+
+# ----------------------------------------------------------------------------------------
+# Low-bit Q / K / V states (BitNet v2 write-up, Tables 2 and 3: the QKV states' bit width
+# varies; 3 bits match full precision).  The formula is a reading: the activations' absmax
+# rule per token or per head, Q = 2^(bits-1) - 1.
+# ----------------------------------------------------------------------------------------
+
+def test_state_bitstream_hand_examples():
+    g = golden("lowbit_state_bitstream.json")
+    for case in g["cases"]:
+        c = np.array([case["codes"]], np.int8)
+        packed = oracle.pack_bits(c, case["bits"])
+        np.testing.assert_array_equal(packed[0], np.array(case["bytes"], np.uint8))
+        np.testing.assert_array_equal(oracle.unpack_bits(packed, c.shape[1], case["bits"]), c)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 8])
+def test_state_bitstream_round_trip(bits):
+    rng = np.random.default_rng(bits)
+    c = rng.integers(-(1 << (bits - 1)), 1 << (bits - 1), size=(5, 96)).astype(np.int8)
+    packed = oracle.pack_bits(c, bits)
+    assert packed.shape == (5, 96 * bits // 8)
+    np.testing.assert_array_equal(oracle.unpack_bits(packed, 96, bits), c)
+
+
+@pytest.mark.parametrize("bits,group", [(3, 64), (3, 512), (4, 128), (8, 512)])
+def test_state_quant_brute_force_and_max_rule(bits, group):
+    Q = (1 << (bits - 1)) - 1
+    rng = np.random.default_rng(bits + group)
+    x = bf16_bits(rng.standard_normal((6, 512)) * 0.7)
+    x[2, :group] = 0  # one all-zero group: zero codes, guarded scale
+    codes, d, pre = oracle.quant_states(x, group, bits)
+    xf = oracle.bf16_to_f64(x).astype(np.float32)
+    G = 512 // group
+    xg = xf.reshape(6, G, group)
+    mx = np.abs(xg).max(axis=2)
+    gm = np.maximum(mx, np.float32(1e-5)).astype(np.float32)
+    s = (np.float32(Q) / gm).astype(np.float32)
+    v = (xg * s[..., None]).astype(np.float32)        # the fp32 product the decision uses
+    ref = _nearest_code_brute(v.reshape(-1), -Q - 1, Q).reshape(6, 512)
+    np.testing.assert_array_equal(codes, ref)
+    np.testing.assert_array_equal(d, (gm / np.float32(Q)).astype(np.float32))
+    # the largest |x| of each live group maps to +-Q
+    cg = codes.reshape(6, G, group)
+    for m in range(6):
+        for g in range(G):
+            if mx[m, g] > 0:
+                k = int(np.argmax(np.abs(xg[m, g])))
+                assert cg[m, g, k] == Q * np.sign(xg[m, g, k])
+    assert not codes[2, :group].any() and d[2, 0] == np.float32(np.float32(1e-5) / np.float32(Q))
+    # every code is within half a step of its value
+    err = np.abs(codes.reshape(6, G, group) * d[..., None].astype(np.float64) - xg)
+    assert np.all(err <= 0.5 * d[..., None] * (1 + 1e-6))
+
+
+def test_state_quant_exact_ties_and_head_independence():
+    # a group with max 1.5: s = 3 / 1.5 = 2 exactly; 0.25, 0.75, 1.25 land on 0.5, 1.5, 2.5
+    row = np.zeros(64)
+    row[:6] = [1.5, 0.25, 0.75, 1.25, -0.75, -1.25]
+    x = bf16_bits(row[None, :])
+    codes, d, pre = oracle.quant_states(x, 64, 3)
+    np.testing.assert_array_equal(pre[0, :6], [3.0, 0.5, 1.5, 2.5, -1.5, -2.5])
+    np.testing.assert_array_equal(codes[0, :6], [3, 0, 2, 2, -2, -2])   # ties to even
+    assert d[0, 0] == np.float32(0.5)
+    # per-head codes are the per-token rule applied to each head alone
+    rng = np.random.default_rng(3)
+    x = bf16_bits(rng.laplace(size=(4, 256)))
+    c_head, d_head, _ = oracle.quant_states(x, 64, 3)
+    for h in range(4):
+        c1, d1, _ = oracle.quant_states(x[:, 64 * h:64 * (h + 1)], 64, 3)
+        np.testing.assert_array_equal(c_head[:, 64 * h:64 * (h + 1)], c1)
+        np.testing.assert_array_equal(d_head[:, h], d1[:, 0])

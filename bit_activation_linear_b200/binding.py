@@ -21,7 +21,7 @@ _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
 ACT_RELU2, ACT_SWIGLU = 1, 2  # bitnet_activation
-PATH_DECODE, PATH_TC, PATH_TC_KSPLIT = 1, 2, 3  # bitnet_product_path
+PATH_DECODE, PATH_TC, PATH_TC_SKINNY = 1, 2, 3  # bitnet_product_path
 
 
 class BitnetError(RuntimeError):
@@ -124,6 +124,10 @@ _SIGS = {
                                                       ctypes.c_int, ctypes.c_void_p,
                                                       ctypes.c_void_p, ctypes.c_size_t,
                                                       ctypes.c_void_p]),
+    "bitnet_state_codes_bytes": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]),
+    "bitnet_quant_states": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p]),
     "bitnet_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bitnet_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int64, ctypes.c_void_p]),
 }
@@ -604,6 +608,28 @@ def bitnet_bitlinear_forward_base3(X, Wp3, gamma, hadamard: bool, activation: in
                                          _stream(stream)),
         "bitnet_bitlinear_forward_base3")
     return Y
+
+
+def bitnet_state_codes_bytes(M: int, C: int, bits: int) -> int:
+    return int(load_library().bitnet_state_codes_bytes(M, C, bits))
+
+
+def bitnet_quant_states(X: torch.Tensor, group: int, bits: int = 3, codes=None, scales=None,
+                        stream=None):
+    """Low-bit absmax codes of bf16 Q/K/V states [M, C], per group of `group` features.
+    Returns (codes uint8 [M, C * bits / 8] bit streams, scales float [M, C / group])."""
+    L = load_library()
+    _check(X, "X", torch.bfloat16, 2)
+    M, C = X.shape
+    if codes is None:
+        codes = torch.empty((M, C * bits // 8), dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty((M, max(C // group, 1)), dtype=torch.float32, device=X.device)
+    _nbytes_at_least(codes, int(L.bitnet_state_codes_bytes(M, C, bits)), "codes")
+    _nbytes_at_least(scales, 4 * M * (C // group), "scales")
+    _rc(L.bitnet_quant_states(X.data_ptr(), M, C, int(group), int(bits), codes.data_ptr(),
+                              scales.data_ptr(), _stream(stream)), "bitnet_quant_states")
+    return codes, scales
 
 
 def bitnet_selftest_wait_timeout(limit_cycles: int, stream=None) -> None:

@@ -144,6 +144,8 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
     a.early_weights = early_weights;
     a.activation = activation;
     if (M <= kGemvMaxTokens) return launched(launch_ternary_gemv(a, stream), 1, "ternary_gemv");
+    if (M <= kSkinnyMaxTokens)
+        return launched(launch_ternary_gemm_skinny(a, g_encode, stream), 1, "ternary_gemm_skinny");
     int n = 0;
     const cudaError_t e = launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream, &n);
     return launched(e, n, "ternary_gemm_tc");
@@ -439,9 +441,13 @@ int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path
         *k_split = 1;
         return BITNET_OK;
     }
-    const int split = ternary_gemm_tc_split(M, N, K, act_bits, st->num_sms);
-    *path = split > 1 ? BITNET_PATH_TC_KSPLIT : BITNET_PATH_TC;
-    *k_split = split;
+    if (M <= kSkinnyMaxTokens) {
+        *path = BITNET_PATH_TC_SKINNY;
+        *k_split = ternary_gemm_skinny_split(N, K);
+        return BITNET_OK;
+    }
+    *path = BITNET_PATH_TC;
+    *k_split = 1;
     return BITNET_OK;
 }
 
@@ -639,6 +645,33 @@ int bitnet_bitlinear_forward_base3(const void *X_dev, int64_t M, int64_t K, cons
     // the quantiser was launched in stream order after whatever wrote Wp3
     return gemv_base3_impl(st, w, scales, rowsum, M, K, Wp3_dev, gamma_dev, N, activation,
                            nullptr, Y_dev, true, s);
+}
+
+size_t bitnet_state_codes_bytes(int64_t M, int64_t C, int bits) {
+    if (M <= 0 || C <= 0 || bits < 2 || bits > 8) return 0;
+    return (size_t)M * (size_t)C * (size_t)bits / 8;
+}
+
+int bitnet_quant_states(const void *X_dev, int64_t M, int64_t C, int64_t group, int bits,
+                        void *codes_dev, float *scales_dev, bitnet_stream_t stream) {
+    if (M < 1 || M > (int64_t)INT32_MAX)
+        return fail(BITNET_ERR_INVALID, "M = %lld must be in 1 .. 2^31-1", (long long)M);
+    if (group < 32 || group % 32 != 0 || group > (1 << 20))
+        return fail(BITNET_ERR_INVALID, "group = %lld must be a positive multiple of 32",
+                    (long long)group);
+    if (C < group || C % group != 0 || C > (1 << 24))
+        return fail(BITNET_ERR_INVALID, "C = %lld must be a multiple of group = %lld",
+                    (long long)C, (long long)group);
+    if (bits < 2 || bits > 8) return fail(BITNET_ERR_INVALID, "bits = %d must be in 2 .. 8", bits);
+    if (!X_dev || !codes_dev || !scales_dev) return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!aligned16(X_dev) || !aligned16(codes_dev))
+        return fail(BITNET_ERR_INVALID, "device pointers must be 16-byte aligned");
+    DeviceState *st = nullptr;
+    int rc = device_state(&st);
+    if (rc) return rc;
+    return launched(launch_quant_states(X_dev, M, C, group, bits, codes_dev, scales_dev,
+                                        reinterpret_cast<cudaStream_t>(stream)),
+                    1, "quant_states");
 }
 
 int bitnet_selftest_wait_timeout(int64_t limit_cycles, bitnet_stream_t stream) {

@@ -40,9 +40,8 @@
 //                them with bulk tensor stores.  (Direct stores of one row per thread touch 32
 //                lines per instruction; on B200 they held up the unpack warps' shared-memory
 //                stores for ~6000 cycles per tile.)
-// Work: a persistent grid of pairs walks units; a unit is one tile (one pass over K) or, with
-// few tiles, one K chunk of a tile whose int32 sums are added atomically into a scratch and
-// finished by splitk_finish_kernel (see the K split section below).
+// Work: a persistent grid of pairs walks the output tiles, each in one pass over K.  (Products of
+// a few tokens, where the tiles would be mostly empty, take gemm_skinny.cu instead.)
 // Commits multicast to both CTAs; every wait is bounded: after ~1 s a role records
 // BITNET_ERR_TIMEOUT and stops; in-flight copies and MMAs are drained and both CTAs meet at a
 // cluster barrier before tensor memory is released.  No TMA multicast is used.
@@ -81,9 +80,7 @@ constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_WTMA = 2, WARP_EPI = 16;
 // What the epilogue writes: the int32 accumulators (parity entry), the rescaled bf16 output, or
 // the rescaled output through an activation (squared ReLU; SwiGLU over interleaved gate/up
 // features, half as many columns).
-// OUT_PARTIAL: the raw int32 sums of a unit's K chunk are added atomically into an int32 [M, N]
-// scratch; splitk_finish_kernel then writes the outputs (see launch_ternary_gemm_tc).
-enum OutMode { OUT_ACC = 0, OUT_BF16 = 1, OUT_RELU2 = 2, OUT_SWIGLU = 3, OUT_PARTIAL = 4 };
+enum OutMode { OUT_ACC = 0, OUT_BF16 = 1, OUT_RELU2 = 2, OUT_SWIGLU = 3 };
 constexpr int NUM_THREADS = 24 * 32;
 
 // Unpack / code warps: eight warps outside the MMA warp's scheduler partition (warp % 4 == 1).
@@ -144,7 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                            const __grid_constant__ CUtensorMap tmap_y,
                            void *__restrict__ Yout, const float *__restrict__ scales,
                            const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
-                           int M, int N, int K, int split, int *status) {
+                           int M, int N, int K, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -166,18 +163,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const int num_tiles = n_ftiles * n_ttiles;
     const int KS = (K + BK - 1) / BK;  // stages per tile (the last one may be half: K % 256 = 128)
     constexpr int B_GROUPS = BITS == 8 ? 2 : 1;
-    // Work units: tile x K chunk (split chunks per tile, split <= KS; split = 1 unless
-    // MODE == OUT_PARTIAL).  Pair p takes units p, p + npairs, ...; unit u is tile u / split,
-    // stages [c*KS/split, (c+1)*KS/split) of it with c = u % split.
-    if constexpr (MODE != OUT_PARTIAL) split = 1;  // a constant: the one-pass loops as written
-    const int num_units = num_tiles * split;
+    // Pair p takes tiles p, p + npairs, ...; a unit is one tile and all KS stages of its K axis.
+    const int num_units = num_tiles;
     const int my_units = pair < num_units ? (num_units - 1 - pair) / npairs + 1 : 0;
     auto unit = [&](int t, int &tile, int &kb, int &ke) {
-        const int u = pair + t * npairs;
-        tile = u / split;
-        const int c = u - tile * split;
-        kb = c * KS / split;
-        ke = (c + 1) * KS / split;
+        tile = pair + t * npairs;
+        kb = 0;
+        ke = KS;
     };
     int total = 0;  // (unit, stage) iterations of this pair
     for (int t = 0; t < my_units; ++t) {
@@ -208,7 +200,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (warp == WARP_TMA && lane == 0) {
         prefetch_tensormap(&tmap_codes);
         prefetch_tensormap(&tmap_w);
-        if (MODE != OUT_ACC && MODE != OUT_PARTIAL) prefetch_tensormap(&tmap_y);
+        if (MODE != OUT_ACC) prefetch_tensormap(&tmap_y);
     }
     if (warp == WARP_MMA) {
         tmem_alloc_pair(&bar->tmem_base, TMEM_COLS);
@@ -401,14 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tmem_ld_32x32b_x32(t_lane + ab * BN + col, v);
                 tmem_wait_ld();
                 const int n0 = nf * BN + col;
-                if constexpr (MODE == OUT_PARTIAL) {
-                    // this unit's K chunk of the raw sums (the code-sum offset is removed once,
-                    // by splitk_finish_kernel); integer additions in any order are exact
-                    int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (m_ok && n0 + j < N) atomicAdd(row + n0 + j, (int)v[j]);
-                } else if constexpr (MODE == OUT_ACC) {
+                if constexpr (MODE == OUT_ACC) {
                     int32_t *row = reinterpret_cast<int32_t *>(Yout) + m * N;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -557,7 +542,7 @@ static int max_pairs(int num_sms) {
 template <int BITS, int MODE>
 static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
                                const CUtensorMap &my, void *out, int64_t tiles, int num_sms,
-                               cudaStream_t stream, int split = 1) {
+                               cudaStream_t stream) {
     auto kern = ternary_gemm_tc_kernel<BITS, MODE>;
     static bool configured[64] = {};
     int dev = 0;
@@ -569,8 +554,7 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
         configured[dev] = true;
     }
     const int pairs_max = max_pairs<BITS, MODE>(num_sms);
-    const int64_t units = tiles * split;
-    const int pairs = (int)(units < pairs_max ? units : pairs_max);
+    const int pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -582,122 +566,14 @@ static cudaError_t launch_tc_t(const GemmArgs &a, const CUtensorMap &mc, const C
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, mc, mw, my, out, a.scales, a.rowsum, a.gamma, (int)a.M,
-                              (int)a.N, (int)a.K, split, a.status);
-}
-
-// ------------------------------------------------------------------------------------------
-// K split for small tile counts.  With few tiles (decode-sized token counts) most pairs would
-// idle while a few walk the whole K axis; instead each tile's K axis is cut into `split` chunks,
-// every (tile, chunk) unit goes to its own pair, and the units' int32 sums are added atomically
-// into a library-owned scratch (exact: integer addition in any order).  splitk_finish_kernel then
-// applies the epilogue arithmetic of the one-pass kernel (same fp32 operations, so the same bf16
-// results) and returns the scratch to zero for the next call.  One scratch per device: calls
-// that take this path must not overlap on the GPU (they are serialised on one stream).
-
-constexpr int64_t kSplitAccElems = int64_t(1) << 21;  // 8 MB of int32: M * N <= 2^21
-__device__ __align__(16) int32_t g_splitk_acc[kSplitAccElems];  // read as int4 vectors
-
-// thread = 8 consecutive features of one token (N % 8 == 0)
-template <int ACT>
-__global__ void __launch_bounds__(256)
-    splitk_finish_kernel(int32_t *__restrict__ acc, const float *__restrict__ scales,
-                         const int32_t *__restrict__ rowsum, const float *__restrict__ gamma_ptr,
-                         int M, int N, int32_t *__restrict__ acc_out,
-                         __nv_bfloat16 *__restrict__ Y) {
-    const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;  // group of 8 features
-    const int64_t groups = (int64_t)M * (N / 8);
-    if (i >= groups) return;
-    const int64_t m = i / (N / 8);
-    const int n0 = (int)(i - m * (N / 8)) * 8;
-    int4 *src = reinterpret_cast<int4 *>(acc + m * N + n0);
-    const int4 a0 = src[0], a1 = src[1];
-    src[0] = make_int4(0, 0, 0, 0);  // the scratch is zero again for the next call
-    src[1] = make_int4(0, 0, 0, 0);
-    const int rs = rowsum[m];
-    const int v[8] = {a0.x - rs, a0.y - rs, a0.z - rs, a0.w - rs,
-                      a1.x - rs, a1.y - rs, a1.z - rs, a1.w - rs};
-    if (acc_out) {
-        int4 *dst = reinterpret_cast<int4 *>(acc_out + m * N + n0);
-        dst[0] = make_int4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_int4(v[4], v[5], v[6], v[7]);
-    }
-    if (!Y) return;
-    const float sc = scales[m] * *gamma_ptr;
-    if constexpr (ACT == OUT_SWIGLU) {
-        uint32_t pk[2];
-#pragma unroll
-        for (int i2 = 0; i2 < 2; ++i2) {
-            float o[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float g = (float)v[4 * i2 + 2 * e] * sc;
-                const float u = (float)v[4 * i2 + 2 * e + 1] * sc;
-                o[e] = __fdiv_rn(g, 1.f + expf(-g)) * u;
-            }
-            const __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
-            pk[i2] = *reinterpret_cast<const uint32_t *>(&h);
-        }
-        *reinterpret_cast<uint2 *>(Y + m * (N / 2) + n0 / 2) = make_uint2(pk[0], pk[1]);
-    } else {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i2 = 0; i2 < 4; ++i2) {
-            float y0 = (float)v[2 * i2] * sc, y1 = (float)v[2 * i2 + 1] * sc;
-            if constexpr (ACT == OUT_RELU2) {
-                y0 = y0 > 0.f ? y0 * y0 : 0.f;
-                y1 = y1 > 0.f ? y1 * y1 : 0.f;
-            }
-            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-            pk[i2] = *reinterpret_cast<const uint32_t *>(&h);
-        }
-        *reinterpret_cast<uint4 *>(Y + m * N + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-}
-
-// Chunks per tile for the K split, or 1 for the one-pass kernel: only when fewer than half of the
-// pairs would get a tile, the K axis has at least two stages and the output fits the scratch.
-static int choose_split(int64_t tiles, int64_t M, int64_t N, int64_t K, int pairs_max) {
-    const int64_t KS = (K + BK - 1) / BK;
-    if (tiles * 2 > pairs_max || KS < 2 || M * N > kSplitAccElems) return 1;
-    int64_t split = pairs_max / tiles;
-    if (split > KS) split = KS;
-    return split < 2 ? 1 : (int)split;
-}
-
-template <int BITS>
-static cudaError_t launch_split(const GemmArgs &a, const CUtensorMap &mc, const CUtensorMap &mw,
-                                int64_t tiles, int split, int num_sms, cudaStream_t stream) {
-    int32_t *acc = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&acc), g_splitk_acc);
-    if (e != cudaSuccess) return e;
-    CUtensorMap unused;
-    memset(&unused, 0, sizeof unused);
-    e = launch_tc_t<BITS, OUT_PARTIAL>(a, mc, mw, unused, acc, tiles, num_sms, stream, split);
-    if (e != cudaSuccess) return e;
-    const int64_t groups = a.M * (a.N / 8);
-    const unsigned blocks = (unsigned)((groups + 255) / 256);
-    auto *Y = reinterpret_cast<__nv_bfloat16 *>(a.Y);
-    switch (a.Y ? a.activation : 0) {
-        case 1:
-            splitk_finish_kernel<OUT_RELU2><<<blocks, 256, 0, stream>>>(
-                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
-            break;
-        case 2:
-            splitk_finish_kernel<OUT_SWIGLU><<<blocks, 256, 0, stream>>>(
-                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
-            break;
-        default:
-            splitk_finish_kernel<OUT_BF16><<<blocks, 256, 0, stream>>>(
-                acc, a.scales, a.rowsum, a.gamma, (int)a.M, (int)a.N, a.acc, Y);
-    }
-    return cudaGetLastError();
+                              (int)a.N, (int)a.K, a.status);
 }
 
 }  // namespace tc
 
-static CUresult encode_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType dt,
-                          const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                          uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+CUresult encode_tmap_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType dt,
+                        const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
     auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(encode_fn);
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_bytes};
@@ -706,14 +582,6 @@ static CUresult encode_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType
     return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-}
-
-int ternary_gemm_tc_split(int64_t M, int64_t N, int64_t K, int act_bits, int num_sms) {
-    using namespace tc;
-    const int64_t tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM);
-    return choose_split(tiles, M, N, K,
-                        act_bits == 8 ? max_pairs<8, OUT_PARTIAL>(num_sms)
-                                      : max_pairs<4, OUT_PARTIAL>(num_sms));
 }
 
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
@@ -728,30 +596,22 @@ cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_s
     // INT4 [M rows][K/2 bytes], one [128 tokens x 128 B] box of packed nibbles per CTA and stage;
     // both with the 128-byte swizzle
     const uint64_t cb = a.act_bits == 8 ? (uint64_t)a.K : (uint64_t)a.K / 2;
-    if (encode_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, cb, (uint64_t)a.M, cb,
+    if (encode_tmap_2d(encode_fn, &mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, cb, (uint64_t)a.M, cb,
                   SUBK, HM, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     // packed weights: [N rows][K/4 bytes], one [128 features x 64 B] box per stage, 64-byte
     // swizzle
-    if (encode_2d(encode_fn, &mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, (uint64_t)a.K / 4,
+    if (encode_tmap_2d(encode_fn, &mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, (uint64_t)a.K / 4,
                   (uint64_t)a.N, (uint64_t)a.K / 4, BK / 4, HN,
                   CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
-    const int split = choose_split(tiles, a.M, a.N, a.K,
-                                   a.act_bits == 8 ? max_pairs<8, OUT_PARTIAL>(num_sms)
-                                                   : max_pairs<4, OUT_PARTIAL>(num_sms));
-    if (split > 1) {
-        if (launches) *launches = 2;
-        return a.act_bits == 8 ? launch_split<8>(a, mc, mw, tiles, split, num_sms, stream)
-                               : launch_split<4>(a, mc, mw, tiles, split, num_sms, stream);
-    }
     if (launches) *launches = (a.Y ? 1 : 0) + (a.acc ? 1 : 0);
     if (a.Y) {
         // bf16 output [M rows][N] (N/2 with SwiGLU), one [32 tokens x 16 features] box per
         // store, 32-byte swizzle
         const uint64_t n_out = a.activation == 2 ? (uint64_t)a.N / 2 : (uint64_t)a.N;
-        if (encode_2d(encode_fn, &my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, n_out, (uint64_t)a.M,
+        if (encode_tmap_2d(encode_fn, &my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, n_out, (uint64_t)a.M,
                       n_out * 2, Y_BOX_N, 32, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
         switch (a.activation * 2 + (a.act_bits == 8 ? 1 : 0)) {

@@ -78,11 +78,28 @@ cudaError_t launch_ternary_gemv(const GemmArgs &a, cudaStream_t stream);
 // base-3 words.
 cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream);
 
-// tcgen05 tensor-core kernel (prefill).  encode is cuTensorMapEncodeTiled.
+// tcgen05 tensor-core kernel (prefill), one pass over K per 256 x 256 tile.  encode is
+// cuTensorMapEncodeTiled.
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream, int *launches = nullptr);
-// The K split launch_ternary_gemm_tc takes for this shape on the current device (1: one pass).
-int ternary_gemm_tc_split(int64_t M, int64_t N, int64_t K, int act_bits, int num_sms);
+
+// tcgen05 tensor-core kernel for kGemvMaxTokens < M <= kSkinnyMaxTokens: weights on the MMA's M
+// side, streamed once, K split over a cluster (gemm_skinny.cu).  One launch.
+constexpr int kSkinnyMaxTokens = 64;
+cudaError_t launch_ternary_gemm_skinny(const GemmArgs &a, void *encode_fn, cudaStream_t stream);
+// CTAs per cluster (K chunks per feature block) that launch takes on the current device.
+int ternary_gemm_skinny_split(int64_t N, int64_t K);
+
+// 2-D tiled tensor map over a row-major array (no interleave, 256-byte L2 promotion, zero fill).
+CUresult encode_tmap_2d(void *encode_fn, CUtensorMap *map, CUtensorMapDataType dt,
+                        const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                        uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+// ---- low-bit Q / K / V states (states.cu) ----
+// Per (token, group) absmax codes of `bits` bits (2..8) as little-endian row bit streams, one
+// fp32 scale per group.  group % 32 == 0, C % group == 0.
+cudaError_t launch_quant_states(const void *X, int64_t M, int64_t C, int64_t group, int bits,
+                                void *codes, float *scales, cudaStream_t stream);
 
 // ---- failure detection self-test (selftest.cu) ----
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, int *status,

@@ -169,13 +169,11 @@ int bitnet_norm_transform_f32(const void *X_dev, int64_t M, int64_t K, const voi
  * Y[m, n]   = bf16_rn(float(acc[m, n]) * (scales[m] * gamma))   (fp32 product)
  * codes/scales/rowsum as written by bitnet_act_quant; Wp/gamma as written by
  * bitnet_quantize_pack_weights.  acc_dev (int32 [M, N]) and Y_dev (bf16 [M, N]) are each
- * optional (NULL to skip); at least one must be given.  Large M runs on the tcgen05 tensor
- * cores, small M (decode) on a weight-streaming kernel; both give the same integers.
- * When M > 8 but the output has few 256 x 256 tiles (fewer than half the GPU's SM pairs) and
- * M * N <= 2^21, the tensor-core product splits K across SM pairs and sums the int32 partials in
- * a library-owned scratch (8 MB per device, zero between calls); two such calls on one device
- * must not run at the same time on the GPU (issue them on one stream, or order them).  The same
- * holds for the forward and activation entries below, which use this product.
+ * optional (NULL to skip); at least one must be given.  Three kernels serve the product, by token count: a weight-streaming kernel (M <= 8), a
+ * tensor-core kernel with the weights on the MMA's M side and K split across a cluster of SMs
+ * (9 <= M <= 64), and a tensor-core kernel over 256 x 256 output tiles (M > 64).  None keeps
+ * state between calls or uses memory other than its arguments: calls on different streams may
+ * run concurrently.
  */
 int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
                         const int32_t *rowsum_dev, int64_t M, int64_t K, const void *Wp_dev,
@@ -185,16 +183,17 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
 /*
  * Which kernel the product of an M x K by N x K shape takes on the current device (a query of
  * the library; the pages have no counterpart).  Every path gives the same integers.
- *   *path    BITNET_PATH_DECODE    weight-streaming kernel (M <= 8 tokens);
+ *   *path    BITNET_PATH_DECODE    weight-streaming kernel on the CUDA cores (M <= 8 tokens);
  *            BITNET_PATH_TC        tensor-core kernel, one pass over K per 256 x 256 tile;
- *            BITNET_PATH_TC_KSPLIT tensor-core kernel with K cut into *k_split chunks.
- *   *k_split chunks of K per output tile (1 unless BITNET_PATH_TC_KSPLIT).
+ *            BITNET_PATH_TC_SKINNY tensor-core kernel for 9 <= M <= 64: 128 output features per
+ *                                  CTA, K cut into *k_split chunks over a cluster of CTAs.
+ *   *k_split chunks of K per output feature block (1 unless BITNET_PATH_TC_SKINNY).
  * Shape and act_bits rules and errors as bitnet_ternary_gemm; enqueues nothing.
  */
 typedef enum {
     BITNET_PATH_DECODE = 1,
     BITNET_PATH_TC = 2,
-    BITNET_PATH_TC_KSPLIT = 3
+    BITNET_PATH_TC_SKINNY = 3
 } bitnet_product_path;
 
 int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path, int *k_split);
@@ -353,6 +352,29 @@ int bitnet_bitlinear_forward_base3(const void *X_dev, int64_t M, int64_t K, cons
                                    const float *gamma_dev, int64_t N, int hadamard,
                                    int activation, void *Y_dev, void *ws_dev, size_t ws_bytes,
                                    bitnet_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* Low-bit Q / K / V states                                                                 */
+/* ---------------------------------------------------------------------------------------- */
+
+/*
+ * The BitNet v2 write-up's Tables 2 and 3 vary the bit width of the attention's Q, K and V states
+ * (a 3-bit KV cache matches full precision); the quantiser's formula is not printed.  This is the
+ * activations' absmax rule applied per token (group = C) or per head (group = head_dim):
+ *   per row m and group j of `group` consecutive features:
+ *   mx = max(max |x| over the group, 1e-5);  s = Q / mx (IEEE fp32), Q = 2^(bits-1) - 1;
+ *   codes = clip(round_half_even(fl32(x * s)), -Q-1, Q);  scales[m * (C / group) + j] = mx / Q.
+ * X_dev       bf16 [M, C] states (e.g. the Q, K or V projection's output), 16-byte aligned.
+ * codes_dev   out: bitnet_state_codes_bytes(M, C, bits) bytes; row m is a little-endian bit
+ *             stream of C two's complement fields, code k in bits bits*k .. bits*k + bits - 1
+ *             (bits = 3: eight codes in three bytes).  16-byte aligned.
+ * scales_dev  out: float [M, C / group].
+ * group % 32 == 0, C % group == 0, 2 <= bits <= 8, else BITNET_ERR_INVALID.
+ */
+size_t bitnet_state_codes_bytes(int64_t M, int64_t C, int bits);
+
+int bitnet_quant_states(const void *X_dev, int64_t M, int64_t C, int64_t group, int bits,
+                        void *codes_dev, float *scales_dev, bitnet_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* Status                                                                                   */

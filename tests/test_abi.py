@@ -168,3 +168,16 @@ def test_rotated_weight_entries_size_and_rejections_before_the_device(lib):
     assert lib.bitnet_quantize_pack_weights_rotated(p, 256, 256, p, p, p, 1024, None) == -5
     q = ctypes.c_void_p(24)
     assert lib.bitnet_quantize_pack_weights_rotated(p, 256, 256, q, p, p, 1 << 30, None) == -1
+
+
+def test_state_quant_size_and_rejections_before_the_device(lib):
+    assert lib.bitnet_state_codes_bytes(16, 4096, 3) == 16 * 4096 * 3 // 8
+    assert lib.bitnet_state_codes_bytes(16, 4096, 9) == 0
+    p = ctypes.c_void_p(16)
+    assert lib.bitnet_quant_states(p, 4, 4096, 100, 3, p, p, None) == -1    # group % 32
+    assert lib.bitnet_quant_states(p, 4, 4000, 128, 3, p, p, None) == -1    # C % group
+    assert lib.bitnet_quant_states(p, 4, 4096, 128, 1, p, p, None) == -1    # bits
+    assert lib.bitnet_quant_states(p, 0, 4096, 128, 3, p, p, None) == -1    # M
+    assert lib.bitnet_quant_states(None, 4, 4096, 128, 3, p, p, None) == -1  # null X
+    q = ctypes.c_void_p(20)
+    assert lib.bitnet_quant_states(q, 4, 4096, 128, 3, p, p, None) == -1    # misaligned

@@ -161,8 +161,8 @@ def staged_product(B, M, K, N, bits, seed):
     (1, 8320, 136), (2, 4096, 8), (6, 8320, 264),           # decode, rows split over 2 / 4 warps
     (8, 16384, 520), (4, 32768, 16),                        # (17 steps: uneven split)
     (7, 4096, 8200),                                        # decode, 4-row groups
-    (9, 256, 256), (130, 384, 136), (300, 2048, 264),       # tensor-core kernel, ragged tiles
-    (64, 8192, 2048), (17, 4096, 1032),                     # tensor cores with the K split
+    (9, 256, 256), (64, 8192, 2048), (17, 4096, 1032),      # skinny tensor-core kernel
+    (130, 384, 136), (300, 2048, 264),                      # 256 x 256 tiles, ragged
     (256, 1024, 1024), (513, 128, 8),
     (1000, 640, 520),                                       # several tiles, 2.5 K stages
 ])
@@ -190,6 +190,60 @@ def sample_rows(M, count, seed):
 def codes_rows(codes, rows, K, bits):
     c = codes[torch.from_numpy(rows).to(codes.device)].cpu().numpy()
     return c.view(np.int8) if bits == 8 else oracle.unpack_int4(c.view(np.uint8), K)
+
+
+# The skinny tensor-core product (9 <= M <= 64: 128 features per CTA, weights unpacked into
+# tensor memory, K split over a cluster and summed through distributed shared memory): every
+# token tile (16 / 32 / 64), ragged token counts, ragged N, K with a partial last 512-stage, both
+# code widths and every cluster size the launcher picks.  int32 bit-exact on all rows.
+@pytest.mark.parametrize("M,K,N", [
+    (9, 128, 8), (16, 640, 136), (17, 2048, 8192), (32, 8192, 2048), (33, 1152, 264),
+    (48, 16384, 4096), (63, 4096, 1032), (64, 2048, 8192), (64, 8192, 2048), (40, 384, 16384),
+])
+@pytest.mark.parametrize("bits", [8, 4])
+def test_skinny_product_int32_exact_and_bf16(B, M, K, N, bits):
+    path, split = B.bitnet_product_plan(M, K, N, bits)
+    assert path == B.PATH_TC_SKINNY and 1 <= split <= min(8, (K + 511) // 512)
+    c, q, d, gamma, acc, Y = staged_product(B, M, K, N, bits, seed=M * 11 + N)
+    acc_ref = oracle.gemm_i64(c, q)
+    np.testing.assert_array_equal(acc.astype(np.int64), acc_ref)
+    y_ref = oracle.bf16_to_f64(oracle.dequant(acc_ref, d, gamma))
+    y = oracle.bf16_to_f64(to_np_bits(Y))
+    rel = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), 1e-30)
+    assert np.all((rel <= Y_REL) | (y_ref == 0)), rel.max()
+    assert np.all(y[y_ref == 0] == 0)
+
+
+def test_product_paths_by_token_count(B):
+    for M, path in ((1, B.PATH_DECODE), (8, B.PATH_DECODE), (9, B.PATH_TC_SKINNY),
+                    (64, B.PATH_TC_SKINNY), (65, B.PATH_TC), (4096, B.PATH_TC)):
+        assert B.bitnet_product_plan(M, 2048, 2048, 8)[0] == path, M
+
+
+def test_concurrent_forwards_on_two_streams(B):
+    """Two decode-size forwards (skinny tensor-core product, K split over clusters) issued on two
+    streams with no ordering between them: no state is shared, so both match the oracle."""
+    wls = [synth.WORKLOADS["decode_m64_k8192"], synth.WORKLOADS["decode_m32_k2048"]]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    inputs = []
+    for i, wl in enumerate(wls):
+        X, W = wl.activations(seed=20 + i), wl.weights(seed=20 + i)
+        Wp, gamma = B.bitnet_quantize_pack_weights(dev_bf16(W))
+        inputs.append((X, W, dev_bf16(X), Wp, gamma))
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(3):  # several rounds so the launches overlap
+        for (X, W, Xd, Wp, gamma), wl, st in zip(inputs, wls, streams):
+            with torch.cuda.stream(st):
+                outs.append(B.bitnet_hbitlinear_forward(Xd, Wp, gamma, wl.act_bits, stream=st))
+    torch.cuda.synchronize()
+    B.bitnet_sync_status()
+    for r in range(3):
+        for i, ((X, W, _, _, _), wl) in enumerate(zip(inputs, wls)):
+            ref = oracle.bitlinear_forward(X, W, wl.hadamard, wl.act_bits)
+            y = oracle.bf16_to_f64(to_np_bits(outs[2 * r + i]))
+            y_ref = oracle.bf16_to_f64(ref["y"])
+            assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
 
 
 # The one-pass tensor-core product at the sizes the benchmark runs: many K stages per tile
@@ -597,7 +651,8 @@ def check_act(Y, y_ref_bits):
     (1, 256, 256), (5, 2048, 272), (8, 384, 528),               # decode kernel
     (8, 8320, 272), (2, 4096, 528),                             # decode, split rows
     (8, 2048, 8192),                                            # decode, 4-row groups
-    (9, 256, 256), (300, 2048, 272), (1000, 640, 528),          # tensor-core kernel
+    (9, 256, 256), (32, 8192, 2064), (64, 2048, 8192),          # skinny tensor-core kernel
+    (300, 2048, 272), (1000, 640, 528),                         # 256 x 256 tiles
 ])
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("act", [1, 2])
@@ -853,3 +908,40 @@ def test_rotated_forward_end_to_end(B, name, rows):
     y_ref = oracle.bf16_to_f64(oracle.dequant(acc, d, g))
     y = oracle.bf16_to_f64(to_np_bits(Y)[sel])
     assert np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref) <= Y_REL
+
+
+# ----------------------------------------------------------------------------------------
+# low-bit Q / K / V states (BitNet v2 write-up, Tables 2 and 3): packed bit streams and scales
+# bit-exact against the oracle
+# ----------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,C,group", [(37, 4096, 128), (16, 2048, 64), (9, 4096, 4096),
+                                       (5, 96, 32), (300, 1024, 1024)])
+@pytest.mark.parametrize("bits", [3, 2, 4, 8])
+def test_state_quant_bit_exact(B, M, C, group, bits):
+    rng = np.random.default_rng(M + C + bits)
+    x = rng.standard_normal((M, C)).astype(np.float32)
+    x[:, rng.choice(C, size=max(1, C // 64), replace=False)] *= 20.0  # outlier channels
+    x[1, :group] = 0.0                                                 # an all-zero group
+    X = synth.f32_to_bf16_bits(x)
+    codes, scales = B.bitnet_quant_states(dev_bf16(X), group, bits)
+    B.bitnet_sync_status()
+    c_ref, d_ref, _ = oracle.quant_states(X, group, bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), oracle.pack_bits(c_ref, bits))
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)
+
+
+def test_state_quant_exact_ties(B):
+    # groups with max 1.5: s = 2 exactly, so 0.25, 0.75, 1.25 -> 0.5, 1.5, 2.5 -> 0, 2, 2
+    K = 64
+    vals = np.array([0.25, 0.75, 1.25, -0.25, -0.75, -1.25, 0.5, 1.0])
+    row = np.tile(vals, K // len(vals))
+    row[0] = 1.5
+    X = bf16_exact(np.stack([row, -row]))
+    codes, scales = B.bitnet_quant_states(dev_bf16(X), K, 3)
+    B.bitnet_sync_status()
+    c = oracle.unpack_bits(codes.cpu().numpy(), K, 3)
+    c_ref, d_ref, pre = oracle.quant_states(X, K, 3)
+    np.testing.assert_array_equal(c, c_ref)
+    assert (pre - np.floor(pre) == 0.5).sum() >= K
+    np.testing.assert_array_equal(scales.cpu().numpy(), d_ref)

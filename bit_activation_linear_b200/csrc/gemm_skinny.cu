@@ -13,12 +13,19 @@
 // product kernels.
 //
 // The packed weights never go through shared memory twice: TMA brings a stage of 128 features x
-// 512 weights (16 KB, 128-byte swizzle); each of four unpack warps turns its 32 rows into int8
-// lanes with one shift-and-mask per four weights (word g of a row holds k = 16g .. 16g+15; the
-// shift by 2p gives k = 16g+4p .. +3, which is exactly tensor-memory column 4g + p of that row) and
-// writes them straight into tensor memory with tcgen05.st, where the MMA reads its A operand
-// (tcgen05.mma ... [d], [a_tmem], b_desc).  Shared memory only holds the packed weights (read
-// once) and the tokens' codes (B operand, K-major, 128-byte swizzle).
+// 512 weights (16 KB, 128-byte swizzle); eight unpack warps (two per tensor-memory lane quadrant,
+// each taking half of the stage's K) turn their rows into int8 lanes with one shift-and-mask per
+// four weights (word g of a row holds k = 16g .. 16g+15; the shift by 2p gives k = 16g+4p .. +3,
+// which is exactly tensor-memory column 4g + p of that row) and write them straight into tensor
+// memory with tcgen05.st, where the MMA reads its A operand (tcgen05.mma ... [d], [a_tmem],
+// b_desc).  Shared memory only holds the packed weights (read once) and the tokens' codes (B
+// operand, K-major, 128-byte swizzle).
+//
+// With so few tokens each MMA holds little work (128 x MT x 32), and one thread issues an MMA only
+// every ~53 cycles on B200 whatever its size; with the operand A in tensor memory two issuing
+// threads double the rate (measured: 128 x 64 x 32 then runs at the tensor pipe's 32 cycles).  So
+// two MMA warps issue alternate halves of every stage into accumulators of their own, and the
+// epilogue adds the two.
 //
 // K split over a cluster: a feature block has KS = K / 512 stages; the S CTAs of a cluster (S <= 8,
 // chosen so that the grid fills the GPU) take consecutive chunks of them.  Each CTA copies its
@@ -28,10 +35,10 @@
 // the same fp32 operations as the other product kernels, so every path gives the same bits.
 // No global scratch is used: calls on different streams may run concurrently.
 //
-// Warp roles (256 threads): warps 0-3 unpack (warp w owns tensor-memory lanes 32w .. 32w+31, i.e.
-// features 32w ..), then run the epilogue; warp 4 issues the TMA loads; warp 5 allocates tensor
-// memory and (one thread) issues the MMAs; warps 6-7 widen INT4 codes to int8 in place (thread =
-// token row).  Every mbarrier wait is bounded: after ~1 s a role records BITNET_ERR_TIMEOUT and
+// Warp roles (416 threads): warps 0-7 unpack (warp w owns tensor-memory lanes 32(w%4) .. +31, i.e.
+// features 32(w%4) .., and half w/4 of each stage's K); warps 0-3 then run the epilogue; warp 8
+// issues the TMA loads; warps 9 and 10 each issue half of the MMAs (one thread each), warp 9 also
+// allocates tensor memory; warps 11-12 widen INT4 codes to int8 in place (thread = token row).  Every mbarrier wait is bounded: after ~1 s a role records BITNET_ERR_TIMEOUT and
 // stops, and every thread still meets the cluster barriers, so the kernel always returns.  No TMA
 // multicast is used.
 #include "common.cuh"
@@ -48,36 +55,43 @@ constexpr int UMMA_K = 32;                // K per kind::i8 MMA
 constexpr int WBYTES = FEAT * KST / 4;    // 16 KB of packed weights per stage
 constexpr int SUB = 128;                  // bytes of K per code sub-tile row (one swizzle row)
 constexpr int SUBS = KST / SUB;           // 4 code sub-tiles per stage
-constexpr int A_STAGES = 2;               // unpacked weight stages in tensor memory
+constexpr int A_STAGES = 3;               // unpacked weight stages in tensor memory
 constexpr int A_COLS = KST / 4;           // 128 columns of 4 int8 each per A stage
 constexpr int ACC_COL = A_STAGES * A_COLS;
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_THREADS = 256;
-constexpr int WARP_TMA = 4, WARP_MMA = 5, WARP_CODE = 6, CODE_WARPS = 2;
-constexpr int MAX_STAGES = 8;
+constexpr int UNPACK_WARPS = 8;           // two per lane quadrant, one per half of a stage's K
+constexpr int ISSUERS = 2;                // MMA-issuing warps, one per half, one accumulator each
+constexpr int W_STAGES = 8;               // packed-weight ring (HBM latency: ~2300 cycles)
+constexpr int WARP_WTMA = 8, WARP_MMA = 9, WARP_CTMA = 11, WARP_CODE = 12, CODE_WARPS = 2;
+constexpr int NUM_THREADS = (WARP_CODE + CODE_WARPS) * 32;
 
 template <int MT>
 struct Cfg {
-    static constexpr int CBYTES = MT * KST;                    // int8 codes per stage
-    static constexpr int STAGE_BYTES = WBYTES + CBYTES;
-    static constexpr int STAGES_FIT = (200 * 1024) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT < MAX_STAGES ? STAGES_FIT : MAX_STAGES;
+    static constexpr int CBYTES = MT * KST;                    // int8 codes of a stage
+    static constexpr int C_STAGES = MT >= 64 ? 3 : 4;          // code ring (L2 hits)
+    static constexpr int W_OFF = 0;
+    static constexpr int C_OFF = W_STAGES * WBYTES;
+    static constexpr int BAR_OFF = C_OFF + C_STAGES * CBYTES;
     static constexpr int RED_BYTES = MT * FEAT * 4;            // int32 partials [MT][FEAT]
-    static_assert(STAGES >= 2, "stages");
-    static_assert(RED_BYTES <= STAGES * STAGE_BYTES, "the partials reuse the stage memory");
-    static_assert(STAGE_BYTES % 1024 == 0 && (MT * SUB) % 1024 == 0, "swizzle-atom alignment");
-    static_assert(ACC_COL + MT <= TMEM_COLS, "tensor-memory budget");
+    static constexpr size_t SMEM = (size_t)BAR_OFF + 512 + 1024;  // + barriers + alignment
+    static_assert(RED_BYTES <= W_STAGES * WBYTES, "the partials reuse the weight ring");
+    static_assert(CBYTES % 1024 == 0 && (MT * SUB) % 1024 == 0, "swizzle-atom alignment");
+    static_assert(ACC_COL + ISSUERS * MT <= TMEM_COLS, "tensor-memory budget");
+    static_assert(SMEM <= 227 * 1024, "shared-memory budget");
 };
 
 struct __align__(8) Bars {
-    uint64_t full[MAX_STAGES];   // TMA bytes of the stage (weights and codes) have landed
-    uint64_t cfull[MAX_STAGES];  // INT4: the code warps have widened the stage's codes
-    uint64_t empty[MAX_STAGES];  // the stage's MMAs have completed (commit)
-    uint64_t a_full[A_STAGES];   // the four unpack warps have written the A stage
-    uint64_t a_empty[A_STAGES];  // the MMAs reading the A stage have completed (commit)
-    uint64_t acc_full;           // every MMA of this CTA has completed (commit)
+    uint64_t full_w[W_STAGES];           // TMA bytes of the weight slot have landed
+    uint64_t empty_w[W_STAGES];          // every unpack warp has read the weight slot
+    uint64_t full_c[4];                  // TMA bytes of the code slot have landed
+    uint64_t cfull[4];                   // INT4: the code warps have widened the slot's codes
+    uint64_t empty_c[4];                 // both issuers' MMAs reading the code slot have completed
+    uint64_t a_full[A_STAGES][ISSUERS];  // the four unpack warps of a half have written it
+    uint64_t a_empty[A_STAGES][ISSUERS]; // the MMAs of that half have completed (commit)
+    uint64_t acc_full;                   // every MMA of this CTA has completed (both issuers)
     uint32_t tmem_base;
 };
+static_assert(sizeof(Bars) <= 512, "barrier area");
 
 // Warp-uniform bounded wait (lane 0 polls; __syncwarp orders the other lanes after it).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int *status, int lane) {
@@ -106,7 +120,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Bars *bar = reinterpret_cast<Bars *>(smem + (size_t)C::STAGES * C::STAGE_BYTES);
+    uint8_t *wring = smem + C::W_OFF;
+    uint8_t *cring = smem + C::C_OFF;
+    Bars *bar = reinterpret_cast<Bars *>(smem + C::BAR_OFF);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -119,19 +135,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     constexpr uint32_t CB = BITS == 8 ? MT * KST : MT * KST / 2;  // code bytes a stage loads
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&bar->full[s], 1);
+        for (int s = 0; s < W_STAGES; ++s) {
+            mbar_init(&bar->full_w[s], 1);
+            mbar_init(&bar->empty_w[s], UNPACK_WARPS);
+        }
+        for (int s = 0; s < C::C_STAGES; ++s) {
+            mbar_init(&bar->full_c[s], 1);
             mbar_init(&bar->cfull[s], CODE_WARPS);
-            mbar_init(&bar->empty[s], 1);
+            mbar_init(&bar->empty_c[s], ISSUERS);
         }
-        for (int a = 0; a < A_STAGES; ++a) {
-            mbar_init(&bar->a_full[a], 4);
-            mbar_init(&bar->a_empty[a], 1);
-        }
-        mbar_init(&bar->acc_full, 1);
+        for (int a = 0; a < A_STAGES; ++a)
+            for (int h = 0; h < ISSUERS; ++h) {
+                mbar_init(&bar->a_full[a][h], UNPACK_WARPS / ISSUERS);
+                mbar_init(&bar->a_empty[a][h], 1);
+            }
+        mbar_init(&bar->acc_full, ISSUERS);
         fence_mbar_init();
     }
-    if (warp == WARP_TMA && lane == 0) {
+    if (warp == WARP_WTMA && lane == 0) {
         prefetch_tensormap(&tmap_w);
         prefetch_tensormap(&tmap_c);
     }
@@ -143,103 +164,128 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+    // the next kernel of the stream may be scheduled now; it waits for this grid's completion
+    // before it reads anything (griddepcontrol.wait)
+    pdl_launch_dependents();
 
-    if (warp == WARP_TMA) {
-        // ------------------------------------------------------------------ TMA producer
+    if (warp == WARP_WTMA) {
+        // ------------------------------------------------------------------ weight TMA
         if (lane == 0) {
-            // The packed weights of the first stages may be requested before the preceding kernel
-            // (the quantiser) has finished, when the caller guarantees they were complete before
-            // it started; every other global read waits for it (programmatic dependent launch).
-            const int pre = early_weights ? (nst < C::STAGES ? nst : C::STAGES) : 0;
-            for (int it = 0; it < pre; ++it) {
-                mbar_arrive_expect_tx(&bar->full[it], WBYTES + CB);
-                tma_load_2d(smem + (size_t)it * C::STAGE_BYTES, &tmap_w, (kb + it) * (KST / 4), n0,
-                            &bar->full[it]);
-            }
-            pdl_wait();
+            // With early_weights the caller guarantees the packed weights were complete before
+            // the preceding kernel (the quantiser) started, so they may be requested before that
+            // kernel finishes; otherwise every global read waits for it (programmatic dependent
+            // launch).
+            if (!early_weights) pdl_wait();
             uint32_t issued = 0, ph = 0;  // slots with a load issued, and that load's phase
             for (int it = 0; it < nst; ++it) {
-                const int s = it % C::STAGES;
-                const uint32_t p = (uint32_t)(it / C::STAGES) & 1;
-                uint8_t *st = smem + (size_t)s * C::STAGE_BYTES;
-                if (it >= pre) {
-                    if (!mbar_wait(&bar->empty[s], p ^ 1, status)) break;
-                    mbar_arrive_expect_tx(&bar->full[s], WBYTES + CB);
-                    tma_load_2d(st, &tmap_w, (kb + it) * (KST / 4), n0, &bar->full[s]);
-                }
+                const int s = it % W_STAGES;
+                const uint32_t p = (uint32_t)(it / W_STAGES) & 1;
+                if (!mbar_wait(&bar->empty_w[s], p ^ 1, status)) break;
+                mbar_arrive_expect_tx(&bar->full_w[s], WBYTES);
+                tma_load_2d(wring + (size_t)s * WBYTES, &tmap_w, (kb + it) * (KST / 4), n0,
+                            &bar->full_w[s]);
+                issued |= 1u << s;
+                ph = (ph & ~(1u << s)) | (p << s);
+            }
+            // no copy may still be landing in shared memory when the CTA moves on
+            for (int s = 0; s < W_STAGES; ++s)
+                if (issued & (1u << s)) mbar_wait(&bar->full_w[s], (ph >> s) & 1, status);
+        }
+        __syncwarp();
+    } else if (warp == WARP_CTMA) {
+        // ------------------------------------------------------------------ code TMA
+        if (lane == 0) {
+            pdl_wait();
+            uint32_t issued = 0, ph = 0;
+            for (int it = 0; it < nst; ++it) {
+                const int s = it % C::C_STAGES;
+                const uint32_t p = (uint32_t)(it / C::C_STAGES) & 1;
+                if (!mbar_wait(&bar->empty_c[s], p ^ 1, status)) break;
+                uint8_t *st = cring + (size_t)s * C::CBYTES;
+                mbar_arrive_expect_tx(&bar->full_c[s], CB);
                 const int kx = (kb + it) * KST;  // first weight of the stage
                 if constexpr (BITS == 8) {
 #pragma unroll
                     for (int j = 0; j < SUBS; ++j)
-                        tma_load_2d(st + WBYTES + j * MT * SUB, &tmap_c, kx + j * SUB, 0,
-                                    &bar->full[s]);
+                        tma_load_2d(st + j * MT * SUB, &tmap_c, kx + j * SUB, 0, &bar->full_c[s]);
                 } else {
                     // packed nibbles (256 B per token) into the last two sub-tiles; the code warps
                     // widen them in place
 #pragma unroll
                     for (int j = 0; j < 2; ++j)
-                        tma_load_2d(st + WBYTES + (2 + j) * MT * SUB, &tmap_c, kx / 2 + j * SUB, 0,
-                                    &bar->full[s]);
+                        tma_load_2d(st + (2 + j) * MT * SUB, &tmap_c, kx / 2 + j * SUB, 0,
+                                    &bar->full_c[s]);
                 }
                 issued |= 1u << s;
                 ph = (ph & ~(1u << s)) | (p << s);
             }
-            // no copy may still be landing in shared memory when the CTA moves on
-            for (int s = 0; s < C::STAGES; ++s)
-                if (issued & (1u << s)) mbar_wait(&bar->full[s], (ph >> s) & 1, status);
+            for (int s = 0; s < C::C_STAGES; ++s)
+                if (issued & (1u << s)) mbar_wait(&bar->full_c[s], (ph >> s) & 1, status);
         }
         __syncwarp();
-    } else if (warp == WARP_MMA) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
+        // ------------------------------------------------------------------ MMA issuers
+        // issuer i takes code sub-tiles 2i and 2i+1 of every stage (half i of its K, written by
+        // unpack warps 4i .. 4i+3) into accumulator i
         if (lane == 0) {
+            const int i = warp - WARP_MMA;
             constexpr uint32_t IDESC = idesc_i8_u8s8(FEAT, MT);
-            const uint32_t base = smem_addr(smem);
+            const uint32_t cbase = smem_addr(cring);
+            const uint32_t d_tmem = tmem + (uint32_t)(ACC_COL + i * MT);
             for (int it = 0; it < nst; ++it) {
-                const int s = it % C::STAGES, as = it % A_STAGES;
-                if (!mbar_wait(&bar->a_full[as], (uint32_t)(it / A_STAGES) & 1, status)) break;
-                if (!mbar_wait(BITS == 8 ? &bar->full[s] : &bar->cfull[s],
-                               (uint32_t)(it / C::STAGES) & 1, status))
+                const int cs = it % C::C_STAGES, as = it % A_STAGES;
+                if (!mbar_wait(&bar->a_full[as][i], (uint32_t)(it / A_STAGES) & 1, status)) break;
+                if (!mbar_wait(BITS == 8 ? &bar->full_c[cs] : &bar->cfull[cs],
+                               (uint32_t)(it / C::C_STAGES) & 1, status))
                     break;
                 tc_fence_after();
-                const uint32_t cst = base + (uint32_t)(s * C::STAGE_BYTES + WBYTES);
+                const uint32_t cst = cbase + (uint32_t)(cs * C::CBYTES);
 #pragma unroll
-                for (int j = 0; j < SUBS; ++j) {
+                for (int jj = 0; jj < SUBS / ISSUERS; ++jj) {
+                    const int j = i * (SUBS / ISSUERS) + jj;
                     const uint64_t bdesc = smem_desc_kmajor_sw128(cst + j * MT * SUB);
 #pragma unroll
                     for (int kk = 0; kk < SUB / UMMA_K; ++kk)
-                        mma_i8_ts(tmem + ACC_COL,
+                        mma_i8_ts(d_tmem,
                                   tmem + (uint32_t)(as * A_COLS + (j * (SUB / UMMA_K) + kk) * 8),
                                   bdesc + (uint64_t)(kk * UMMA_K / 16), IDESC,
-                                  (it | j | kk) != 0 ? 1u : 0u);
+                                  (it | jj | kk) != 0 ? 1u : 0u);
                 }
-                mma_commit(&bar->empty[s]);
-                mma_commit(&bar->a_empty[as]);
+                mma_commit(&bar->a_empty[as][i]);
+                mma_commit(&bar->empty_c[cs]);
             }
-            // arrives once every MMA issued above has completed (also after a time-out)
+            // arrives once every MMA this thread issued has completed (also after a time-out)
             mma_commit(&bar->acc_full);
         }
         __syncwarp();
     } else if (warp >= WARP_CODE) {
         // ------------------------------------------------------------------ INT4 code widening
         if constexpr (BITS == 4) {
-            // thread = token row: its 256 packed bytes (512 codes) sit in sub-tiles 2 and 3; it
-            // reads them all, then writes 512 int8 codes over the four sub-tiles of its row
+            // thread = token row: its 256 packed bytes (512 codes) sit in sub-tiles 2 and 3.  Half
+            // h2 reads packed sub-tile 2 + h2 (codes 256*h2 ..) whole, then writes its 256 int8
+            // codes over sub-tiles 2*h2 and 2*h2 + 1 of the row: half 0 writes sub-tiles 0-1 (no
+            // input there), half 1 overwrites sub-tile 2 (already read) and 3 (read just before)
             const int row = (warp - WARP_CODE) * 32 + lane;
             const int sx = row & 7;
             for (int it = 0; it < nst; ++it) {
-                const int s = it % C::STAGES;
-                if (!warp_wait(&bar->full[s], (uint32_t)(it / C::STAGES) & 1, status, lane)) break;
+                const int s = it % C::C_STAGES;
+                if (!warp_wait(&bar->full_c[s], (uint32_t)(it / C::C_STAGES) & 1, status, lane))
+                    break;
                 if (row < MT) {
-                    uint8_t *crow = smem + (size_t)s * C::STAGE_BYTES + WBYTES + row * SUB;
-                    uint4 raw[16];
+                    uint8_t *crow = cring + (size_t)s * C::CBYTES + row * SUB;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        raw[c] = *reinterpret_cast<const uint4 *>(
-                            crow + (2 + c / 8) * MT * SUB + (((c & 7) ^ sx) << 4));
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                    uint4 raw[8];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        // 32 codes k = 32c .. 32c+31 -> output chunks 2c (words x, y), 2c+1 (z, w)
-                        const uint32_t wd[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+                    for (int cc = 0; cc < 8; ++cc)
+                        raw[cc] = *reinterpret_cast<const uint4 *>(crow + (2 + h2) * MT * SUB +
+                                                                    ((cc ^ sx) << 4));
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        // 32 codes k = 32c .. 32c+31 (c = 8*h2 + cc) -> output chunks 2c (words
+                        // x, y) and 2c+1 (z, w)
+                        const int c = 8 * h2 + cc;
+                        const uint32_t wd[4] = {raw[cc].x, raw[cc].y, raw[cc].z, raw[cc].w};
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const uint32_t w0 = wd[2 * h], w1 = wd[2 * h + 1];
@@ -253,6 +299,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                                        (((oc & 7) ^ sx) << 4)) = o;
                         }
                     }
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -261,22 +308,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------------ weight unpack
-        const int r = warp * 32 + lane;  // feature row of the block = tensor-memory lane
-        const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+        const int quad = warp & 3, half = warp >> 2;
+        const int r = quad * 32 + lane;  // feature row of the block = tensor-memory lane
+        const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         for (int it = 0; it < nst; ++it) {
-            const int s = it % C::STAGES, as = it % A_STAGES;
-            if (!warp_wait(&bar->full[s], (uint32_t)(it / C::STAGES) & 1, status, lane)) break;
-            // row r of the weight tile: 128 B, 16-byte chunk c stored at chunk c ^ (r & 7)
-            const uint8_t *wrow = smem + (size_t)s * C::STAGE_BYTES + r * (KST / 4);
-            uint4 v[8];
+            const int s = it % W_STAGES, as = it % A_STAGES;
+            if (!warp_wait(&bar->full_w[s], (uint32_t)(it / W_STAGES) & 1, status, lane)) break;
+            // row r of the weight tile: 128 B, 16-byte chunk c stored at chunk c ^ (r & 7); this
+            // warp takes chunks 4*half .. 4*half+3 (k = 256*half .. +255)
+            const uint8_t *wrow = wring + (size_t)s * WBYTES + r * (KST / 4);
+            uint4 v[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                v[c] = *reinterpret_cast<const uint4 *>(wrow + ((c ^ (r & 7)) << 4));
-            if (!warp_wait(&bar->a_empty[as], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status, lane))
+            for (int c = 0; c < 4; ++c)
+                v[c] = *reinterpret_cast<const uint4 *>(wrow + (((4 * half + c) ^ (r & 7)) << 4));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar->empty_w[s]);  // the slot may be refilled
+            if (!warp_wait(&bar->a_empty[as][half], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status,
+                           lane))
                 break;
             tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {  // words 8q .. 8q+7 -> columns 32q .. 32q+31
+            for (int q = 0; q < 2; ++q) {  // words 8q .. 8q+7 of the half -> 32 columns
                 uint32_t o[32];
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
@@ -287,26 +339,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     o[4 * g + 2] = (w >> 4) & 0x03030303u;
                     o[4 * g + 3] = (w >> 6) & 0x03030303u;
                 }
-                tmem_st_32x32b_x32(t_lane + (uint32_t)(as * A_COLS + 32 * q), o);
+                tmem_st_32x32b_x32(t_lane + (uint32_t)(as * A_COLS + 64 * half + 32 * q), o);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar->a_full[as]);
+            if (lane == 0) mbar_arrive(&bar->a_full[as][half]);
         }
-        // ---- this CTA's partial sums: tensor memory -> shared memory [MT tokens][FEAT] ----
-        warp_wait(&bar->acc_full, 0, status, lane);
-        tc_fence_after();
-        int32_t *red = reinterpret_cast<int32_t *>(smem);  // every stage has been consumed
+        if (warp < 4) {
+            // ---- this CTA's partial sums (the two accumulators added): tensor memory ->
+            // shared memory [MT tokens][FEAT] ----
+            warp_wait(&bar->acc_full, 0, status, lane);
+            tc_fence_after();
+            // the weight ring has been consumed: every unpack warp has read every slot, and the
+            // MMAs that followed have completed
+            int32_t *red = reinterpret_cast<int32_t *>(wring);
 #pragma unroll
-        for (int q = 0; q < MT / 16; ++q) {
-            uint32_t v16[16];
-            tmem_ld_32x32b_x16(t_lane + (uint32_t)(ACC_COL + 16 * q), v16);
-            tmem_wait_ld();
+            for (int q = 0; q < MT / 16; ++q) {
+                uint32_t v0[16], v1[16];
+                tmem_ld_32x32b_x16(t_lane + (uint32_t)(ACC_COL + 16 * q), v0);
+                tmem_ld_32x32b_x16(t_lane + (uint32_t)(ACC_COL + MT + 16 * q), v1);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) red[(16 * q + j) * FEAT + r] = (int32_t)v16[j];
+                for (int j = 0; j < 16; ++j)
+                    red[(16 * q + j) * FEAT + r] = (int32_t)(v0[j] + v1[j]);
+            }
+            tc_fence_before();
         }
-        tc_fence_before();
     }
 
     // every CTA of the cluster has its partial sums in shared memory
@@ -318,7 +377,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // unit = (token m, 8 consecutive features); CTA `rank` takes every S-th group of 128
         pdl_wait();  // scales, code sums and Y belong to the stream order (returns at once here)
         const float gamma = *gamma_ptr;
-        const uint32_t red_addr = smem_addr(smem);
+        const uint32_t red_addr = smem_addr(wring);
         const int units = M * (FEAT / 8);
         for (int u = rank * 128 + (int)threadIdx.x; u < units; u += S * 128) {
             const int m = u / (FEAT / 8);
@@ -399,8 +458,7 @@ static cudaError_t configure(int dev) {
     if (done[dev]) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(ternary_gemm_skinny_kernel<BITS, MT, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(Cfg<MT>::STAGES * Cfg<MT>::STAGE_BYTES +
-                                               sizeof(Bars) + 1024));
+                                         (int)Cfg<MT>::SMEM);
     if (e == cudaSuccess) done[dev] = true;
     return e;
 }
@@ -418,7 +476,7 @@ static int max_clusters(int S) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(S * 16), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Cfg<64>::STAGES * Cfg<64>::STAGE_BYTES + sizeof(Bars) + 1024;
+    cfg.dynamicSmemBytes = Cfg<64>::SMEM;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)S;
@@ -459,7 +517,7 @@ static cudaError_t launch_skinny_t(const GemmArgs &a, const CUtensorMap &mw, con
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(blocks * S), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = Cfg<MT>::STAGES * Cfg<MT>::STAGE_BYTES + sizeof(Bars) + 1024;
+    cfg.dynamicSmemBytes = Cfg<MT>::SMEM;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -115,6 +115,10 @@ int act_quant_impl(DeviceState *st, const void *X, int64_t M, int64_t K, int had
             return fail(BITNET_ERR_UNSUPPORTED,
                         "H-BitLinear needs K to be a power of two in [128, 32768], got %lld",
                         (long long)K);
+        if (!nrm.on && hadamard_tc_supported(lk))
+            return launched(launch_hadamard_tc(X, M, lk, act_bits, codes, scales, rowsum, zout,
+                                               st->status_word, g_encode, st->num_sms, stream),
+                            1, "hadamard_tc");
         return launched(launch_fwht_quant(X, M, lk, act_bits, nrm, codes, scales, rowsum, zout,
                                           st->status_word, stream),
                         1, "fwht_quant");

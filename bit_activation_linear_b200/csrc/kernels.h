@@ -43,6 +43,15 @@ cudaError_t launch_fwht_quant(const void *X, int64_t M, int logk, int act_bits,
 // INT4 codes, layout as act_bits 4); the launchers reject it together with a norm or a z output.
 constexpr int kActInt4Absmax = 0x204;
 
+// The transform with its first seven butterfly levels as a tensor-core product (hadamard_tc.cu),
+// for K = 2^logk with hadamard_tc_supported(logk) and no norm: the same outputs as
+// launch_fwht_quant (codes, scales, rowsum; or z when zout != nullptr).  encode is
+// cuTensorMapEncodeTiled.
+bool hadamard_tc_supported(int logk);
+cudaError_t launch_hadamard_tc(const void *X, int64_t M, int logk, int act_bits, void *codes,
+                               float *scales, int32_t *rowsum, float *zout, int *status,
+                               void *encode_fn, int num_sms, cudaStream_t stream);
+
 // Quantise without a transform; K % 128 == 0.  zout != nullptr (with nrm.on) writes the
 // normalised rows in fp32 instead of codes.
 cudaError_t launch_act_quant_plain(const void *X, int64_t M, int64_t K, int act_bits,

@@ -44,13 +44,16 @@ def to_np_bits(t):
 
 
 def check_codes(codes_gpu, codes_ref, pre):
+    """Codes may differ by +-1 only within CODE_BOUNDARY of a .5 boundary, on at most a fraction
+    CODE_FRACTION of the elements: at most floor(CODE_FRACTION * n) of n codes, and at least one
+    allowed (below 10^4 codes a single near-tie flip already exceeds the rate)."""
     diff = codes_gpu.astype(np.int32) - codes_ref.astype(np.int32)
     bad = diff != 0
     if bad.any():
         assert np.abs(diff).max() <= 1
         dist = np.abs(np.abs(pre[bad] - np.floor(pre[bad])) - 0.5)
         assert np.all(dist < CODE_BOUNDARY), dist.max()
-        assert bad.mean() <= CODE_FRACTION
+        assert bad.sum() <= max(1, math.floor(CODE_FRACTION * bad.size)), bad.sum()
     return int(bad.sum())
 
 

@@ -46,6 +46,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
+# the activation quantiser's kernel, by the library's own plan query (bitnet_quant_path)
+QUANT_KERNEL = {1: "act_quant_plain", 2: "fwht_quant", 3: "hadamard_tc_quant"}
 METRIC = "H-BitLinear tokens/s and effective int8 TOPS (% of roofline) on 1 B200"
 
 
@@ -480,7 +482,7 @@ def run_gpu(args, wl, rank, world, device):
                 "us": 1e3 * phase_ms[0], "bound": "hbm", "bytes": w_bytes,
                 "achieved_gbs": w_bytes / (phase_ms[0] * 1e-3) / 1e9,
                 "frac": w_bytes / (phase_ms[0] * 1e-3) / 1e9 / hbm},
-            ("fwht_quant" if wl.hadamard else "act_quant_plain")
+            QUANT_KERNEL[B.bitnet_act_quant_plan(K, wl.hadamard, bool(args.rmsnorm))]
             + ("+rmsnorm" if args.rmsnorm else "") + ("+absmax4" if args.absmax4 else "")
             + " (alone, outside the timed steps)": {
                 "us": 1e3 * phase_ms[1], "bound": "hbm", "bytes": q_bytes,

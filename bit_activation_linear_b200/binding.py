@@ -22,6 +22,7 @@ _lib = None
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
 ACT_RELU2, ACT_SWIGLU = 1, 2  # bitnet_activation
 PATH_DECODE, PATH_TC, PATH_TC_SKINNY = 1, 2, 3  # bitnet_product_path
+QUANT_PLAIN, QUANT_FWHT, QUANT_HADAMARD_TC = 1, 2, 3  # bitnet_quant_path
 
 
 class BitnetError(RuntimeError):
@@ -63,6 +64,8 @@ _SIGS = {
     "bitnet_product_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                            ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                            ctypes.POINTER(ctypes.c_int)]),
+    "bitnet_act_quant_plan": (ctypes.c_int, [ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                             ctypes.POINTER(ctypes.c_int)]),
     "bitnet_bitlinear_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                                 ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
@@ -210,6 +213,14 @@ def bitnet_product_plan(M: int, K: int, N: int, act_bits: int):
     _rc(load_library().bitnet_product_plan(M, K, N, int(act_bits), ctypes.byref(path),
                                            ctypes.byref(split)), "bitnet_product_plan")
     return path.value, split.value
+
+
+def bitnet_act_quant_plan(K: int, hadamard: bool, norm: bool = False) -> int:
+    """Which kernel quantises a K-wide row (QUANT_* values); host only, no device needed."""
+    path = ctypes.c_int(0)
+    _rc(load_library().bitnet_act_quant_plan(K, int(bool(hadamard)), int(bool(norm)),
+                                             ctypes.byref(path)), "bitnet_act_quant_plan")
+    return path.value
 
 
 def bitnet_quantize_pack_weights(W: torch.Tensor, Wp: torch.Tensor | None = None,

@@ -216,6 +216,9 @@ __global__ void __launch_bounds__(P::THREADS, P::MIN_BLOCKS)
             a[c | m] = bfly_sub(x, y);
         }
     }
+    // the refill is an async-proxy write into the slot this thread has just read: a proxy fence
+    // orders the plain reads before it
+    fence_proxy_async_smem();
     team_sync<TEAM>(team);  // this slot is read and the previous row's tbuf reads are done
     issue(row + P::RING * stride, slot);  // refill the slot with the row after next
 

@@ -455,6 +455,23 @@ int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path
     return BITNET_OK;
 }
 
+int bitnet_act_quant_plan(int64_t K, int hadamard, int norm, int *path) {
+    int rc = check_shape(1, K, 8, false, false);
+    if (rc) return rc;
+    if (!path) return fail(BITNET_ERR_INVALID, "null pointer argument");
+    if (!hadamard) {
+        *path = BITNET_QUANT_PLAIN;
+        return BITNET_OK;
+    }
+    const int lk = log2_exact(K);
+    if (lk < 7 || lk > 15)
+        return fail(BITNET_ERR_UNSUPPORTED,
+                    "H-BitLinear needs K to be a power of two in [128, 32768], got %lld",
+                    (long long)K);
+    *path = !norm && hadamard_tc_supported(lk) ? BITNET_QUANT_HADAMARD_TC : BITNET_QUANT_FWHT;
+    return BITNET_OK;
+}
+
 size_t bitnet_workspace_bytes(int64_t M, int64_t K, int64_t N, int act_bits) {
     (void)N;
     if (M <= 0 || K <= 0) return 0;

@@ -321,6 +321,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 v[c] = *reinterpret_cast<const uint4 *>(wrow + (((4 * half + c) ^ (r & 7)) << 4));
+            // the refill is an async-proxy write: without a proxy fence after each lane's plain
+            // reads it may overtake them (measured on B200: rows of a slot read after the refill
+            // had begun landing)
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar->empty_w[s]);  // the slot may be refilled
             if (!warp_wait(&bar->a_empty[as][half], ((uint32_t)(it / A_STAGES) & 1) ^ 1, status,

@@ -199,6 +199,26 @@ typedef enum {
 int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path, int *k_split);
 
 /*
+ * Which kernel quantises the activations of a K-wide row (a query of the library, host only: it
+ * touches no device and enqueues nothing; the pages have no counterpart).  Every path gives the
+ * same codes up to the near-tie flips the activation entries document.
+ *   *path  BITNET_QUANT_PLAIN        per-token absmax / absmean rule on the raw row (hadamard 0);
+ *          BITNET_QUANT_FWHT         fast Walsh-Hadamard transform in registers, then the rule;
+ *          BITNET_QUANT_HADAMARD_TC  H_K = H_128 (x) H_(K/128) with the H_128 factor as bf16
+ *                                    tensor-core products (K = 8192 or 16384, no RMS norm).
+ * hadamard, norm: as the activation entries (norm != 0 for the bitnet_act_quant_norm family).
+ * Errors: BITNET_ERR_INVALID for K not a positive multiple of 128 or a null path,
+ * BITNET_ERR_UNSUPPORTED for hadamard != 0 with K not a power of two in [128, 32768].
+ */
+typedef enum {
+    BITNET_QUANT_PLAIN = 1,
+    BITNET_QUANT_FWHT = 2,
+    BITNET_QUANT_HADAMARD_TC = 3
+} bitnet_quant_path;
+
+int bitnet_act_quant_plan(int64_t K, int hadamard, int norm, int *path);
+
+/*
  * Activations fused into the product's epilogue, for the up / gate projections that feed the
  * FFN (BitNet b1.58 2B4T article, section 一.3: squared ReLU; BitNet v2 write-up: SwishGLU).
  * With y = float(acc) * (scales[m] * gamma) as in bitnet_ternary_gemm:

@@ -181,3 +181,20 @@ def test_state_quant_size_and_rejections_before_the_device(lib):
     assert lib.bitnet_quant_states(None, 4, 4096, 128, 3, p, p, None) == -1  # null X
     q = ctypes.c_void_p(20)
     assert lib.bitnet_quant_states(q, 4, 4096, 128, 3, p, p, None) == -1    # misaligned
+
+
+def test_act_quant_plan_host_only():
+    """The quantiser plan is a host query: it needs no device and names the kernel each case
+    takes (the tensor-core Hadamard only for K = 8192 / 16384 without the RMS norm)."""
+    from bit_activation_linear_b200 import binding as B
+    assert B.bitnet_act_quant_plan(4096, False) == B.QUANT_PLAIN
+    assert B.bitnet_act_quant_plan(2048, True) == B.QUANT_FWHT
+    assert B.bitnet_act_quant_plan(8192, True) == B.QUANT_HADAMARD_TC
+    assert B.bitnet_act_quant_plan(16384, True) == B.QUANT_HADAMARD_TC
+    assert B.bitnet_act_quant_plan(16384, True, norm=True) == B.QUANT_FWHT
+    assert B.bitnet_act_quant_plan(32768, True) == B.QUANT_FWHT
+    lib = B.load_library()
+    out = ctypes.c_int(0)
+    assert lib.bitnet_act_quant_plan(3 * 128, 1, 0, ctypes.byref(out)) == -2   # not 2^k
+    assert lib.bitnet_act_quant_plan(100, 0, 0, ctypes.byref(out)) == -1       # K % 128
+    assert lib.bitnet_act_quant_plan(4096, 1, 0, None) == -1                   # null path

@@ -46,6 +46,9 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense ratio on B200: 4.5 POPS int8 vs 2.25 PFLOP/s bf16
+# the product's kernel by the library's plan query (bitnet_product_path), for M > 8
+PRODUCT_KERNEL = {1: "ternary_gemv", 2: "ternary_gemm_tc", 3: "ternary_gemm_skinny",
+                  4: "ternary_gemm_pair_ts"}
 # the activation quantiser's kernel, by the library's own plan query (bitnet_quant_path)
 QUANT_KERNEL = {1: "act_quant_plain", 2: "fwht_quant", 3: "hadamard_tc_quant"}
 METRIC = "H-BitLinear tokens/s and effective int8 TOPS (% of roofline) on 1 B200"
@@ -491,21 +494,25 @@ def run_gpu(args, wl, rank, world, device):
         }
         prod_bytes = work["ternary_gemm_tc"]["bytes"]
         prod_gbs = prod_bytes / (gemm_ms * 1e-3) / 1e9
-        if M > 8:
-            per_kernel["ternary_gemm_tc"] = {
+        # the product kernel the library's plan query names for this shape
+        path = B.bitnet_product_plan(M, K, N, wl.act_bits)[0]
+        if path in (B.PATH_TC, B.PATH_TC_TMEM):
+            tc_name = PRODUCT_KERNEL[path]
+            per_kernel[tc_name] = {
                 "us": 1e3 * gemm_ms, "bound": "tensor", "ops": work["ternary_gemm_tc"]["ops"],
                 "achieved_tops": achieved, "frac": achieved / int8_peak}
-            roofline = {"kernel": "ternary_gemm_tc", "bound": "tensor",
+            roofline = {"kernel": tc_name, "bound": "tensor",
                         "achieved": achieved, "peak": int8_peak, "unit": "TOPS",
                         "frac": achieved / int8_peak,
-                        "traffic": ncu_traffic("ternary_gemm_tc_kernel", wl.name),
+                        "traffic": ncu_traffic(tc_name + "_kernel", wl.name),
                         "ms_per_launch": gemm_ms,
                         "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x "
                                        f"{INT8_PER_BF16} (nominal int8:bf16 dense ratio)"}
         else:
             # a few tokens: the product streams the stored weights once (bytes = weights +
             # codes + bf16 Y), so HBM bounds it
-            gemv = "ternary_gemv_base3" if args.base3 else "ternary_gemv"
+            gemv = ("ternary_gemv_base3" if args.base3 else
+                    PRODUCT_KERNEL.get(path, "ternary_gemv"))
             per_kernel[gemv] = {
                 "us": 1e3 * gemm_ms, "bound": "hbm", "bytes": prod_bytes,
                 "achieved_gbs": prod_gbs, "frac": prod_gbs / hbm,

@@ -21,7 +21,7 @@ _lib = None
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
 ACT_RELU2, ACT_SWIGLU = 1, 2  # bitnet_activation
-PATH_DECODE, PATH_TC, PATH_TC_SKINNY = 1, 2, 3  # bitnet_product_path
+PATH_DECODE, PATH_TC, PATH_TC_SKINNY, PATH_TC_TMEM = 1, 2, 3, 4  # bitnet_product_path
 QUANT_PLAIN, QUANT_FWHT, QUANT_HADAMARD_TC = 1, 2, 3  # bitnet_quant_path
 
 

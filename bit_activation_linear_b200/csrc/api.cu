@@ -151,6 +151,12 @@ int gemm_impl(DeviceState *st, const void *codes, const float *scales, const int
     if (M <= kSkinnyMaxTokens)
         return launched(launch_ternary_gemm_skinny(a, g_encode, stream), 1, "ternary_gemm_skinny");
     int n = 0;
+    if (use_pair_ts(act_bits, K)) {
+        // INT4 codes are widened on chip; with the weights unpacked into tensor memory that
+        // widening no longer shares shared memory with the unpacked weights
+        const cudaError_t e = launch_ternary_gemm_pair_ts(a, g_encode, st->num_sms, stream, &n);
+        return launched(e, n, "ternary_gemm_pair_ts");
+    }
     const cudaError_t e = launch_ternary_gemm_tc(a, g_encode, st->num_sms, stream, &n);
     return launched(e, n, "ternary_gemm_tc");
 }
@@ -450,7 +456,7 @@ int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path
         *k_split = ternary_gemm_skinny_split(N, K);
         return BITNET_OK;
     }
-    *path = BITNET_PATH_TC;
+    *path = use_pair_ts(act_bits, K) ? BITNET_PATH_TC_TMEM : BITNET_PATH_TC;
     *k_split = 1;
     return BITNET_OK;
 }

@@ -92,6 +92,16 @@ cudaError_t launch_ternary_gemv_base3(const GemmArgs &a, cudaStream_t stream);
 cudaError_t launch_ternary_gemm_tc(const GemmArgs &a, void *encode_fn, int num_sms,
                                    cudaStream_t stream, int *launches = nullptr);
 
+// tcgen05 tensor-core kernel (prefill) on CTA pairs with the unpacked weights in tensor memory
+// (operand A) and 256-feature x 192-token tiles (gemm_pair_ts.cu).
+cudaError_t launch_ternary_gemm_pair_ts(const GemmArgs &a, void *encode_fn, int num_sms,
+                                        cudaStream_t stream, int *launches = nullptr);
+// The product of INT4 codes with K >= kPairTsMinK takes it: its single accumulator makes a
+// tile's MMAs wait for the previous tile's epilogue, which short K axes cannot hide (measured on
+// B200: slower than the shared-memory kernel at K <= 4096, faster from K = 8192).
+constexpr int64_t kPairTsMinK = 8192;
+inline bool use_pair_ts(int act_bits, int64_t K) { return act_bits == 4 && K >= kPairTsMinK; }
+
 // tcgen05 tensor-core kernel for kGemvMaxTokens < M <= kSkinnyMaxTokens: weights on the MMA's M
 // side, streamed once, K split over a cluster (gemm_skinny.cu).  One launch.
 constexpr int kSkinnyMaxTokens = 64;

@@ -184,7 +184,12 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
  * Which kernel the product of an M x K by N x K shape takes on the current device (a query of
  * the library; the pages have no counterpart).  Every path gives the same integers.
  *   *path    BITNET_PATH_DECODE    weight-streaming kernel on the CUDA cores (M <= 8 tokens);
- *            BITNET_PATH_TC        tensor-core kernel, one pass over K per 256 x 256 tile;
+ *            BITNET_PATH_TC        tensor-core kernel (M > 64; INT8, or INT4 with K < 8192),
+ *                                  one pass over K per 256 x 256 tile, both operands in shared
+ *                                  memory;
+ *            BITNET_PATH_TC_TMEM   tensor-core kernel (M > 64, INT4, K >= 8192), one pass over K
+ *                                  per 256-feature x 256-token tile, the unpacked weights in
+ *                                  tensor memory (the MMA's A operand);
  *            BITNET_PATH_TC_SKINNY tensor-core kernel for 9 <= M <= 64: 128 output features per
  *                                  CTA, K cut into *k_split chunks over a cluster of CTAs.
  *   *k_split chunks of K per output feature block (1 unless BITNET_PATH_TC_SKINNY).
@@ -193,7 +198,8 @@ int bitnet_ternary_gemm(const void *codes_dev, const float *scales_dev,
 typedef enum {
     BITNET_PATH_DECODE = 1,
     BITNET_PATH_TC = 2,
-    BITNET_PATH_TC_SKINNY = 3
+    BITNET_PATH_TC_SKINNY = 3,
+    BITNET_PATH_TC_TMEM = 4
 } bitnet_product_path;
 
 int bitnet_product_plan(int64_t M, int64_t K, int64_t N, int act_bits, int *path, int *k_split);

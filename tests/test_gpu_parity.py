@@ -168,6 +168,7 @@ def staged_product(B, M, K, N, bits, seed):
     (130, 384, 136), (300, 2048, 264),                      # 256 x 256 tiles, ragged
     (256, 1024, 1024), (513, 128, 8),
     (1000, 640, 520),                                       # several tiles, 2.5 K stages
+    (65, 8192, 8), (700, 8448, 264),                        # INT4: tensor-memory kernel
 ])
 @pytest.mark.parametrize("bits", [8, 4])
 def test_product_int32_exact_and_bf16(B, M, K, N, bits):
@@ -221,6 +222,11 @@ def test_product_paths_by_token_count(B):
     for M, path in ((1, B.PATH_DECODE), (8, B.PATH_DECODE), (9, B.PATH_TC_SKINNY),
                     (64, B.PATH_TC_SKINNY), (65, B.PATH_TC), (4096, B.PATH_TC)):
         assert B.bitnet_product_plan(M, 2048, 2048, 8)[0] == path, M
+    for M, path in ((8, B.PATH_DECODE), (64, B.PATH_TC_SKINNY), (65, B.PATH_TC_TMEM),
+                    (16384, B.PATH_TC_TMEM)):
+        assert B.bitnet_product_plan(M, 8192, 2048, 4)[0] == path, M
+    # INT4 below K = 8192 stays on the shared-memory kernel
+    assert B.bitnet_product_plan(4096, 4096, 2048, 4)[0] == B.PATH_TC
 
 
 def test_concurrent_forwards_on_two_streams(B):
@@ -260,10 +266,12 @@ def test_concurrent_forwards_on_two_streams(B):
     (16384, 16384, 4096, 4, "down_7b"),
     (4000, 2048, 2056, 8, None),
     (3000, 1152, 3080, 4, None),
+    (3000, 8320, 3080, 4, None),   # tensor-memory kernel: ragged M and N, half last stage
 ])
 def test_product_one_pass_full_size_bit_exact(B, M, K, N, bits, name):
     path, split = B.bitnet_product_plan(M, K, N, bits)
-    assert (path, split) == (B.PATH_TC, 1), "this shape must take the one-pass kernel"
+    expect = B.PATH_TC_TMEM if bits == 4 and K >= 8192 else B.PATH_TC
+    assert (path, split) == (expect, 1), "this shape must take the one-pass kernel"
     if name is not None:
         wl = synth.WORKLOADS[name]
         X, W = wl.activations(seed=3), wl.weights(seed=3)

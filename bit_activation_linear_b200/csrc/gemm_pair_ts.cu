@@ -27,7 +27,12 @@
 // accumulator out (eight epilogue warps, each 128 tokens of one lane quadrant, release it after
 // their last tcgen05.ld); two accumulators would leave no columns for the A stages, and
 // 192-token tiles with two accumulators measured slower: the issuing thread pays the same
-// ~50 cycles for a 256 x 192 x 32 MMA as for a 256 x 256 x 32 one.
+// ~50 cycles for a 256 x 192 x 32 MMA as for a 256 x 256 x 32 one.  Measured with clock64
+// stamps on B200 (7B down projection): a steady 256-deep stage takes ~1500 cycles with the
+// operands ready (~90 cycles of barrier tests per stage); the epilogue holds the accumulator
+// ~7700 cycles per tile of ~96000.  Each epilogue warp keeps its tokens' (d_m * gamma, sum_k c)
+// in a shared-memory table filled while the tile's MMAs run, read by broadcast (two shuffles
+// per element before: ~10200 cycles).
 //
 // Warp roles (per CTA):
 //   warp 0       code TMA: two [128 tokens x 128 B] boxes per 256-deep stage (INT8; the pair form
@@ -103,7 +108,9 @@ struct __align__(8) Barriers {
 // even CTA's offsets).
 constexpr size_t OFF_C = 0;
 constexpr size_t OFF_W = OFF_C + (size_t)C_STAGES * C_STAGE_BYTES;
-constexpr size_t OFF_BAR = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
+// per epilogue warp: (d_m * gamma, sum_k c) of its 128 tokens of the current tile
+constexpr size_t OFF_TOK = OFF_W + (size_t)W_STAGES * W_STAGE_BYTES;
+constexpr size_t OFF_BAR = OFF_TOK + (size_t)EPI_WARPS * (BT / 2) * 8;
 constexpr size_t SMEM_BYTES = OFF_BAR + sizeof(Barriers) + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared-memory budget");
 
@@ -335,10 +342,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<BITS>(),
         const uint32_t t_lane = tmem + ((uint32_t)(quad * 32) << 16);
         const float gamma = *gamma_ptr;
         constexpr int CHUNKS = BT / 2 / 32;
+        float2 *tok = reinterpret_cast<float2 *>(smem + OFF_TOK) + (warp - WARP_EPI) * (BT / 2);
         for (int t = 0; t < my_tiles; ++t) {
             const int tile = pair + t * npairs;
             const int nf = tile % n_ftiles, mt = tile / n_ftiles;
             const int n = nf * BF + (int)rank * HF + quad * 32 + lane;  // this thread's feature
+            // the warp's token table, filled while the tile's MMAs run: every element then reads
+            // its token's scale and code sum with one broadcast shared-memory load
+            __syncwarp();  // the previous tile's reads of the table are done
+#pragma unroll
+            for (int q = 0; q < CHUNKS; ++q) {
+                const int mj = mt * BT + eh * (BT / 2) + q * 32 + lane;
+                tok[q * 32 + lane] = make_float2(mj < M ? scales[mj] * gamma : 0.f,
+                                                 __int_as_float(mj < M ? rowsum[mj] : 0));
+            }
+            __syncwarp();
             if (!warp_wait(&bar->acc_full, (uint32_t)t & 1, status, lane)) break;
             tc_fence_after();
 #pragma unroll 1
@@ -346,10 +364,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<BITS>(),
                 const int m0 = mt * BT + eh * (BT / 2) + ch * 32;  // first token of the chunk
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(t_lane + (uint32_t)(ACC_COL + eh * (BT / 2) + ch * 32), v);
-                // lane j fetches token m0 + j's scale and code sum, broadcast below
-                const int mj = m0 + lane;
-                const float sc_j = mj < M ? scales[mj] * gamma : 0.f;
-                const int rs_j = mj < M ? rowsum[mj] : 0;
                 tmem_wait_ld();
                 if (ch == CHUNKS - 1) {
                     // the accumulator is read out: the next tile's MMAs may start
@@ -361,8 +375,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<BITS>(),
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int m = m0 + j;
-                    const float sc = __shfl_sync(0xFFFFFFFFu, sc_j, j);
-                    const int rs = __shfl_sync(0xFFFFFFFFu, rs_j, j);
+                    const float2 tk = tok[ch * 32 + j];
+                    const float sc = tk.x;
+                    const int rs = __float_as_int(tk.y);
                     const int a = (int)v[j] - rs;
                     if constexpr (MODE == OUT_ACC) {
                         if (m < M && n < N) reinterpret_cast<int32_t *>(Yout)[(int64_t)m * N + n] = a;

@@ -26,6 +26,13 @@ namespace bitnet {
 
 constexpr int kGemvWarps = 4;  // warps per CTA
 
+// d = c + sum_j a.u8[j] * b.s8[j]: unsigned bytes of a against signed bytes of b
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // Reduce the lanes' partial sums (shuffles), then the KS warps' partial sums of the row group
 // (shared memory, one barrier for the whole CTA), remove the weight offset with the code sums and
 // write the results from the group's first warp: lane r*T + t stores (row n0 + r, token t).
@@ -134,8 +141,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < T; ++t) acc[r][t] = 0;
+    // With few (row, token) pairs, each 2-bit field p of a word is masked in place instead of
+    // shifted down: byte j of w & (0x03030303 << 2p) holds 4^p u, so its dot product is 4^p
+    // times the field's, kept in a sum of its own and scaled back (an exact shift: every term is
+    // a multiple of 4^p) once per batch of S steps: a batch adds S * 4 terms of at most
+    // 64 * 2 * 128 in magnitude to a field sum, far below 2^31.
+    // One mask instead of a shift and a mask per field and dot product.
+    constexpr bool FIELD_SUMS = R * T <= 4;
+    int fs[FIELD_SUMS ? R : 1][FIELD_SUMS ? T : 1][4];
 
     for (int b0 = 0; b0 < mine; b0 += S) {
+        if constexpr (FIELD_SUMS) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) fs[r][t][p] = 0;
+        }
         uint32_t w[R][S];
 #pragma unroll
         for (int j = 0; j < S; ++j) {
@@ -180,10 +203,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
             for (int r = 0; r < R; ++r)
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const int u = (int)((w[r][j] >> (2 * p)) & 0x03030303u);
+                    if constexpr (FIELD_SUMS) {
+                        const uint32_t um = w[r][j] & (0x03030303u << (2 * p));
 #pragma unroll
-                    for (int t = 0; t < T; ++t) acc[r][t] = __dp4a(u, (int)xs[t][p], acc[r][t]);
+                        for (int t = 0; t < T; ++t) fs[r][t][p] = dp4a_us(um, xs[t][p], fs[r][t][p]);
+                    } else {
+                        const int u = (int)((w[r][j] >> (2 * p)) & 0x03030303u);
+#pragma unroll
+                        for (int t = 0; t < T; ++t) acc[r][t] = __dp4a(u, (int)xs[t][p], acc[r][t]);
+                    }
                 }
+        }
+        if constexpr (FIELD_SUMS) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+                    acc[r][t] += fs[r][t][0] + (fs[r][t][1] >> 2) + (fs[r][t][2] >> 4) +
+                                 (fs[r][t][3] >> 6);
         }
     }
     // the scales and code sums are read below: make sure this warp has waited
@@ -290,8 +327,24 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < T; ++t) acc[r][t] = 0;
+    // With few (row, token) pairs, each 2-bit field p of a word is masked in place instead of
+    // shifted down: byte j of w & (0x03030303 << 2p) holds 4^p u, so its dot product is 4^p
+    // times the field's, kept in a sum of its own and scaled back (an exact shift: every term is
+    // a multiple of 4^p) once per batch of S steps: a batch adds S * 4 terms of at most
+    // 64 * 2 * 128 in magnitude to a field sum, far below 2^31.
+    // One mask instead of a shift and a mask per field and dot product.
+    constexpr bool FIELD_SUMS = R * T <= 4;
+    int fs[FIELD_SUMS ? R : 1][FIELD_SUMS ? T : 1][4];
 
     for (int b0 = 0; b0 < mine; b0 += S) {
+        if constexpr (FIELD_SUMS) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) fs[r][t][p] = 0;
+        }
         uint32_t w[R][S];
 #pragma unroll
         for (int j = 0; j < S; ++j) {

@@ -30,9 +30,11 @@
 // ~50 cycles for a 256 x 192 x 32 MMA as for a 256 x 256 x 32 one.  Measured with clock64
 // stamps on B200 (7B down projection): a steady 256-deep stage takes ~1500 cycles with the
 // operands ready (~90 cycles of barrier tests per stage); the epilogue holds the accumulator
-// ~7700 cycles per tile of ~96000.  Each epilogue warp keeps its tokens' (d_m * gamma, sum_k c)
-// in a shared-memory table filled while the tile's MMAs run, read by broadcast (two shuffles
-// per element before: ~10200 cycles).
+// ~5400 cycles per tile of ~96000.  What it took to get there: each epilogue warp keeps its
+// tokens' (d_m * gamma, sum_k c) in a shared-memory table filled while the tile's MMAs run, read
+// by broadcast (two shuffles per element before: ~10200 cycles), and the int -> fp32 and
+// fp32 -> bf16 conversions, whose unit was the limit, are done on the FMA pipe and two at a time
+// (~7700 cycles before).
 //
 // Warp roles (per CTA):
 //   warp 0       code TMA: two [128 tokens x 128 B] boxes per 256-deep stage (INT8; the pair form
@@ -343,6 +345,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<BITS>(),
         const float gamma = *gamma_ptr;
         constexpr int CHUNKS = BT / 2 / 32;
         float2 *tok = reinterpret_cast<float2 *>(smem + OFF_TOK) + (warp - WARP_EPI) * (BT / 2);
+        // |sum_k q c| <= 128 K (INT8) or 8 K (INT4): below 2^22 the exact FMA-pipe conversion
+        // applies (always for the shapes this kernel takes)
+        const bool small_acc = (int64_t)K * (BITS == 8 ? 128 : 8) < (int64_t(1) << 22);
         for (int t = 0; t < my_tiles; ++t) {
             const int tile = pair + t * npairs;
             const int nf = tile % n_ftiles, mt = tile / n_ftiles;
@@ -372,30 +377,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(num_threads<BITS>(),
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_addr(&bar->acc_empty), 0));
                 }
                 if (m0 >= M) continue;
+                if constexpr (MODE == OUT_ACC) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int m = m0 + j;
-                    const float2 tk = tok[ch * 32 + j];
-                    const float sc = tk.x;
-                    const int rs = __float_as_int(tk.y);
-                    const int a = (int)v[j] - rs;
-                    if constexpr (MODE == OUT_ACC) {
+                    for (int j = 0; j < 32; ++j) {
+                        const int m = m0 + j;
+                        const int a = (int)v[j] - __float_as_int(tok[ch * 32 + j].y);
                         if (m < M && n < N) reinterpret_cast<int32_t *>(Yout)[(int64_t)m * N + n] = a;
-                    } else if constexpr (MODE == OUT_SWIGLU) {
-                        // features 2i (gate) and 2i + 1 (up) sit in lanes 2i, 2i + 1
-                        const float y = (float)a * sc;
-                        const float up = __shfl_xor_sync(0xFFFFFFFFu, y, 1);
-                        if ((lane & 1) == 0 && m < M && n < N) {
-                            const float o = __fdiv_rn(y, 1.f + expf(-y)) * up;
-                            reinterpret_cast<__nv_bfloat16 *>(Yout)[(int64_t)m * (N / 2) + n / 2] =
-                                __float2bfloat16_rn(o);
+                    }
+                } else {
+                    // The conversion unit (~16 per clock per SM on B200) set the epilogue's pace
+                    // with an int -> fp32 and an fp32 -> bf16 conversion per element: the first
+                    // is done exactly on the FMA pipe (|a| < 2^22: the fp32 with bit pattern
+                    // 0x4B400000 + a is 1.5 * 2^23 + a), the second two tokens at a time.
+                    const bool glu = MODE == OUT_SWIGLU;
+                    const bool store = glu ? (lane & 1) == 0 && n < N : n < N;
+                    const int64_t ld = glu ? N / 2 : N;
+                    unsigned short *yp = reinterpret_cast<unsigned short *>(Yout) +
+                                         (int64_t)m0 * ld + (glu ? n / 2 : n);
+                    const int rows = store ? min(M - m0, 32) : 0;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float y[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float2 tk = tok[ch * 32 + j + e];
+                            const int a = (int)v[j + e] - __float_as_int(tk.y);
+                            const float af = small_acc ? __fsub_rn(__int_as_float(0x4B400000 + a), 12582912.f)
+                                                       : (float)a;
+                            y[e] = af * tk.x;
+                            if constexpr (MODE == OUT_RELU2) y[e] = y[e] > 0.f ? y[e] * y[e] : 0.f;
+                            if constexpr (MODE == OUT_SWIGLU) {
+                                // features 2p (gate) and 2p + 1 (up) sit in lanes 2p, 2p + 1; the
+                                // even lane keeps silu(gate) * up
+                                const float up = __shfl_xor_sync(0xFFFFFFFFu, y[e], 1);
+                                y[e] = __fdiv_rn(y[e], 1.f + expf(-y[e])) * up;
+                            }
                         }
-                    } else {
-                        float y = (float)a * sc;
-                        if constexpr (MODE == OUT_RELU2) y = y > 0.f ? y * y : 0.f;
-                        if (m < M && n < N)
-                            reinterpret_cast<__nv_bfloat16 *>(Yout)[(int64_t)m * N + n] =
-                                __float2bfloat16_rn(y);
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(y[0], y[1]);
+                        const uint32_t hw = *reinterpret_cast<const uint32_t *>(&h);
+                        if (j < rows) *yp = (unsigned short)(hw & 0xFFFFu);
+                        yp += ld;
+                        if (j + 1 < rows) *yp = (unsigned short)(hw >> 16);
+                        yp += ld;
                     }
                 }
             }

@@ -664,6 +664,7 @@ def check_act(Y, y_ref_bits):
     (8, 2048, 8192),                                            # decode, 4-row groups
     (9, 256, 256), (32, 8192, 2064), (64, 2048, 8192),          # skinny tensor-core kernel
     (300, 2048, 272), (1000, 640, 528),                         # 256 x 256 tiles
+    (300, 8192, 528),                                           # INT4: tensor-memory kernel
 ])
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("act", [1, 2])

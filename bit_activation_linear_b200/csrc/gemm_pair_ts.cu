@@ -47,9 +47,9 @@
 //   warps 4-7    unpack: warp w owns tensor-memory lanes 32(w%4) .. +31 (features): 64 packed
 //                bytes -> 64 columns of int8 lanes with one shift-and-mask per four weights,
 //                tcgen05.st into the A stage;
-//   warps 8-15   epilogue: thread = feature, tokens 128 ((w-8)/4) .. +127 of the tile, 32 at a
-//                time: tcgen05.ld, offset, scale, activation, stores (a warp store covers 32
-//                consecutive features of one token);
+//   warps 8-15   epilogue: thread = feature, tokens 128 ((w-8)/4) .. +127 of the tile, read 64
+//                at a time (tcgen05.ld), then offset, scale, activation and stores 32 at a time
+//                (a warp store covers 32 consecutive features of one token);
 //   warps 16-19  INT4 only: widen the stage's packed codes in place, thread = token row.
 // Every mbarrier wait is bounded (~1 s, then BITNET_ERR_TIMEOUT and the kernel winds down).  No
 // TMA multicast is used.
